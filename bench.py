@@ -1,0 +1,430 @@
+#!/usr/bin/env python3
+"""Benchmark of the W4A8 MXFP4 MoE decode step on B200.
+
+Workload: the Ling-shaped MoE layer at M=1 token (H=2560, I=768, E=256
+experts, top-8; MXFP4 expert weights, FP8 E4M3 activations; softmax router
+with the 8th/9th logit gap forced >= 1e-3). Inputs are synthetic and seeded.
+
+The timed unit is one layer-step: the whole hot path (quantise, route, top-k,
+union, gate/up + SwiGLU, down, combine). To keep the 126 MB L2 from serving
+the weights, each layer-step reads a different layer of a 32-layer pool
+(32 x 256 experts = 25.7 GB of MXFP4 weights), with the same x. One bench
+"step" is one pass over the pool: 32 layer-steps, captured in one CUDA graph
+and replayed.
+
+Output: one JSON line from rank 0. `value` is tokens per second summed over
+all ranks, where a token-step is M tokens through one layer-step. The line
+also reports us/layer-step, expert-weight GB/s, the roofline of the kernel,
+the CPU oracle baseline, an end-to-end number through the public API with
+host buffers, and the SM clocks sampled during the timed region.
+
+--impl reference times the CPU oracle (test infrastructure) on a bounded
+sample of the same workload and prints the same metric.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MXFP4 MoE decode µs/layer-step, tokens/s; HBM GB/s as % of B200 peak"
+H, I, E, K = 2560, 768, 256, 8
+POOL_LAYERS = 32
+SEED = 0
+
+
+def expert_bytes(h=H, i=I):
+    return 2 * i * h // 2 + 2 * i * h // 32 + h * i // 2 + h * i // 32
+
+
+def algorithmic_bytes(M, U, h=H, i=I, e=E):
+    """Bytes a layer-step must move: active expert weights, router, x, y."""
+    return U * expert_bytes(h, i) + e * h * 4 + 2 * M * h * 2
+
+
+def load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            pk = json.load(f)
+        return float(pk["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "mxfp4_weight_streaming_fp8_b200", "csrc")
+    for fn in sorted(os.listdir(csrc)):
+        if fn.endswith((".cu", ".cuh", ".h")):
+            h.update(open(os.path.join(csrc, fn), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        rec = json.load(open(path))[kernel][workload]
+    except Exception:
+        return None
+    if rec.get("source_hash") != kernel_source_hash():
+        return None
+    return rec.get("bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ distributed
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def max_over_ranks(value: float, ws: int, device=None) -> float:
+    """Max of a per-rank float over all ranks (identity at world size 1)."""
+    if ws == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(value: float, ws: int, device=None) -> float:
+    if ws == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ workload
+def build_pool(device, M, mode, layers=POOL_LAYERS, seed=SEED):
+    import torch
+    from mxfp4_weight_streaming_fp8_b200 import moe, synth
+    x = synth.gen_x(seed, M, H)
+    ctxs, weights = [], []
+    for l in range(layers):
+        wr = synth.force_router(x, synth.gen_router(seed, l, E, H), K, mode, seed=seed, layer=l)
+        ex = synth.layer_experts_torch(seed, l, E, H, I, device)
+        wr_d = torch.from_numpy(wr).to(device)
+        ctx = moe.MoELayer(H, I, E, K, M, device=device.index)
+        ctx.load_experts(wr_d, *ex, validate=False)
+        ctxs.append(ctx)
+        weights.append((wr_d, ex))
+    return x, ctxs, weights
+
+
+def run_ours(args):
+    import torch
+    ws, rank, local = dist_env()
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    device = torch.device("cuda", local if ws > 1 else 0)
+    torch.cuda.set_device(device)
+    from mxfp4_weight_streaming_fp8_b200 import moe
+    M = args.tokens
+    L = args.layers
+    x, ctxs, _weights = build_pool(device, M, args.routing, layers=L)
+    info = ctxs[0].query()
+    x_d = x.to(device)
+    ys = [torch.empty_like(x_d) for _ in range(L)]
+
+    # union size of each layer (from the kernel's own routing outputs)
+    Us = []
+    for l in range(L):
+        y, ids, _, _, _ = ctxs[l].decode(x_d, routing=True)
+        Us.append(len(set(ids.cpu().numpy().ravel().tolist())))
+    torch.cuda.synchronize()
+    for c in ctxs:
+        st = c.sync_status()
+        if st != moe.MOE_OK:
+            raise RuntimeError(f"kernel status {moe.status_string(st)}")
+
+    # one bench step = L layer-steps, captured once
+    stream = torch.cuda.Stream(device)
+    stream.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(stream):
+        for l in range(L):
+            assert ctxs[l].decode_raw(x_d, M, ys[l], stream=stream) == moe.MOE_OK
+    torch.cuda.current_stream().wait_stream(stream)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for l in range(L):
+            st = ctxs[l].decode_raw(x_d, M, ys[l], stream=stream)
+            assert st == moe.MOE_OK, moe.status_string(st)
+
+    cur = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(device.index) as clk:
+        ev0.record(cur)
+        for _ in range(args.steps):
+            graph.replay()
+        ev1.record(cur)
+        ev1.synchronize()
+    torch.cuda.synchronize()
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    ms_local = ev0.elapsed_time(ev1)
+    ms = max_over_ranks(ms_local, ws, device)
+    for c in ctxs:
+        st = c.sync_status()
+        if st != moe.MOE_OK:
+            raise RuntimeError(f"kernel status {moe.status_string(st)}")
+
+    layer_steps = args.steps * L
+    us_per_layer = ms * 1e3 / layer_steps
+    U_mean = sum(Us) / len(Us)
+    tokens_total = ws * M * layer_steps
+    value = tokens_total / (ms / 1e3)
+    alg = algorithmic_bytes(M, U_mean)
+    exp_b = U_mean * expert_bytes()
+    peak, peak_kind = load_peaks()
+    achieved = alg / (us_per_layer * 1e-6) / 1e9
+    workload = f"ling_layer_M{M}_{args.routing}"
+    traffic = recorded_traffic("k_fused", workload)
+
+    # ---- end to end through the public API with host buffers
+    e2e = run_e2e(args, ctxs, x, device, M, L)
+
+    # ---- CPU oracle baseline (rank 0 only)
+    cpu = run_cpu_baseline(args, M) if rank == 0 and not args.no_cpu else None
+
+    launches = layer_steps * (3 if info["variant"] == "split" else 1)
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp8e4m3 x mxfp4 (f16/fp32 accumulate)",
+        "data": "synthetic (seeded SplitMix64; random MXFP4 weights, N(0,1) bf16 activations)",
+        "config": {"workload": workload, "hidden": H, "inter": I, "num_experts": E, "top_k": K, "tokens": M,
+                   "routing": args.routing, "layers_in_pool": L, "pool_weight_bytes": L * E * expert_bytes(),
+                   "l2": "inputs larger than L2: each layer-step reads a different layer of the pool",
+                   "step": f"{L} layer-steps in one CUDA graph", "parallelism": f"replicas x{ws}",
+                   "variant": info["variant"]},
+        "us_per_layer_step": round(us_per_layer, 3),
+        "union_experts": U_mean,
+        "expert_gbs": round(exp_b / (us_per_layer * 1e-6) / 1e9, 1),
+        "expert_frac_of_8tbs": round(exp_b / (us_per_layer * 1e-6) / 8e12, 4),
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
+                     "traffic": traffic, "kernel": "k_fused" if info["variant"] == "fused" else "k_gateup+k_down",
+                     "algorithmic_bytes_per_launch": alg},
+        "gpu_launches": launches,
+        "clocks": clk.summary(),
+        "e2e": e2e,
+    }
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del graph
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_e2e(args, ctxs, x_cpu, device, M, L):
+    """Per step: pinned-host x -> device, L moe_decode calls through the
+    Python/C-ABI API, final y -> pinned host; timed with events."""
+    import torch
+    from mxfp4_weight_streaming_fp8_b200 import moe
+    xh = x_cpu.pin_memory()
+    yh = torch.empty_like(xh).pin_memory()
+    xd = torch.empty_like(xh, device=device)
+    ys = [torch.empty_like(xd) for _ in range(L)]
+    cur = torch.cuda.current_stream()
+
+    def step():
+        xd.copy_(xh, non_blocking=True)
+        for l in range(L):
+            ctxs[l].decode_raw(xd, M, ys[l], stream=cur)
+        yh.copy_(ys[-1], non_blocking=True)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(cur)
+    for _ in range(args.steps):
+        step()
+    e1.record(cur)
+    e1.synchronize()
+    ms = e0.elapsed_time(e1)
+    ws, _, _ = dist_env()
+    ms = max_over_ranks(ms, ws, device)
+    tokens = ws * M * L * args.steps
+    return {"value": round(tokens / (ms / 1e3), 1), "unit": "tokens/s",
+            "h2d_bytes_per_step": xh.numel() * 2, "d2h_bytes_per_step": yh.numel() * 2,
+            "how": f"per step: H2D x, {L} moe_decode calls (direct launches), D2H y"}
+
+
+def cpu_sample_steps(M, n_layers, seed=SEED):
+    """Inputs of a bounded oracle sample: n_layers layer-steps of the pool."""
+    import numpy as np
+    import oracle
+    from mxfp4_weight_streaming_fp8_b200 import synth
+    x = synth.gen_x(seed, M, H)
+    xb = x.view(__import__("torch").int16).numpy().view(np.uint16)
+    steps = []
+    for l in range(n_layers):
+        wr = synth.force_router(x, synth.gen_router(seed, l, E, H), K, "gap", seed=seed, layer=l)
+        ids, _ = oracle.topk(oracle.router_logits(xb, wr), K)
+        per = [[None] * E for _ in range(4)]
+        for e in sorted(set(ids.ravel().tolist())):
+            parts = synth.expert_np(seed, l, e, H, I)
+            for t in range(4):
+                per[t][e] = parts[t]
+        steps.append((wr, per))
+    return xb, steps
+
+
+def run_cpu_baseline(args, M, n_layers=None):
+    import oracle
+    n_layers = n_layers or args.cpu_layers
+    xb, steps = cpu_sample_steps(M, n_layers)
+    t0 = time.perf_counter()
+    for wr, per in steps:
+        oracle.moe_decode(xb, wr, *per, H, I, E, K)
+    dt = time.perf_counter() - t0
+    return {"value": round(M * n_layers / dt, 3), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{n_layers} layer-steps of the same workload (M={M}, distinct pool layers), "
+                      f"single-threaded fp64 C++ oracle, {dt:.2f} s"}
+
+
+def run_reference(args):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return
+    M = args.tokens
+    import oracle
+    n = max(1, args.ref_layers)
+    xb, steps = cpu_sample_steps(M, n)
+    for _ in range(min(args.warmup, 1)):
+        oracle.moe_decode(xb, steps[0][0], *steps[0][1], H, I, E, K)
+    t0 = time.perf_counter()
+    for s in range(args.steps):
+        wr, per = steps[s % n]
+        oracle.moe_decode(xb, wr, *per, H, I, E, K)
+    dt = time.perf_counter() - t0
+    value = M * args.steps / dt
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s",
+            "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(dt * 1e3 / args.steps, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"ling_layer_M{M}_{args.routing}", "hidden": H, "inter": I,
+                       "num_experts": E, "top_k": K, "tokens": M,
+                       "step": "one layer-step of the CPU oracle on host cores"},
+            "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                             "sample": f"{args.steps} layer-steps cycling over {n} pool layers"},
+            "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--tokens", type=int, default=1)
+    ap.add_argument("--routing", default="gap", choices=["gap", "zipf", "distinct", "shared", "natural"])
+    ap.add_argument("--layers", type=int, default=POOL_LAYERS)
+    ap.add_argument("--cpu-layers", type=int, default=6)
+    ap.add_argument("--ref-layers", type=int, default=4)
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,150 @@
+/*
+ * moe.h -- C ABI of libmoe: the decode step of a mixture-of-experts layer with
+ * MXFP4 expert weights and FP8 E4M3 activations (W4A8) on an NVIDIA B200
+ * (sm_100a).
+ *
+ * What the step computes. Sources: MarkTechPost, "NVIDIA Shows 3 Ways to
+ * Speed Up MoE Inference on DGX Spark" (aitujian.cn copy). The section "Why
+ * is MoE decoding on DGX Spark memory-bound?" says batch-1 decode is bound by
+ * reading weights, and that the recipe is W4A8 with MXFP4 MoE kernels. The
+ * section "What are the 3 optimizations?" covers the MXFP4 MoE kernels for
+ * the narrow 768-wide expert layer, and says a 4-token verify activates up
+ * to 32 experts. The section "What is Ling 3.0 ..." says each token is routed
+ * to 8 experts. The element formats follow OCP MX v1.0 (E2M1 codes with one
+ * E8M0 scale per 32 elements) and OCP OFP8 (E4M3).
+ *
+ * Per token m (M tokens, hidden size H, expert width I, E experts, top_k):
+ *   A1  q[m] = E4M3_rne_sat(x[m] * 448/amax_m), s_m = amax_m/448 (fp32)
+ *   A2  logits[m][e] = sum_h x[m][h] * router_w[e][h]  (bf16 x, fp32 weights)
+ *   A3  ids = top_k logits, highest first, ties to the lower expert index;
+ *       w = softmax over the top_k kept logits (sums to 1)
+ *   A4  union of the selected experts over the M tokens
+ *   A5  g_n = s_m * <W13[e][n], q[m]>, up_n = s_m * <W13[e][I+n], q[m]>
+ *   A6  h_n = silu(g_n) * up_n   (fp32, not requantised)
+ *   A7  d_r = <W2[e][r], h>
+ *   A8  y[m][r] = bf16( sum over the token's top_k slots of w * d_r )
+ * where an MXFP4 weight is E2M1(code) * 2^(E8M0 - 127) per block of 32 along K.
+ *
+ * Weight layout (row-major, K contiguous; all device memory):
+ *   w13_codes  uint8 [E][2I][H/2]  rows 0..I-1 gate, rows I..2I-1 up
+ *   w13_scales uint8 [E][2I][H/32]
+ *   w2_codes   uint8 [E][H][I/2]
+ *   w2_scales  uint8 [E][H][I/32]
+ *   Byte j of a code row holds element 2j in bits 3:0 and element 2j+1 in
+ *   bits 7:4. Scale byte t of a row covers elements [32t, 32t+32).
+ *   router_w   float [E][H]
+ *
+ * Threading and errors. A context serves one layer and one stream at a time.
+ * Calls on one context must not overlap, because they share its workspace.
+ * All argument checks are synchronous and happen before any GPU work. A
+ * failed check returns an error code and enqueues nothing. Device-side
+ * failures, such as a grid barrier that times out, set a status word in the
+ * workspace. moe_sync_status() reads it. Nothing falls back silently: a shape
+ * or device the kernels do not support returns MOE_ERR_UNSUPPORTED.
+ */
+#ifndef LIBMOE_MOE_H
+#define LIBMOE_MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,  /* null pointer, bad size, misaligned pointer      */
+  MOE_ERR_UNSUPPORTED = 2,  /* shape or device outside what the kernels cover  */
+  MOE_ERR_CUDA = 3,         /* a CUDA runtime call failed                      */
+  MOE_ERR_OOM = 4,          /* workspace allocation failed                     */
+  MOE_ERR_NOT_LOADED = 5,   /* moe_decode before moe_load_experts              */
+  MOE_ERR_TIMEOUT = 6,      /* a device-side wait gave up (see moe_sync_status) */
+  MOE_ERR_BAD_WEIGHTS = 7   /* an E8M0 scale byte is 0xFF (NaN)                */
+} moe_status;
+
+/* moe_config.flags */
+#define MOE_FLAG_SPLIT_KERNELS 0x1u /* run the step as three kernels (route, gate/up,
+                                       down) instead of one persistent kernel */
+#define MOE_FLAG_PRE_RMSNORM  0x2u  /* x <- bf16(x / sqrt(mean(x^2) + 1e-6)) before
+                                       A1/A2 (unit-weight RMSNorm between layers) */
+
+typedef struct {
+  int32_t hidden;      /* H: multiple of 32, 32..8192                        */
+  int32_t inter;       /* I: multiple of 32, 32..4096                        */
+  int32_t num_experts; /* E: 1..1024                                         */
+  int32_t top_k;       /* 1..min(E, 32)                                      */
+  int32_t max_tokens;  /* upper bound on M per call: 1..32                   */
+  uint32_t flags;      /* MOE_FLAG_*                                         */
+  int32_t device;      /* CUDA device ordinal the context lives on          */
+} moe_config;
+
+typedef struct moe_ctx moe_ctx; /* opaque */
+
+/* Create a context: validates cfg, checks the device is sm_100, allocates the
+ * workspace (sized from max_tokens) on cfg->device. *out is set only on
+ * MOE_OK. Returns INVALID_ARG / UNSUPPORTED / CUDA / OOM. */
+moe_status moe_create(const moe_config* cfg, moe_ctx** out);
+
+/* moe_load_experts load_flags */
+#define MOE_LOAD_BORROW 0x0u        /* keep the caller's pointers (they must outlive the ctx) */
+#define MOE_LOAD_SKIP_VALIDATE 0x1u /* do not scan scale bytes for 0xFF */
+
+/* Attach one layer's weights (device pointers, layouts above, each 16-byte
+ * aligned). The context borrows them: nothing is copied, and the caller keeps
+ * ownership. Unless MOE_LOAD_SKIP_VALIDATE is set, the scale bytes are scanned
+ * on the device for the NaN encoding 0xFF, synchronously on the legacy
+ * default stream; MOE_ERR_BAD_WEIGHTS if any is found. May be called again to
+ * re-point the context at other weights. */
+moe_status moe_load_experts(moe_ctx* ctx, const float* router_w,
+                            const uint8_t* w13_codes, const uint8_t* w13_scales,
+                            const uint8_t* w2_codes, const uint8_t* w2_scales,
+                            uint32_t load_flags);
+
+/* One decode step, enqueued on `stream` (a cudaStream_t; NULL = legacy
+ * default stream), asynchronous, allocation-free and capturable into a CUDA
+ * graph.
+ *   x_bf16  [M][H] bf16 device, read only
+ *   y_bf16  [M][H] bf16 device, written (must not alias x)
+ *   M       0..max_tokens; M == 0 returns MOE_OK and enqueues nothing
+ * Optional device outputs (NULL to skip):
+ *   topk_ids [M][top_k] int32, highest logit first
+ *   topk_w   [M][top_k] fp32 routing weights in the same order
+ *   xq       [M][H] uint8 E4M3 activation codes
+ *   xscale   [M] fp32 per-token activation scales
+ * Returns INVALID_ARG (null/misaligned/size), NOT_LOADED, CUDA (launch). */
+moe_status moe_decode(moe_ctx* ctx, const void* x_bf16, int32_t M, void* y_bf16,
+                      void* stream, int32_t* topk_ids, float* topk_w, uint8_t* xq,
+                      float* xscale);
+
+/* Synchronise `stream`, then read and clear the context's device status word.
+ * Returns MOE_ERR_TIMEOUT if a device-side wait gave up since the last call,
+ * and resets the barrier state so the context can be used again. */
+moe_status moe_sync_status(moe_ctx* ctx, void* stream);
+
+/* Write a JSON description of the context into buf (always NUL-terminated
+ * when len > 0): device, sm, kernel variant, grid, threads, shared memory,
+ * shapes. Lets a caller confirm at start-up which path runs. Returns
+ * INVALID_ARG if buf is NULL or too small (the JSON is then truncated). */
+moe_status moe_query(const moe_ctx* ctx, char* buf, size_t len);
+
+/* Free the workspace and the context (NULL is a no-op). Borrowed weights are
+ * not touched. */
+void moe_destroy(moe_ctx* ctx);
+
+/* Test hook for the failure path of the persistent kernel (ignored by the
+ * split path, which has no device-side waits). Sets the budget, in clock64
+ * cycles, of every device-side wait; budget_cycles <= 0 restores the default
+ * (about 0.5 s). With force_stall != 0 the logits wait looks for a tag no CTA
+ * ever writes, so that wait runs out on purpose: the kernel sets the status
+ * word, finishes with garbage output and returns, and moe_sync_status then
+ * reports MOE_ERR_TIMEOUT. Returns INVALID_ARG for a NULL ctx. */
+moe_status moe_debug_set_wait(moe_ctx* ctx, long long budget_cycles, int force_stall);
+
+/* Static string naming a status code. */
+const char* moe_status_string(moe_status s);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* LIBMOE_MOE_H */

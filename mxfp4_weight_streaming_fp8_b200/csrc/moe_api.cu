@@ -1,0 +1,396 @@
+// moe_api.cu -- the C ABI of libmoe (declared in include/moe.h): argument
+// validation, the per-context workspace, and kernel launches on the caller's
+// stream. No allocation happens after moe_create; nothing falls back to the
+// CPU.
+#include <cuda_runtime.h>
+
+#include <cstdio>
+#include <cstring>
+#include <new>
+
+#include "../../include/moe.h"
+#include "moe_device.cuh"
+#include "moe_fused.cuh"
+#include "moe_split.cuh"
+
+namespace {
+
+enum Variant { kFused = 0, kSplit = 1 };
+
+// ~0.5 s at ~2 GHz: far longer than any legitimate wait, short enough that a
+// stuck wait returns an error instead of hanging the GPU.
+constexpr long long kDefaultSpinLimit = 1000000000LL;
+
+struct DeviceGuard {
+  int prev = -1;
+  bool ok = true;
+  explicit DeviceGuard(int dev) {
+    if (cudaGetDevice(&prev) != cudaSuccess) { ok = false; return; }
+    if (prev != dev && cudaSetDevice(dev) != cudaSuccess) ok = false;
+  }
+  ~DeviceGuard() {
+    int cur;
+    if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
+  }
+};
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Shared-memory plan of the persistent kernel (mirrors k_fused's carving).
+bool make_plan(const moe_config& c, int sm_count, size_t smem_limit, moe::FusedPlan* pl) {
+  const size_t H = c.hidden, I = c.inter, E = c.num_experts, K = c.top_k, MM = c.max_tokens;
+  const size_t G = sm_count;
+  const size_t NP = MM * K, UMAX = (E < NP ? E : NP);
+  const size_t nr_max = (I + G - 1) / G, nrd_max = (H + G - 1) / G;
+  pl->G = (int)G;
+  pl->max_tokens = (int)MM;
+  pl->max_pairs = (int)NP;
+  pl->max_union = (int)UMAX;
+  pl->rpc_max = (int)nrd_max;
+  pl->slot_gu = (int)align_up(nr_max * H + 2 * (nr_max * H / 32 + 32), 128);
+  pl->slot_d = (int)align_up(nrd_max * (I / 2) + nrd_max * (I / 32) + 32, 128);
+  const size_t kMaxSlots = 64;
+  size_t off = 0;
+  auto take = [&](size_t bytes, size_t a) { off = align_up(off, a); size_t o = off; off += bytes; return o; };
+  pl->o_bar = (int)take((4 * kMaxSlots + 1) * 8, 16);
+  pl->o_misc = (int)take((2 * moe::kMaxTokens + 4 * moe::kFusedWarps + 8) * 4, 16);
+  pl->o_ids = (int)take(NP * 4, 16);
+  pl->o_w = (int)take(NP * 4, 16);
+  pl->o_pm = (int)take(NP * 4, 16);
+  pl->o_ppos = (int)take(NP * 4, 16);
+  pl->o_union = (int)take(UMAX * 4, 16);
+  pl->o_poff = (int)take((UMAX + 1) * 4, 16);
+  pl->o_cnt = (int)take(E * 4, 16);
+  pl->o_act = (int)take(MM * H, 16);
+  pl->o_dsm = (int)take(NP * nrd_max * 4, 16);
+  off = align_up(off, 128);
+  if (off >= smem_limit) return false;
+  const size_t room = smem_limit - off;
+  const size_t per = pl->slot_gu + pl->slot_d;
+  size_t n_both = room / per;
+  if (n_both < 2) return false;
+  size_t ns_gu, ns_d;
+  if (n_both >= UMAX) {
+    ns_gu = ns_d = UMAX;
+  } else {
+    ns_gu = ns_d = n_both;
+    ns_gu += (room - n_both * per) / pl->slot_gu;
+    if (ns_gu > UMAX) ns_gu = UMAX;
+  }
+  if (ns_gu > kMaxSlots) ns_gu = kMaxSlots;
+  if (ns_d > kMaxSlots) ns_d = kMaxSlots;
+  pl->ns_gu = (int)ns_gu;
+  pl->ns_d = (int)ns_d;
+  pl->o_ring_gu = (int)off;
+  pl->o_ring_d = (int)(off + ns_gu * pl->slot_gu);
+  pl->smem_bytes = (int)(pl->o_ring_d + ns_d * pl->slot_d);
+  pl->wr_bytes_max = (int)(((E + G - 1) / G) * H * 4);
+  if ((size_t)pl->wr_bytes_max > ns_gu * pl->slot_gu) return false;  // router rows alias ring_gu
+  return (size_t)pl->smem_bytes <= smem_limit;
+}
+
+}  // namespace
+
+struct moe_ctx {
+  moe_config cfg{};
+  int dev = 0;
+  int sm_count = 0;
+  int variant = kFused;
+  void* ws_base = nullptr;
+  size_t ws_bytes = 0;
+  moe::Workspace ws{};
+  const float* wr = nullptr;
+  const uint8_t* w13c = nullptr;
+  const uint8_t* w13s = nullptr;
+  const uint8_t* w2c = nullptr;
+  const uint8_t* w2s = nullptr;
+  bool loaded = false;
+  // launch shapes
+  int grid_route = 0, grid_gateup = 0, grid_down = 0, grid_fused = 0;
+  size_t smem_gateup = 0, smem_fused = 0;
+  long long spin_limit = 0;
+  int force_stall = 0;
+  moe::FusedPlan plan{};
+  moe::FusedWs fws{};
+};
+
+extern "C" {
+
+const char* moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+    case MOE_ERR_OOM: return "MOE_ERR_OOM";
+    case MOE_ERR_NOT_LOADED: return "MOE_ERR_NOT_LOADED";
+    case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT";
+    case MOE_ERR_BAD_WEIGHTS: return "MOE_ERR_BAD_WEIGHTS";
+  }
+  return "MOE_ERR_UNKNOWN";
+}
+
+moe_status moe_create(const moe_config* cfg, moe_ctx** out) {
+  if (!cfg || !out) return MOE_ERR_INVALID_ARG;
+  const moe_config c = *cfg;
+  if (c.hidden < 32 || c.hidden > 8192 || c.hidden % 32) return MOE_ERR_INVALID_ARG;
+  if (c.inter < 32 || c.inter > 4096 || c.inter % 32) return MOE_ERR_INVALID_ARG;
+  if (c.num_experts < 1 || c.num_experts > moe::kMaxExperts) return MOE_ERR_INVALID_ARG;
+  if (c.top_k < 1 || c.top_k > c.num_experts || c.top_k > moe::kMaxTopK) return MOE_ERR_INVALID_ARG;
+  if (c.max_tokens < 1 || c.max_tokens > moe::kMaxTokens) return MOE_ERR_INVALID_ARG;
+  if (c.flags & ~(MOE_FLAG_SPLIT_KERNELS | MOE_FLAG_PRE_RMSNORM)) return MOE_ERR_INVALID_ARG;
+  if (c.flags & MOE_FLAG_PRE_RMSNORM) return MOE_ERR_UNSUPPORTED;
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess) return MOE_ERR_CUDA;
+  if (c.device < 0 || c.device >= ndev) return MOE_ERR_INVALID_ARG;
+  DeviceGuard guard(c.device);
+  if (!guard.ok) return MOE_ERR_CUDA;
+  cudaDeviceProp prop;
+  if (cudaGetDeviceProperties(&prop, c.device) != cudaSuccess) return MOE_ERR_CUDA;
+  if (prop.major != 10 || prop.minor != 0) return MOE_ERR_UNSUPPORTED;  // built for sm_100a only
+
+  moe_ctx* ctx = new (std::nothrow) moe_ctx();
+  if (!ctx) return MOE_ERR_OOM;
+  ctx->cfg = c;
+  ctx->dev = c.device;
+  ctx->sm_count = prop.multiProcessorCount;
+  ctx->variant = (c.flags & MOE_FLAG_SPLIT_KERNELS) ? kSplit : kFused;
+  ctx->spin_limit = kDefaultSpinLimit;
+
+  // workspace layout
+  const size_t H = c.hidden, I = c.inter, E = c.num_experts, K = c.top_k, MM = c.max_tokens;
+  const size_t NP = MM * K, UMAX = (E < NP ? E : NP);
+  size_t off = 0;
+  auto take = [&](size_t bytes) { size_t o = off; off = align_up(off + bytes, 256); return o; };
+  const size_t o_ctrl = take(64 * sizeof(unsigned));
+  const size_t o_logits = take(MM * E * sizeof(float));
+  const size_t o_xq = take(MM * H);
+  const size_t o_xscale = take(MM * sizeof(float));
+  const size_t o_ids = take(NP * sizeof(int));
+  const size_t o_wts = take(NP * sizeof(float));
+  const size_t o_meta = take(16 * sizeof(int));
+  const size_t o_union = take(UMAX * sizeof(int));
+  const size_t o_poff = take((UMAX + 1) * sizeof(int));
+  const size_t o_ptok = take(NP * sizeof(int));
+  const size_t o_pslot = take(NP * sizeof(int));
+  const size_t o_pw = take(NP * sizeof(float));
+  const size_t o_h = take(NP * I * sizeof(float));
+  const size_t o_l64 = take(MM * E * sizeof(unsigned long long));
+  const size_t o_flag = take(UMAX * (size_t)ctx->sm_count * sizeof(unsigned));
+  ctx->ws_bytes = off;
+  if (cudaMalloc(&ctx->ws_base, ctx->ws_bytes) != cudaSuccess) {
+    cudaGetLastError();
+    delete ctx;
+    return MOE_ERR_OOM;
+  }
+  if (cudaMemset(ctx->ws_base, 0, ctx->ws_bytes) != cudaSuccess) {
+    cudaFree(ctx->ws_base);
+    delete ctx;
+    return MOE_ERR_CUDA;
+  }
+  char* b = static_cast<char*>(ctx->ws_base);
+  moe::Workspace& w = ctx->ws;
+  w.ctrl = reinterpret_cast<unsigned*>(b + o_ctrl);
+  w.logits = reinterpret_cast<float*>(b + o_logits);
+  w.xq = reinterpret_cast<uint8_t*>(b + o_xq);
+  w.xscale = reinterpret_cast<float*>(b + o_xscale);
+  w.ids = reinterpret_cast<int*>(b + o_ids);
+  w.wts = reinterpret_cast<float*>(b + o_wts);
+  w.meta = reinterpret_cast<int*>(b + o_meta);
+  w.union_ids = reinterpret_cast<int*>(b + o_union);
+  w.pair_off = reinterpret_cast<int*>(b + o_poff);
+  w.pair_tok = reinterpret_cast<int*>(b + o_ptok);
+  w.pair_slot = reinterpret_cast<int*>(b + o_pslot);
+  w.pair_w = reinterpret_cast<float*>(b + o_pw);
+  w.h = reinterpret_cast<float*>(b + o_h);
+  ctx->fws.logits64 = reinterpret_cast<unsigned long long*>(b + o_l64);
+  ctx->fws.guflag = reinterpret_cast<unsigned*>(b + o_flag);
+  ctx->fws.epoch = w.ctrl + 5;
+
+  // launch shapes
+  ctx->grid_route = (int)(E < (size_t)ctx->sm_count ? E : (size_t)ctx->sm_count);
+  ctx->smem_gateup = MM * H * 2;
+  cudaError_t err = cudaFuncSetAttribute(moe::k_gateup, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)ctx->smem_gateup);
+  int occ_g = 0, occ_d = 0;
+  if (err == cudaSuccess)
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_g, moe::k_gateup, moe::kThreads, ctx->smem_gateup);
+  if (err == cudaSuccess)
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_d, moe::k_down, moe::kThreads, 0);
+  const bool plan_ok = make_plan(c, ctx->sm_count, (size_t)prop.sharedMemPerBlockOptin, &ctx->plan);
+  if (err == cudaSuccess && plan_ok)
+    err = cudaFuncSetAttribute(moe::k_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, ctx->plan.smem_bytes);
+  int occ_f = 0;
+  if (err == cudaSuccess && plan_ok)
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_f, moe::k_fused, moe::kFusedThreads,
+                                                        ctx->plan.smem_bytes);
+  if (err != cudaSuccess || occ_g < 1 || occ_d < 1 || !plan_ok || occ_f < 1) {
+    cudaGetLastError();
+    cudaFree(ctx->ws_base);
+    delete ctx;
+    return MOE_ERR_UNSUPPORTED;
+  }
+  ctx->grid_gateup = occ_g * ctx->sm_count;
+  ctx->grid_down = occ_d * ctx->sm_count;
+  ctx->grid_fused = ctx->plan.G;
+  ctx->smem_fused = ctx->plan.smem_bytes;
+  *out = ctx;
+  return MOE_OK;
+}
+
+void moe_destroy(moe_ctx* ctx) {
+  if (!ctx) return;
+  DeviceGuard guard(ctx->dev);
+  if (ctx->ws_base) cudaFree(ctx->ws_base);
+  delete ctx;
+}
+
+moe_status moe_load_experts(moe_ctx* ctx, const float* router_w, const uint8_t* w13_codes,
+                            const uint8_t* w13_scales, const uint8_t* w2_codes, const uint8_t* w2_scales,
+                            uint32_t load_flags) {
+  if (!ctx || !router_w || !w13_codes || !w13_scales || !w2_codes || !w2_scales) return MOE_ERR_INVALID_ARG;
+  if (load_flags & ~MOE_LOAD_SKIP_VALIDATE) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(router_w) || !aligned16(w13_codes) || !aligned16(w13_scales) || !aligned16(w2_codes) ||
+      !aligned16(w2_scales))
+    return MOE_ERR_INVALID_ARG;
+  DeviceGuard guard(ctx->dev);
+  if (!guard.ok) return MOE_ERR_CUDA;
+  const moe_config& c = ctx->cfg;
+  if (!(load_flags & MOE_LOAD_SKIP_VALIDATE)) {
+    const size_t E = c.num_experts, H = c.hidden, I = c.inter;
+    unsigned* bad = ctx->ws.ctrl + 4;
+    if (cudaMemset(bad, 0, sizeof(unsigned)) != cudaSuccess) return MOE_ERR_CUDA;
+    moe::k_scan_scales<<<ctx->sm_count * 4, 256>>>(w13_scales, E * 2 * I * (H / 32), bad);
+    moe::k_scan_scales<<<ctx->sm_count * 4, 256>>>(w2_scales, E * H * (I / 32), bad);
+    unsigned nbad = 0;
+    if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaMemcpy(&nbad, bad, sizeof(unsigned), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+    if (nbad) {
+      ctx->loaded = false;
+      return MOE_ERR_BAD_WEIGHTS;
+    }
+  }
+  ctx->wr = router_w;
+  ctx->w13c = w13_codes;
+  ctx->w13s = w13_scales;
+  ctx->w2c = w2_codes;
+  ctx->w2s = w2_scales;
+  ctx->loaded = true;
+  return MOE_OK;
+}
+
+moe_status moe_decode(moe_ctx* ctx, const void* x_bf16, int32_t M, void* y_bf16, void* stream,
+                      int32_t* topk_ids, float* topk_w, uint8_t* xq, float* xscale) {
+  if (!ctx) return MOE_ERR_INVALID_ARG;
+  const moe_config& c = ctx->cfg;
+  if (M < 0 || M > c.max_tokens) return MOE_ERR_INVALID_ARG;
+  if (M == 0) return MOE_OK;
+  if (!x_bf16 || !y_bf16 || !aligned16(x_bf16) || !aligned16(y_bf16)) return MOE_ERR_INVALID_ARG;
+  const size_t xbytes = (size_t)M * c.hidden * 2;
+  const char* xb = static_cast<const char*>(x_bf16);
+  const char* yb = static_cast<const char*>(y_bf16);
+  if (xb < yb + xbytes && yb < xb + xbytes) return MOE_ERR_INVALID_ARG;  // aliasing
+  if ((xq && !aligned16(xq)) || (topk_ids && (reinterpret_cast<uintptr_t>(topk_ids) & 3)) ||
+      (topk_w && (reinterpret_cast<uintptr_t>(topk_w) & 3)) ||
+      (xscale && (reinterpret_cast<uintptr_t>(xscale) & 3)))
+    return MOE_ERR_INVALID_ARG;
+  if (!ctx->loaded) return MOE_ERR_NOT_LOADED;
+  DeviceGuard guard(ctx->dev);
+  if (!guard.ok) return MOE_ERR_CUDA;
+  moe::Params p{};
+  p.H = c.hidden;
+  p.I = c.inter;
+  p.E = c.num_experts;
+  p.K = c.top_k;
+  p.M = M;
+  p.x = static_cast<const __nv_bfloat16*>(x_bf16);
+  p.y = static_cast<__nv_bfloat16*>(y_bf16);
+  p.wr = ctx->wr;
+  p.w13c = ctx->w13c;
+  p.w13s = ctx->w13s;
+  p.w2c = ctx->w2c;
+  p.w2s = ctx->w2s;
+  p.ws = ctx->ws;
+  p.out_ids = topk_ids;
+  p.out_w = topk_w;
+  p.out_xq = xq;
+  p.out_xscale = xscale;
+  p.spin_limit = ctx->spin_limit;
+  p.force_stall = ctx->force_stall;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (ctx->variant == kSplit) {
+    moe::k_route<<<ctx->grid_route, moe::kThreads, 0, st>>>(p);
+    moe::k_gateup<<<ctx->grid_gateup, moe::kThreads, (size_t)M * c.hidden * 2, st>>>(p);
+    moe::k_down<<<ctx->grid_down, moe::kThreads, 0, st>>>(p);
+  } else {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(ctx->grid_fused);
+    cfg.blockDim = dim3(moe::kFusedThreads);
+    cfg.dynamicSmemBytes = ctx->smem_fused;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, moe::k_fused, p, ctx->fws, ctx->plan) != cudaSuccess) {
+      cudaGetLastError();
+      return MOE_ERR_CUDA;
+    }
+  }
+  if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+moe_status moe_sync_status(moe_ctx* ctx, void* stream) {
+  if (!ctx) return MOE_ERR_INVALID_ARG;
+  DeviceGuard guard(ctx->dev);
+  if (!guard.ok) return MOE_ERR_CUDA;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MOE_ERR_CUDA;
+  unsigned status = 0;
+  if (cudaMemcpy(&status, ctx->ws.ctrl, sizeof(unsigned), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (status == 0) return MOE_OK;
+  // a wait gave up: clear the whole workspace (status, barrier state, epoch
+  // and every epoch-tagged word) so the next call starts clean
+  if (cudaMemset(ctx->ws_base, 0, ctx->ws_bytes) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
+  return MOE_ERR_TIMEOUT;
+}
+
+moe_status moe_debug_set_wait(moe_ctx* ctx, long long budget_cycles, int force_stall) {
+  if (!ctx) return MOE_ERR_INVALID_ARG;
+  ctx->spin_limit = budget_cycles > 0 ? budget_cycles : kDefaultSpinLimit;
+  ctx->force_stall = force_stall ? 1 : 0;
+  return MOE_OK;
+}
+
+moe_status moe_query(const moe_ctx* ctx, char* buf, size_t len) {
+  if (!ctx || !buf || len == 0) return MOE_ERR_INVALID_ARG;
+  const moe_config& c = ctx->cfg;
+  const moe::FusedPlan& pl = ctx->plan;
+  int n;
+  if (ctx->variant == kSplit) {
+    n = snprintf(buf, len,
+                 "{\"lib\": \"libmoe\", \"arch\": \"sm_100a\", \"device\": %d, \"sm_count\": %d, "
+                 "\"variant\": \"split\", \"kernels\": [\"k_route\", \"k_gateup\", \"k_down\"], "
+                 "\"grid\": [%d, %d, %d], \"threads\": %d, \"smem_gateup\": %zu, "
+                 "\"hidden\": %d, \"inter\": %d, \"num_experts\": %d, \"top_k\": %d, \"max_tokens\": %d}",
+                 ctx->dev, ctx->sm_count, ctx->grid_route, ctx->grid_gateup, ctx->grid_down, moe::kThreads,
+                 ctx->smem_gateup, c.hidden, c.inter, c.num_experts, c.top_k, c.max_tokens);
+  } else {
+    n = snprintf(buf, len,
+                 "{\"lib\": \"libmoe\", \"arch\": \"sm_100a\", \"device\": %d, \"sm_count\": %d, "
+                 "\"variant\": \"fused\", \"kernels\": [\"k_fused\"], \"grid\": [%d], \"threads\": %d, "
+                 "\"smem\": %d, \"ring_gu\": [%d, %d], \"ring_d\": [%d, %d], \"pdl\": true, "
+                 "\"hidden\": %d, \"inter\": %d, \"num_experts\": %d, \"top_k\": %d, \"max_tokens\": %d}",
+                 ctx->dev, ctx->sm_count, pl.G, moe::kFusedThreads, pl.smem_bytes, pl.ns_gu, pl.slot_gu, pl.ns_d,
+                 pl.slot_d, c.hidden, c.inter, c.num_experts, c.top_k, c.max_tokens);
+  }
+  if (n < 0 || (size_t)n >= len) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,156 @@
+"""ctypes binding of libmoe (the C ABI in include/moe.h).
+
+Argument marshalling only: every step of the decode runs in the CUDA kernels
+behind the C ABI. torch supplies device memory, streams and data pointers. If
+libmoe.so is missing, the first call raises. There is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import json
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libmoe.so")
+
+MOE_OK = 0
+STATUS_NAMES = {
+    0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_CUDA",
+    4: "MOE_ERR_OOM", 5: "MOE_ERR_NOT_LOADED", 6: "MOE_ERR_TIMEOUT", 7: "MOE_ERR_BAD_WEIGHTS",
+}
+MOE_FLAG_SPLIT_KERNELS = 0x1
+MOE_FLAG_PRE_RMSNORM = 0x2
+MOE_LOAD_BORROW = 0x0
+MOE_LOAD_SKIP_VALIDATE = 0x1
+
+
+class MoEError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {STATUS_NAMES.get(status, status)}")
+
+
+class moe_config(ctypes.Structure):
+    _fields_ = [("hidden", ctypes.c_int32), ("inter", ctypes.c_int32), ("num_experts", ctypes.c_int32),
+                ("top_k", ctypes.c_int32), ("max_tokens", ctypes.c_int32), ("flags", ctypes.c_uint32),
+                ("device", ctypes.c_int32)]
+
+
+_lib = None
+_vp = ctypes.c_void_p
+
+
+def lib() -> ctypes.CDLL:
+    """Load libmoe.so (built in-tree by mxfp4_weight_streaming_fp8_b200.build)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libmoe.so not found at {LIB_PATH}: build it with "
+                               "`python -m mxfp4_weight_streaming_fp8_b200.build` (no fallback path exists)")
+        L = ctypes.CDLL(LIB_PATH)
+        L.moe_create.argtypes = [ctypes.POINTER(moe_config), ctypes.POINTER(_vp)]
+        L.moe_create.restype = ctypes.c_int
+        L.moe_load_experts.argtypes = [_vp] * 6 + [ctypes.c_uint32]
+        L.moe_load_experts.restype = ctypes.c_int
+        L.moe_decode.argtypes = [_vp, _vp, ctypes.c_int32, _vp, _vp, _vp, _vp, _vp, _vp]
+        L.moe_decode.restype = ctypes.c_int
+        L.moe_sync_status.argtypes = [_vp, _vp]
+        L.moe_sync_status.restype = ctypes.c_int
+        L.moe_query.argtypes = [_vp, ctypes.c_char_p, ctypes.c_size_t]
+        L.moe_query.restype = ctypes.c_int
+        L.moe_destroy.argtypes = [_vp]
+        L.moe_destroy.restype = None
+        L.moe_status_string.argtypes = [ctypes.c_int]
+        L.moe_status_string.restype = ctypes.c_char_p
+        L.moe_debug_set_wait.argtypes = [_vp, ctypes.c_longlong, ctypes.c_int]
+        L.moe_debug_set_wait.restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def status_string(s: int) -> str:
+    return lib().moe_status_string(int(s)).decode()
+
+
+class MoELayer:
+    """One MoE layer's context: moe_create / moe_load_experts / moe_decode."""
+
+    def __init__(self, hidden: int, inter: int, num_experts: int, top_k: int, max_tokens: int,
+                 flags: int = 0, device: int = 0):
+        self.cfg = moe_config(hidden, inter, num_experts, top_k, max_tokens, flags, device)
+        self.hidden, self.inter, self.num_experts, self.top_k = hidden, inter, num_experts, top_k
+        self.max_tokens = max_tokens
+        self.device = device
+        self._ctx = _vp()
+        st = lib().moe_create(ctypes.byref(self.cfg), ctypes.byref(self._ctx))
+        if st != MOE_OK:
+            raise MoEError(st, "moe_create")
+        self._weights = None
+
+    def load_experts(self, router_w, w13_codes, w13_scales, w2_codes, w2_scales, validate: bool = True):
+        """Borrow device tensors (kept referenced here so they outlive the context)."""
+        flags = 0 if validate else MOE_LOAD_SKIP_VALIDATE
+        st = lib().moe_load_experts(self._ctx, _ptr(router_w), _ptr(w13_codes), _ptr(w13_scales),
+                                    _ptr(w2_codes), _ptr(w2_scales), flags)
+        if st != MOE_OK:
+            raise MoEError(st, "moe_load_experts")
+        self._weights = (router_w, w13_codes, w13_scales, w2_codes, w2_scales)
+
+    def decode_raw(self, x, M: int, y, stream=None, topk_ids=None, topk_w=None, xq=None, xscale=None) -> int:
+        """moe_decode with explicit buffers; returns the status code."""
+        return lib().moe_decode(self._ctx, _ptr(x), int(M), _ptr(y), _stream_handle(stream), _ptr(topk_ids),
+                                _ptr(topk_w), _ptr(xq), _ptr(xscale))
+
+    def decode(self, x, y=None, stream=None, routing: bool = False):
+        """x: bf16 [M, H] on the device. Returns y (and the routing outputs if asked)."""
+        import torch
+        M = x.shape[0]
+        if y is None:
+            y = torch.empty_like(x)
+        extra = [None] * 4
+        if routing:
+            dev = x.device
+            extra = [torch.empty((M, self.top_k), dtype=torch.int32, device=dev),
+                     torch.empty((M, self.top_k), dtype=torch.float32, device=dev),
+                     torch.empty((M, self.hidden), dtype=torch.uint8, device=dev),
+                     torch.empty((M,), dtype=torch.float32, device=dev)]
+        st = self.decode_raw(x, M, y, stream, *extra)
+        if st != MOE_OK:
+            raise MoEError(st, "moe_decode")
+        return (y, *extra) if routing else y
+
+    def sync_status(self, stream=None) -> int:
+        return lib().moe_sync_status(self._ctx, _stream_handle(stream))
+
+    def set_wait(self, budget_cycles: int, force_stall: bool = False) -> int:
+        return lib().moe_debug_set_wait(self._ctx, int(budget_cycles), int(bool(force_stall)))
+
+    def query(self) -> dict:
+        buf = ctypes.create_string_buffer(1024)
+        st = lib().moe_query(self._ctx, buf, len(buf))
+        if st != MOE_OK:
+            raise MoEError(st, "moe_query")
+        return json.loads(buf.value.decode())
+
+    def close(self):
+        if self._ctx:
+            lib().moe_destroy(self._ctx)
+            self._ctx = _vp()
+        self._weights = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -1,0 +1,98 @@
+"""Shared helpers for the GPU parity tests: build a seeded layer on the device,
+run the CUDA path through the C ABI, run the oracle on the same inputs, and
+compare.
+
+The tolerance on y is a per-token bound: every element must satisfy
+|y_gpu - y_oracle_fp64| <= 2e-3 * ||y_oracle[m]||_2. FP8 activation codes and
+expert ids must match bit for bit. Where ids are compared, the oracle's fp64
+gap at rank k must be at least 1e-5, because closer pairs can legitimately
+reorder under fp32.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+from mxfp4_weight_streaming_fp8_b200 import moe, synth
+
+Y_TOL = 2e-3      # per-token relative-to-norm bound on y
+W_TOL = 1e-5      # routing weights (fp32 softmax vs fp64)
+GAP_MIN = 1e-5    # fp64 logit gap needed to demand identical ids
+
+
+def bits(t: torch.Tensor) -> np.ndarray:
+    return t.contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
+
+
+class Layer:
+    """Seeded inputs of one MoE layer, on the device and (lazily) on the CPU."""
+
+    def __init__(self, H, I, E, K, M, seed=0, layer=0, mode="gap", device="cuda:0"):
+        self.H, self.I, self.E, self.K, self.M = H, I, E, K, M
+        self.seed, self.layer = seed, layer
+        self.x = synth.gen_x(seed, M, H, layer=layer)
+        self.wr = synth.force_router(self.x, synth.gen_router(seed, layer, E, H), K, mode, seed=seed,
+                                     layer=layer) if M > 0 else synth.gen_router(seed, layer, E, H)
+        self.dev = torch.device(device)
+        self.experts = synth.layer_experts_torch(seed, layer, E, H, I, self.dev)
+        self.wr_d = torch.from_numpy(self.wr).to(self.dev)
+        self.x_d = self.x.to(self.dev)
+
+    def expert_slices(self, ids):
+        per = [[None] * self.E for _ in range(4)]
+        for e in sorted(set(int(i) for i in np.asarray(ids).ravel())):
+            parts = synth.expert_np(self.seed, self.layer, e, self.H, self.I)
+            for t in range(4):
+                per[t][e] = parts[t]
+        return per
+
+    def oracle(self, tokens=None):
+        """Oracle outputs for the given token subset (default all)."""
+        xb = bits(self.x)
+        if tokens is not None:
+            xb = xb[list(tokens)]
+        logits = oracle.router_logits(xb, self.wr)
+        ids, _ = oracle.topk(logits, self.K)
+        per = self.expert_slices(ids)
+        return oracle.moe_decode(xb, self.wr, *per, self.H, self.I, self.E, self.K)
+
+    def make_ctx(self, flags=0, max_tokens=None):
+        ctx = moe.MoELayer(self.H, self.I, self.E, self.K, max_tokens or max(1, self.M), flags=flags,
+                           device=self.dev.index or 0)
+        ctx.load_experts(self.wr_d, *self.experts)
+        return ctx
+
+    def run(self, ctx):
+        y, ids, w, xq, xs = ctx.decode(self.x_d, routing=True)
+        torch.cuda.synchronize()
+        st = ctx.sync_status()
+        assert st == moe.MOE_OK, moe.status_string(st)
+        return dict(y=y, ids=ids.cpu().numpy(), w=w.cpu().numpy(), q=xq.cpu().numpy(), s=xs.cpu().numpy())
+
+
+def min_gap(logits: np.ndarray, k: int) -> float:
+    """Smallest fp64 gap among each token's k+1 largest logits."""
+    s = -np.sort(-logits, axis=1)[:, :k + 1]
+    if s.shape[1] < 2:
+        return np.inf
+    return float(np.min(s[:, :-1] - s[:, 1:]))
+
+
+def compare(layer: Layer, got: dict, ref: dict, tokens=None, check_ids=True):
+    """Assert parity; returns the worst y error as a fraction of the bound."""
+    t = list(range(layer.M)) if tokens is None else list(tokens)
+    assert np.array_equal(got["q"][t], ref["q"]), "E4M3 activation codes differ"
+    assert np.array_equal(got["s"][t], ref["s"]), "activation scales differ"
+    if check_ids:
+        gap = min_gap(ref["logits"], layer.K)
+        if gap >= GAP_MIN:
+            assert np.array_equal(got["ids"][t], ref["ids"]), "expert ids differ"
+            assert np.all(np.abs(got["w"][t] - ref["weights"]) <= W_TOL), "routing weights differ"
+    y = got["y"].float().cpu().numpy().astype(np.float64)[t]
+    norm = np.linalg.norm(ref["y64"], axis=1, keepdims=True)
+    bound = Y_TOL * norm
+    err = np.abs(y - ref["y64"])
+    worst = float(np.max(err / np.maximum(bound, 1e-300))) if err.size else 0.0
+    assert np.all(err <= bound), f"y error {err.max():.3e} exceeds bound {bound.min():.3e} (ratio {worst:.2f})"
+    return worst

@@ -1,0 +1,68 @@
+"""The C-ABI library builds, loads and exports every entry point include/moe.h
+declares; host-side argument checks work without a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from mxfp4_weight_streaming_fp8_b200 import build as libbuild
+from mxfp4_weight_streaming_fp8_b200 import moe
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    libbuild.build()
+    return moe.lib()
+
+
+def declared_functions():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names += re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(moe_\w+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for want in ("moe_create", "moe_load_experts", "moe_decode", "moe_sync_status", "moe_query",
+                 "moe_destroy", "moe_status_string"):
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+
+
+def test_status_strings(L):
+    for code, name in moe.STATUS_NAMES.items():
+        assert moe.status_string(code) == name
+
+
+def test_create_rejects_bad_config_without_gpu(L):
+    out = ctypes.c_void_p()
+    assert L.moe_create(None, ctypes.byref(out)) == 1
+    bad = [moe.moe_config(100, 64, 16, 2, 1, 0, 0),   # H not a multiple of 32
+           moe.moe_config(256, 48, 16, 2, 1, 0, 0),   # I not a multiple of 32
+           moe.moe_config(256, 64, 16, 17, 1, 0, 0),  # top_k > E
+           moe.moe_config(256, 64, 16, 2, 33, 0, 0),  # max_tokens > 32
+           moe.moe_config(256, 64, 2000, 2, 1, 0, 0),  # E > 1024
+           moe.moe_config(256, 64, 16, 2, 1, 0x80, 0)]  # unknown flag
+    for c in bad:
+        assert L.moe_create(ctypes.byref(c), ctypes.byref(out)) == 1
+        assert not out.value
+
+
+def test_null_context_calls(L):
+    assert L.moe_decode(None, None, 1, None, None, None, None, None, None) == 1
+    assert L.moe_sync_status(None, None) == 1
+    buf = ctypes.create_string_buffer(64)
+    assert L.moe_query(None, buf, 64) == 1
+    assert L.moe_debug_set_wait(None, 0, 0) == 1
+    L.moe_destroy(None)

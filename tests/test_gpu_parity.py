@@ -1,0 +1,209 @@
+"""CUDA path (through the C ABI) against the CPU oracle, element by element.
+
+Shapes: the tiny 16-expert layer (H=256, I=64, top-2), a ragged layer whose
+sizes divide into no tile evenly, the Ling-shaped layer (H=2560, I=768,
+E=256, top-8) at M=1, the 4-token verify shape with 32 distinct, 8 shared and
+random experts, and an M sweep up to 32 under a Zipf expert prior. Both the
+persistent kernel and the three-kernel path are checked, plus edge cases,
+determinism and the error paths.
+"""
+import numpy as np
+import pytest
+import torch
+
+from cases import Layer, compare, min_gap, bits
+from mxfp4_weight_streaming_fp8_b200 import moe, synth
+
+pytestmark = pytest.mark.gpu
+
+VARIANTS = {"fused": 0, "split": moe.MOE_FLAG_SPLIT_KERNELS}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    from mxfp4_weight_streaming_fp8_b200 import build
+    build.build()
+    assert torch.cuda.is_available()
+
+
+@pytest.mark.parametrize("variant", VARIANTS)
+def test_tiny_layer_seed0(variant):
+    L = Layer(256, 64, 16, 2, 1, seed=0, mode="natural")
+    ctx = L.make_ctx(VARIANTS[variant])
+    assert ctx.query()["variant"] == variant
+    got = L.run(ctx)
+    ref = L.oracle()
+    gap = min_gap(ref["logits"], 2)
+    print(f"tiny seed 0: fp64 gap at rank 2 = {gap:.3e}")
+    compare(L, got, ref)
+
+
+@pytest.mark.parametrize("variant", VARIANTS)
+@pytest.mark.parametrize("shape", [(96, 32, 5, 3, 3), (160, 96, 12, 4, 7), (544, 224, 40, 6, 5)])
+def test_ragged_shapes(variant, shape):
+    H, I, E, K, M = shape
+    L = Layer(H, I, E, K, M, seed=3, mode="gap")
+    got = L.run(L.make_ctx(VARIANTS[variant]))
+    compare(L, got, L.oracle())
+
+
+@pytest.mark.parametrize("variant", VARIANTS)
+def test_ling_layer_m1(variant):
+    L = Layer(2560, 768, 256, 8, 1, seed=0, mode="gap")
+    got = L.run(L.make_ctx(VARIANTS[variant]))
+    worst = compare(L, got, L.oracle())
+    print(f"Ling M=1 {variant}: worst y error = {worst:.3f} of the bound")
+
+
+@pytest.mark.parametrize("variant", VARIANTS)
+@pytest.mark.parametrize("mode,U", [("distinct", 32), ("shared", 8), ("gap", None)])
+def test_verify_shape_m4(variant, mode, U):
+    L = Layer(2560, 768, 256, 8, 4, seed=1, mode=mode)
+    got = L.run(L.make_ctx(VARIANTS[variant]))
+    if U is not None:
+        assert len(set(got["ids"].ravel().tolist())) == U
+    compare(L, got, L.oracle())
+
+
+@pytest.mark.parametrize("M", [2, 8, 16, 32])
+def test_zipf_sweep_sampled(M):
+    """Routing outputs for every token; y checked on a sample of tokens."""
+    L = Layer(2560, 768, 256, 8, M, seed=2, mode="zipf")
+    got = L.run(L.make_ctx(0, max_tokens=32))
+    split = L.run(L.make_ctx(moe.MOE_FLAG_SPLIT_KERNELS, max_tokens=32))
+    assert np.array_equal(got["ids"], split["ids"])
+    sample = sorted(set([0, M - 1, M // 2, (7 * M) // 9]))
+    compare(L, got, L.oracle(tokens=sample), tokens=sample)
+    compare(L, split, L.oracle(tokens=sample), tokens=sample)
+
+
+def test_max_tokens_all_checked_small_layer():
+    L = Layer(256, 64, 16, 4, 32, seed=4, mode="gap")
+    got = L.run(L.make_ctx(0))
+    compare(L, got, L.oracle())
+
+
+def test_all_experts_selected():
+    L = Layer(128, 64, 8, 8, 3, seed=5, mode="natural")
+    got = L.run(L.make_ctx(0))
+    ref = L.oracle()
+    assert sorted(got["ids"][0].tolist()) == list(range(8))
+    compare(L, got, ref, check_ids=False)
+
+
+@pytest.mark.parametrize("variant", VARIANTS)
+def test_zero_input(variant):
+    L = Layer(256, 64, 16, 2, 2, seed=6, mode="natural")
+    L.x = torch.zeros_like(L.x)
+    L.x_d = L.x.to(L.dev)
+    got = L.run(L.make_ctx(VARIANTS[variant]))
+    assert not got["y"].float().abs().sum().item()
+    assert np.all(got["q"] == 0) and np.all(got["s"] == 1.0)
+    assert np.array_equal(got["ids"], np.array([[0, 1], [0, 1]]))
+    assert np.allclose(got["w"], 0.5)
+
+
+def test_empty_batch_is_a_no_op():
+    L = Layer(256, 64, 16, 2, 1, seed=0, mode="natural")
+    ctx = L.make_ctx(0)
+    y = torch.full_like(L.x_d, 7.0)
+    assert ctx.decode_raw(L.x_d, 0, y) == moe.MOE_OK
+    torch.cuda.synchronize()
+    assert torch.all(y == 7.0)
+
+
+def test_deterministic_and_repeatable():
+    L = Layer(2560, 768, 256, 8, 4, seed=7, mode="gap")
+    ctx = L.make_ctx(0)
+    a = L.run(ctx)
+    b = L.run(ctx)
+    assert torch.equal(a["y"], b["y"])
+    for _ in range(3):
+        c = L.run(ctx)
+    assert torch.equal(a["y"], c["y"])
+
+
+def test_fused_and_split_agree():
+    L = Layer(2560, 768, 256, 8, 4, seed=8, mode="gap")
+    a = L.run(L.make_ctx(0))
+    b = L.run(L.make_ctx(moe.MOE_FLAG_SPLIT_KERNELS))
+    assert np.array_equal(a["q"], b["q"]) and np.array_equal(a["ids"], b["ids"])
+    ya, yb = a["y"].float(), b["y"].float()
+    assert torch.all((ya - yb).abs() <= 4e-3 * ya.norm(dim=1, keepdim=True))
+
+
+def test_consecutive_layers_share_stream():
+    """Back-to-back calls on different contexts (programmatic dependent
+    launch between them) give the same results as separate calls."""
+    Ls = [Layer(2560, 768, 256, 8, 1, seed=9, layer=l, mode="gap") for l in range(3)]
+    ctxs = [L.make_ctx(0) for L in Ls]
+    ys = [torch.empty_like(L.x_d) for L in Ls]
+    for L, c, y in zip(Ls, ctxs, ys):
+        assert c.decode_raw(L.x_d, 1, y) == moe.MOE_OK
+    torch.cuda.synchronize()
+    for L, c, y in zip(Ls, ctxs, ys):
+        alone = L.run(c)["y"]
+        assert torch.equal(alone, y)
+
+
+def test_graph_capture_and_replay():
+    L = Layer(2560, 768, 256, 8, 1, seed=10, mode="gap")
+    ctx = L.make_ctx(0)
+    y = torch.empty_like(L.x_d)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        assert ctx.decode_raw(L.x_d, 1, y, stream=s) == moe.MOE_OK
+    torch.cuda.current_stream().wait_stream(s)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        assert ctx.decode_raw(L.x_d, 1, y) == moe.MOE_OK
+    y.zero_()
+    g.replay()
+    g.replay()
+    torch.cuda.synchronize()
+    assert ctx.sync_status() == moe.MOE_OK
+    ref = L.oracle()
+    got = dict(y=y, q=ref["q"], s=ref["s"], ids=ref["ids"], w=ref["weights"])
+    compare(L, got, ref, check_ids=False)
+
+
+def test_error_paths():
+    L = Layer(256, 64, 16, 2, 1, seed=0, mode="natural")
+    ctx = moe.MoELayer(256, 64, 16, 2, 2)
+    y = torch.empty_like(L.x_d)
+    assert ctx.decode_raw(L.x_d, 1, y) == 5  # not loaded
+    ctx.load_experts(L.wr_d, *L.experts)
+    assert ctx.decode_raw(L.x_d, 3, y) == 1   # M > max_tokens
+    assert ctx.decode_raw(L.x_d, -1, y) == 1
+    assert ctx.decode_raw(L.x_d, 1, L.x_d) == 1  # y aliases x
+    xs = torch.empty(2 * 256 + 8, dtype=torch.bfloat16, device=L.dev)
+    assert ctx.decode_raw(xs[1:257], 1, y) == 1  # misaligned x
+    bad = L.experts[1].clone()
+    bad.view(-1)[12345] = 0xFF
+    with pytest.raises(moe.MoEError) as ei:
+        ctx.load_experts(L.wr_d, L.experts[0], bad, L.experts[2], L.experts[3])
+    assert ei.value.status == 7
+    assert ctx.decode_raw(L.x_d, 1, y) == 5  # a failed load leaves the ctx unloaded
+
+
+def test_forced_timeout_is_reported_and_recovers():
+    L = Layer(256, 64, 16, 2, 1, seed=0, mode="natural")
+    ctx = L.make_ctx(0)
+    good = L.run(ctx)["y"].clone()
+    assert ctx.set_wait(20000, force_stall=True) == moe.MOE_OK
+    y = torch.empty_like(L.x_d)
+    assert ctx.decode_raw(L.x_d, 1, y) == moe.MOE_OK
+    assert ctx.sync_status() == 6  # MOE_ERR_TIMEOUT
+    assert ctx.set_wait(0, force_stall=False) == moe.MOE_OK
+    again = L.run(ctx)["y"]
+    assert torch.equal(again, good)
+
+
+def test_device_generator_matches_cpu_slices():
+    H, I, E = 2560, 768, 8
+    full = synth.layer_experts_torch(11, 3, E, H, I, "cuda:0")
+    for e in (0, 5):
+        part = synth.expert_np(11, 3, e, H, I)
+        for a, b in zip(full, part):
+            assert np.array_equal(a[e].cpu().numpy(), b)
