@@ -132,6 +132,14 @@ moe_status moe_query(const moe_ctx* ctx, char* buf, size_t len);
  * not touched. */
 void moe_destroy(moe_ctx* ctx);
 
+/* Host-only: the launch plan the persistent kernel would get for cfg on a
+ * device with sm_count SMs and smem_limit bytes of opt-in shared memory per
+ * block (grid, shared-memory carving, ring slots), as JSON in buf. Makes no
+ * CUDA call. Returns INVALID_ARG for a bad cfg or a NULL / too small buf,
+ * UNSUPPORTED when the shape does not fit (buf still holds the plan). */
+moe_status moe_plan_query(const moe_config* cfg, int32_t sm_count, size_t smem_limit,
+                          char* buf, size_t len);
+
 /* Test hook for the failure path of the persistent kernel (ignored by the
  * split path, which has no device-side waits). Sets the budget, in clock64
  * cycles, of every device-side wait; budget_cycles <= 0 restores the default

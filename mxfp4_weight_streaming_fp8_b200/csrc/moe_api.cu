@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdio>
+#include <algorithm>
 #include <cstring>
 #include <new>
 
@@ -37,6 +38,17 @@ struct DeviceGuard {
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+moe_status validate_config(const moe_config& c) {
+  if (c.hidden < 32 || c.hidden > 8192 || c.hidden % 32) return MOE_ERR_INVALID_ARG;
+  if (c.inter < 32 || c.inter > 4096 || c.inter % 32) return MOE_ERR_INVALID_ARG;
+  if (c.num_experts < 1 || c.num_experts > moe::kMaxExperts) return MOE_ERR_INVALID_ARG;
+  if (c.top_k < 1 || c.top_k > c.num_experts || c.top_k > moe::kMaxTopK) return MOE_ERR_INVALID_ARG;
+  if (c.max_tokens < 1 || c.max_tokens > moe::kMaxTokens) return MOE_ERR_INVALID_ARG;
+  if (c.flags & ~(MOE_FLAG_SPLIT_KERNELS | MOE_FLAG_PRE_RMSNORM)) return MOE_ERR_INVALID_ARG;
+  if (c.flags & MOE_FLAG_PRE_RMSNORM) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
 
 // Shared-memory plan of the persistent kernel (mirrors k_fused's carving).
 bool make_plan(const moe_config& c, int sm_count, size_t smem_limit, moe::FusedPlan* pl) {
@@ -83,11 +95,13 @@ bool make_plan(const moe_config& c, int sm_count, size_t smem_limit, moe::FusedP
   if (ns_d > kMaxSlots) ns_d = kMaxSlots;
   pl->ns_gu = (int)ns_gu;
   pl->ns_d = (int)ns_d;
-  pl->o_ring_gu = (int)off;
-  pl->o_ring_d = (int)(off + ns_gu * pl->slot_gu);
-  pl->smem_bytes = (int)(pl->o_ring_d + ns_d * pl->slot_d);
+  // the router rows of a CTA are staged at the start of ring_gu before any
+  // weight chunk lands there; make ring_gu at least that large
   pl->wr_bytes_max = (int)(((E + G - 1) / G) * H * 4);
-  if ((size_t)pl->wr_bytes_max > ns_gu * pl->slot_gu) return false;  // router rows alias ring_gu
+  const size_t ring_gu_bytes = align_up(std::max(ns_gu * (size_t)pl->slot_gu, (size_t)pl->wr_bytes_max), 128);
+  pl->o_ring_gu = (int)off;
+  pl->o_ring_d = (int)(off + ring_gu_bytes);
+  pl->smem_bytes = (int)(pl->o_ring_d + ns_d * pl->slot_d);
   return (size_t)pl->smem_bytes <= smem_limit;
 }
 
@@ -135,13 +149,8 @@ const char* moe_status_string(moe_status s) {
 moe_status moe_create(const moe_config* cfg, moe_ctx** out) {
   if (!cfg || !out) return MOE_ERR_INVALID_ARG;
   const moe_config c = *cfg;
-  if (c.hidden < 32 || c.hidden > 8192 || c.hidden % 32) return MOE_ERR_INVALID_ARG;
-  if (c.inter < 32 || c.inter > 4096 || c.inter % 32) return MOE_ERR_INVALID_ARG;
-  if (c.num_experts < 1 || c.num_experts > moe::kMaxExperts) return MOE_ERR_INVALID_ARG;
-  if (c.top_k < 1 || c.top_k > c.num_experts || c.top_k > moe::kMaxTopK) return MOE_ERR_INVALID_ARG;
-  if (c.max_tokens < 1 || c.max_tokens > moe::kMaxTokens) return MOE_ERR_INVALID_ARG;
-  if (c.flags & ~(MOE_FLAG_SPLIT_KERNELS | MOE_FLAG_PRE_RMSNORM)) return MOE_ERR_INVALID_ARG;
-  if (c.flags & MOE_FLAG_PRE_RMSNORM) return MOE_ERR_UNSUPPORTED;
+  const moe_status v = validate_config(c);
+  if (v != MOE_OK) return v;
   int ndev = 0;
   if (cudaGetDeviceCount(&ndev) != cudaSuccess) return MOE_ERR_CUDA;
   if (c.device < 0 || c.device >= ndev) return MOE_ERR_INVALID_ARG;
@@ -358,6 +367,24 @@ moe_status moe_sync_status(moe_ctx* ctx, void* stream) {
   if (cudaMemset(ctx->ws_base, 0, ctx->ws_bytes) != cudaSuccess) return MOE_ERR_CUDA;
   if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
   return MOE_ERR_TIMEOUT;
+}
+
+moe_status moe_plan_query(const moe_config* cfg, int32_t sm_count, size_t smem_limit, char* buf, size_t len) {
+  if (!cfg || !buf || len == 0 || sm_count < 1) return MOE_ERR_INVALID_ARG;
+  const moe_status v = validate_config(*cfg);
+  if (v != MOE_OK) return v;
+  moe::FusedPlan pl{};
+  const bool ok = make_plan(*cfg, sm_count, smem_limit, &pl);
+  const int n = snprintf(buf, len,
+                         "{\"ok\": %s, \"grid\": %d, \"threads\": %d, \"smem\": %d, \"slot_gu\": %d, "
+                         "\"ns_gu\": %d, \"slot_d\": %d, \"ns_d\": %d, \"rows_per_cta_down\": %d, "
+                         "\"router_bytes_per_cta\": %d, \"o_act\": %d, \"o_dsm\": %d, \"o_ring_gu\": %d, "
+                         "\"o_ring_d\": %d}",
+                         ok ? "true" : "false", pl.G, moe::kFusedThreads, pl.smem_bytes, pl.slot_gu, pl.ns_gu,
+                         pl.slot_d, pl.ns_d, pl.rpc_max, pl.wr_bytes_max, pl.o_act, pl.o_dsm, pl.o_ring_gu,
+                         pl.o_ring_d);
+  if (n < 0 || (size_t)n >= len) return MOE_ERR_INVALID_ARG;
+  return ok ? MOE_OK : MOE_ERR_UNSUPPORTED;
 }
 
 moe_status moe_debug_set_wait(moe_ctx* ctx, long long budget_cycles, int force_stall) {

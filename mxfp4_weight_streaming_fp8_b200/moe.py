@@ -62,6 +62,9 @@ def lib() -> ctypes.CDLL:
         L.moe_destroy.restype = None
         L.moe_status_string.argtypes = [ctypes.c_int]
         L.moe_status_string.restype = ctypes.c_char_p
+        L.moe_plan_query.argtypes = [ctypes.POINTER(moe_config), ctypes.c_int32, ctypes.c_size_t,
+                                     ctypes.c_char_p, ctypes.c_size_t]
+        L.moe_plan_query.restype = ctypes.c_int
         L.moe_debug_set_wait.argtypes = [_vp, ctypes.c_longlong, ctypes.c_int]
         L.moe_debug_set_wait.restype = ctypes.c_int
         _lib = L
@@ -77,6 +80,14 @@ def _stream_handle(stream):
     if stream is None:
         stream = torch.cuda.current_stream()
     return ctypes.c_void_p(stream.cuda_stream)
+
+
+def plan_query(hidden, inter, num_experts, top_k, max_tokens, flags=0, sm_count=148, smem_limit=232448):
+    """(status, plan dict) of the persistent kernel for a shape; host only."""
+    cfg = moe_config(hidden, inter, num_experts, top_k, max_tokens, flags, 0)
+    buf = ctypes.create_string_buffer(1024)
+    st = lib().moe_plan_query(ctypes.byref(cfg), sm_count, smem_limit, buf, len(buf))
+    return st, (json.loads(buf.value.decode()) if buf.value else None)
 
 
 def status_string(s: int) -> str:

@@ -66,3 +66,30 @@ def test_null_context_calls(L):
     assert L.moe_query(None, buf, 64) == 1
     assert L.moe_debug_set_wait(None, 0, 0) == 1
     L.moe_destroy(None)
+
+
+@pytest.mark.parametrize("shape", [(256, 64, 16, 2, 1), (96, 32, 5, 3, 3), (160, 96, 12, 4, 7),
+                                   (544, 224, 40, 6, 5), (2560, 768, 256, 8, 1), (2560, 768, 256, 8, 4),
+                                   (2560, 768, 256, 8, 32), (256, 64, 16, 4, 32), (128, 64, 8, 8, 3),
+                                   (32, 32, 1, 1, 1), (4096, 1024, 512, 8, 8)])
+def test_persistent_kernel_plan_fits(L, shape):
+    """Host-only launch plan (no CUDA call): shared-memory carving fits the
+    227 KB opt-in limit, the router rows of a CTA fit their staging area, and
+    every ring holds at least two slots big enough for one CTA's slice."""
+    st, pl = moe.plan_query(*shape)
+    assert st == 0 and pl["ok"], pl
+    H, I, E, K, MM = shape
+    G = pl["grid"]
+    assert G == 148 and pl["smem"] <= 232448
+    assert pl["o_ring_d"] - pl["o_ring_gu"] >= pl["router_bytes_per_cta"]
+    assert pl["router_bytes_per_cta"] == -(-E // G) * H * 4
+    nr, nrd = -(-I // G), -(-H // G)
+    assert pl["slot_gu"] >= nr * H + 2 * (nr * H // 32 + 30)
+    assert pl["slot_d"] >= nrd * I // 2 + nrd * I // 32 + 30
+    assert pl["ns_gu"] >= min(2, min(E, MM * K)) and pl["ns_d"] >= min(2, min(E, MM * K))
+    assert pl["o_act"] % 16 == 0 and pl["o_ring_gu"] % 128 == 0 and pl["o_ring_d"] % 128 == 0
+
+
+def test_plan_rejects_what_does_not_fit(L):
+    st, pl = moe.plan_query(8192, 4096, 1024, 32, 32)
+    assert st == 2 and not pl["ok"]
