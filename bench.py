@@ -170,7 +170,7 @@ def sum_over_ranks(value: float, ws: int, device=None) -> float:
 
 
 # ------------------------------------------------------------------ workload
-def build_pool(device, M, mode, layers=POOL_LAYERS, seed=SEED):
+def build_pool(device, M, mode, layers=POOL_LAYERS, seed=SEED, flags=0):
     import torch
     from mxfp4_weight_streaming_fp8_b200 import moe, synth
     x = synth.gen_x(seed, M, H)
@@ -179,7 +179,7 @@ def build_pool(device, M, mode, layers=POOL_LAYERS, seed=SEED):
         wr = synth.force_router(x, synth.gen_router(seed, l, E, H), K, mode, seed=seed, layer=l)
         ex = synth.layer_experts_torch(seed, l, E, H, I, device)
         wr_d = torch.from_numpy(wr).to(device)
-        ctx = moe.MoELayer(H, I, E, K, M, device=device.index)
+        ctx = moe.MoELayer(H, I, E, K, M, flags=flags, device=device.index)
         ctx.load_experts(wr_d, *ex, validate=False)
         ctxs.append(ctx)
         weights.append((wr_d, ex))
@@ -199,7 +199,8 @@ def run_ours(args):
     from mxfp4_weight_streaming_fp8_b200 import moe
     M = args.tokens
     L = args.layers
-    x, ctxs, _weights = build_pool(device, M, args.routing, layers=L)
+    flags = moe.MOE_FLAG_SPLIT_KERNELS if args.variant == "split" else 0
+    x, ctxs, _weights = build_pool(device, M, args.routing, layers=L, flags=flags)
     info = ctxs[0].query()
     x_d = x.to(device)
     ys = [torch.empty_like(x_d) for _ in range(L)]
@@ -417,6 +418,7 @@ def main():
     ap.add_argument("--cpu-layers", type=int, default=6)
     ap.add_argument("--ref-layers", type=int, default=4)
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--variant", choices=["fused", "split"], default="fused")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3

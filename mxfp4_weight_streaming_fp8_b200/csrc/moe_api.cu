@@ -56,6 +56,7 @@ bool make_plan(const moe_config& c, int sm_count, size_t smem_limit, moe::FusedP
   const size_t G = sm_count;
   const size_t NP = MM * K, UMAX = (E < NP ? E : NP);
   const size_t nr_max = (I + G - 1) / G, nrd_max = (H + G - 1) / G;
+  *pl = moe::FusedPlan{};
   pl->G = (int)G;
   pl->max_tokens = (int)MM;
   pl->max_pairs = (int)NP;
@@ -63,10 +64,12 @@ bool make_plan(const moe_config& c, int sm_count, size_t smem_limit, moe::FusedP
   pl->rpc_max = (int)nrd_max;
   pl->slot_gu = (int)align_up(nr_max * H + 2 * (nr_max * H / 32 + 32), 128);
   pl->slot_d = (int)align_up(nrd_max * (I / 2) + nrd_max * (I / 32) + 32, 128);
-  const size_t kMaxSlots = 64;
+  pl->hpairs = (int)std::min<size_t>(moe::kHPairs, MM);
+  pl->hslot = (int)align_up((size_t)pl->hpairs * I * 2 + moe::kHPairs * 4, 16);
+  const size_t kMaxSlots = moe::kMaxSlots;
   size_t off = 0;
   auto take = [&](size_t bytes, size_t a) { off = align_up(off, a); size_t o = off; off += bytes; return o; };
-  pl->o_bar = (int)take((4 * kMaxSlots + 1) * 8, 16);
+  pl->o_bar = (int)take((5 * kMaxSlots + 1) * 8 + 2 * kMaxSlots * 4, 16);
   pl->o_misc = (int)take((2 * moe::kMaxTokens + 4 * moe::kFusedWarps + 8) * 4, 16);
   pl->o_ids = (int)take(NP * 4, 16);
   pl->o_w = (int)take(NP * 4, 16);
@@ -79,8 +82,9 @@ bool make_plan(const moe_config& c, int sm_count, size_t smem_limit, moe::FusedP
   pl->o_dsm = (int)take(NP * nrd_max * 4, 16);
   off = align_up(off, 128);
   if (off >= smem_limit) return false;
+  // each down slot carries its staged h
   const size_t room = smem_limit - off;
-  const size_t per = pl->slot_gu + pl->slot_d;
+  const size_t per = pl->slot_gu + pl->slot_d + pl->hslot;
   size_t n_both = room / per;
   if (n_both < 2) return false;
   size_t ns_gu, ns_d;
@@ -95,13 +99,18 @@ bool make_plan(const moe_config& c, int sm_count, size_t smem_limit, moe::FusedP
   if (ns_d > kMaxSlots) ns_d = kMaxSlots;
   pl->ns_gu = (int)ns_gu;
   pl->ns_d = (int)ns_d;
-  // the router rows of a CTA are staged at the start of ring_gu before any
-  // weight chunk lands there; make ring_gu at least that large
+  pl->o_h = (int)off;
+  off = align_up(off + ns_d * pl->hslot, 128);
+  // ring_gu also holds the router rows of the CTA and then the gathered
+  // logits [M][E] fp32 between routing and the first weight chunk
   pl->wr_bytes_max = (int)(((E + G - 1) / G) * H * 4);
-  const size_t ring_gu_bytes = align_up(std::max(ns_gu * (size_t)pl->slot_gu, (size_t)pl->wr_bytes_max), 128);
+  const size_t staged = std::max((size_t)pl->wr_bytes_max, MM * E * 4);
+  const size_t ring_gu_bytes = align_up(std::max(ns_gu * (size_t)pl->slot_gu, staged), 128);
   pl->o_ring_gu = (int)off;
   pl->o_ring_d = (int)(off + ring_gu_bytes);
   pl->smem_bytes = (int)(pl->o_ring_d + ns_d * pl->slot_d);
+  // ring_d holds the bf16 activations during routing when they fit
+  pl->x_staged = (MM * H * 2 <= ns_d * (size_t)pl->slot_d) ? 1 : 0;
   return (size_t)pl->smem_bytes <= smem_limit;
 }
 
@@ -186,8 +195,11 @@ moe_status moe_create(const moe_config* cfg, moe_ctx** out) {
   const size_t o_pslot = take(NP * sizeof(int));
   const size_t o_pw = take(NP * sizeof(float));
   const size_t o_h = take(NP * I * sizeof(float));
-  const size_t o_l64 = take(MM * E * sizeof(unsigned long long));
-  const size_t o_flag = take(UMAX * (size_t)ctx->sm_count * sizeof(unsigned));
+  const size_t o_flog = take(MM * E * sizeof(float));
+  const size_t o_rcnt = take(sizeof(unsigned long long));
+  const size_t o_rdone = take(moe::kFlagCopies * moe::kFlagStride * sizeof(unsigned));
+  const size_t o_gcnt = take(UMAX * sizeof(unsigned long long));
+  const size_t o_gdone = take(UMAX * moe::kFlagCopies * moe::kFlagStride * sizeof(unsigned));
   ctx->ws_bytes = off;
   if (cudaMalloc(&ctx->ws_base, ctx->ws_bytes) != cudaSuccess) {
     cudaGetLastError();
@@ -214,8 +226,11 @@ moe_status moe_create(const moe_config* cfg, moe_ctx** out) {
   w.pair_slot = reinterpret_cast<int*>(b + o_pslot);
   w.pair_w = reinterpret_cast<float*>(b + o_pw);
   w.h = reinterpret_cast<float*>(b + o_h);
-  ctx->fws.logits64 = reinterpret_cast<unsigned long long*>(b + o_l64);
-  ctx->fws.guflag = reinterpret_cast<unsigned*>(b + o_flag);
+  ctx->fws.logits = reinterpret_cast<float*>(b + o_flog);
+  ctx->fws.route_cnt = reinterpret_cast<unsigned long long*>(b + o_rcnt);
+  ctx->fws.route_done = reinterpret_cast<unsigned*>(b + o_rdone);
+  ctx->fws.gu_cnt = reinterpret_cast<unsigned long long*>(b + o_gcnt);
+  ctx->fws.gu_done = reinterpret_cast<unsigned*>(b + o_gdone);
   ctx->fws.epoch = w.ctrl + 5;
 
   // launch shapes
@@ -379,10 +394,10 @@ moe_status moe_plan_query(const moe_config* cfg, int32_t sm_count, size_t smem_l
                          "{\"ok\": %s, \"grid\": %d, \"threads\": %d, \"smem\": %d, \"slot_gu\": %d, "
                          "\"ns_gu\": %d, \"slot_d\": %d, \"ns_d\": %d, \"rows_per_cta_down\": %d, "
                          "\"router_bytes_per_cta\": %d, \"o_act\": %d, \"o_dsm\": %d, \"o_ring_gu\": %d, "
-                         "\"o_ring_d\": %d}",
+                         "\"o_ring_d\": %d, \"o_h\": %d, \"hslot\": %d, \"hpairs\": %d, \"x_staged\": %d}",
                          ok ? "true" : "false", pl.G, moe::kFusedThreads, pl.smem_bytes, pl.slot_gu, pl.ns_gu,
                          pl.slot_d, pl.ns_d, pl.rpc_max, pl.wr_bytes_max, pl.o_act, pl.o_dsm, pl.o_ring_gu,
-                         pl.o_ring_d);
+                         pl.o_ring_d, pl.o_h, pl.hslot, pl.hpairs, pl.x_staged);
   if (n < 0 || (size_t)n >= len) return MOE_ERR_INVALID_ARG;
   return ok ? MOE_OK : MOE_ERR_UNSUPPORTED;
 }

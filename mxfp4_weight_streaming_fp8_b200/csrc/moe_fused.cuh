@@ -11,11 +11,13 @@
 //  1. Before griddepcontrol.wait (programmatic dependent launch), each CTA
 //     starts a TMA bulk copy of its slice of the router weights into shared
 //     memory. Router weights never depend on the previous kernel.
-//  2. Each CTA quantises all M tokens to E4M3 into shared memory (A1). It
-//     computes the logits of its router rows (A2) and publishes them as
-//     64-bit words {logit, epoch}. A reader knows a word is fresh when its tag
-//     equals the launch's epoch, so no separate grid barrier is needed.
-//  3. Every CTA reads all the logits and, redundantly, computes top-k,
+//  2. Each CTA quantises all M tokens to E4M3 into shared memory (A1) and
+//     computes the logits of its router rows (A2). A grid-wide arrival
+//     counter (+G per launch) tells when all logits are in L2. The CTA whose
+//     arrival completes the count writes the launch epoch to 8 flag copies on
+//     separate L2 lines, and each CTA polls one copy from a single thread,
+//     with back-off.
+//  3. Every CTA gathers all the logits and, redundantly, computes top-k,
 //     softmax and the expert union (A3, A4) in shared memory.
 //  4. Warp 0, lane 0 is the producer. It issues TMA bulk copies of this CTA's
 //     share of every union expert into two shared-memory rings:
@@ -23,12 +25,15 @@
 //         gate rows, up rows and their E8M0 scale bytes
 //       - down: output rows [H*b/G, H*(b+1)/G) of each expert, with scales
 //     Each active weight byte is read from HBM once, by one CTA.
-//  5. Warps 1..15 consume. For gate/up items (A5, A6) they decode E2M1 in
-//     registers, run f16x2 FMAs on exact products, apply the E8M0 scale in
-//     fp32, then SwiGLU, and write h to global memory. When a CTA has
-//     finished all its gate/up work for expert u, it sets flag[u][cta] =
-//     epoch. A down item for expert u (A7) waits until all G flags of u are
-//     set, so down work on early experts overlaps gate/up work on later ones.
+//  5. Warps 1..15 take items from one in-order queue: the gate/up items of
+//     entry u, then its down items, then entry u+1, in the order the
+//     producer issues the chunks, which rules out deadlock. For gate/up
+//     items (A5, A6) they decode E2M1 in registers, run f16x2 FMAs on exact
+//     products, apply the E8M0 scale in fp32, then SwiGLU, and write h to L2.
+//     When a CTA has finished entry u, it arrives on that entry's grid
+//     counter. The first down item of u (A7) waits on the counter's flag and
+//     stages h once into shared memory for the CTA, so down work on early
+//     experts overlaps gate/up work on later ones.
 //  6. Each CTA combines its output rows in slot order (A8) and writes bf16 y.
 //
 // Every wait is bounded: on timeout the kernel sets the status word and goes
@@ -44,25 +49,35 @@ constexpr int kFusedWarps = kFusedThreads / 32;
 constexpr int kConsumers = kFusedWarps - 1;  // warp 0 produces
 constexpr int kGuRowsPerItem = 2;           // intermediate rows per gate/up item
 constexpr int kDownRowsPerItem = 6;         // output rows per down item
+constexpr int kHPairs = 4;                  // (token, slot) pairs of one expert whose h is staged in smem
+constexpr int kFlagCopies = 8;              // completion flags are replicated over this many L2 lines
+constexpr int kFlagStride = 32;             // u32 words between copies (one 128-byte line)
+constexpr int kMaxSlots = 64;
 
 // Launch-invariant plan computed on the host at moe_create.
 struct FusedPlan {
-  int G;              // grid size (CTAs)
+  int G;                // grid size (CTAs)
   int max_tokens, max_pairs, max_union;
   int slot_gu, slot_d;  // bytes per ring slot
   int ns_gu, ns_d;      // slots per ring
   int rpc_max;          // max output rows per CTA
+  int hslot;            // bytes of staged h per down slot
+  int hpairs;           // pairs staged per down slot (min(kHPairs, max_tokens))
   // shared memory offsets (bytes)
-  int o_bar, o_misc, o_ids, o_w, o_pm, o_ppos, o_union, o_poff, o_cnt, o_act, o_dsm, o_ring_gu, o_ring_d;
+  int o_bar, o_misc, o_ids, o_w, o_pm, o_ppos, o_union, o_poff, o_cnt, o_act, o_dsm, o_h, o_ring_gu, o_ring_d;
   int smem_bytes;
-  int wr_bytes_max;   // router rows staged per CTA (alias the rings)
+  int wr_bytes_max;     // router rows staged per CTA (alias ring_gu)
+  int x_staged;         // bf16 x fits in ring_d and is staged there during routing
 };
 
-// Workspace pieces only the fused kernel uses.
+// Workspace pieces only the persistent kernel uses.
 struct FusedWs {
-  unsigned long long* logits64;  // [maxM][E] {fp32 logit, epoch}
-  unsigned* guflag;              // [max_union][G] epoch when CTA finished gate/up of union entry u
-  unsigned* epoch;               // launch counter (ctrl word)
+  float* logits;                  // [maxM][E]
+  unsigned long long* route_cnt;  // router arrivals; += G per launch
+  unsigned* route_done;           // [kFlagCopies * kFlagStride] epoch of the last complete router phase
+  unsigned long long* gu_cnt;     // [max_union] gate/up arrivals per union entry; += G per launch
+  unsigned* gu_done;              // [max_union][kFlagCopies * kFlagStride]
+  unsigned* epoch;                // launch counter
 };
 
 // ---------------------------------------------------------------- PTX helpers
@@ -105,20 +120,13 @@ __device__ __forceinline__ void mbar_wait(uint64_t* bar, unsigned parity, const 
   }
 }
 
-__device__ __forceinline__ uint64_t l2_evict_first_policy() {
-  uint64_t pol;
-  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
-  return pol;
-}
-
 // 1-D TMA bulk copy global -> shared, completion counted on `bar`.
-// dst, src 16-byte aligned; bytes a multiple of 16.
-__device__ __forceinline__ void tma_load_1d(void* dst, const void* src, unsigned bytes, uint64_t* bar,
-                                            uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;"
-      ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
-      : "memory");
+// dst, src 16-byte aligned; bytes a multiple of 16. (No L2 eviction hint: an
+// evict-first policy measured slower on this stream.)
+__device__ __forceinline__ void tma_load_1d(void* dst, const void* src, unsigned bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
 }
 
 __device__ __forceinline__ void fence_mbar_init() {
@@ -138,11 +146,74 @@ __device__ __forceinline__ unsigned ld_relaxed_u32(const unsigned* p) {
   asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
 }
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
 __device__ __forceinline__ void st_relaxed_u64(unsigned long long* p, unsigned long long v) {
   asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
 __device__ __forceinline__ void st_relaxed_u32(unsigned* p, unsigned v) {
   asm volatile("st.relaxed.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ unsigned long long atom_add_acqrel_u64(unsigned long long* p, unsigned long long v) {
+  unsigned long long old;
+  asm volatile("atom.acq_rel.gpu.global.add.u64 %0, [%1], %2;" : "=l"(old) : "l"(p), "l"(v) : "memory");
+  return old;
+}
+__device__ __forceinline__ void st_release_u32(unsigned* p, unsigned v) {
+  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ unsigned atom_add_acqrel_cta_smem(unsigned* p, unsigned v) {
+  unsigned old;
+  asm volatile("atom.acq_rel.cta.shared::cta.add.u32 %0, [%1], %2;" : "=r"(old) : "r"(smem_u32(p)), "r"(v) : "memory");
+  return old;
+}
+
+// Arrive on a grid-wide completion point: a monotonic counter that gains G
+// per launch. The CTA whose arrival completes the launch's count publishes
+// `epoch` to kFlagCopies flag words on separate L2 lines (release), so
+// waiters spread their polling instead of hammering one line.
+__device__ __forceinline__ void grid_arrive(unsigned long long* cnt, unsigned* done, unsigned long long target,
+                                            unsigned epoch) {
+  const unsigned long long old = atom_add_acqrel_u64(cnt, 1ull);
+  if (old + 1 == target) {
+#pragma unroll
+    for (int k = 0; k < kFlagCopies; ++k) st_release_u32(done + k * kFlagStride, epoch);
+  }
+}
+
+// Wait (one thread) until flag copy `which` reads `want` (acquire), with a
+// growing sleep between polls; bounded by the wait budget.
+__device__ __forceinline__ void grid_wait(const unsigned* done, int which, unsigned want, const Params& p) {
+  const unsigned* f = done + (which % kFlagCopies) * kFlagStride;
+  if (ld_acquire_u32(f) == want) return;
+  const long long t0 = clock64();
+  unsigned ns = 32;
+  while (ld_acquire_u32(f) != want) {
+    __nanosleep(ns);
+    if (ns < 256) ns <<= 1;
+    if (clock64() - t0 > p.spin_limit) {
+      atomicOr(p.ws.ctrl, kStatusTimeout);
+      return;
+    }
+  }
+}
+
+// Wait (one thread) until a shared-memory count reaches `target`.
+__device__ __forceinline__ void smem_count_wait(const unsigned* c, unsigned target, const Params& p) {
+  const volatile unsigned* v = c;
+  if (*v >= target) return;
+  const long long t0 = clock64();
+  while (*v < target) {
+    __nanosleep(32);
+    if (clock64() - t0 > p.spin_limit) {
+      atomicOr(p.ws.ctrl, kStatusTimeout);
+      return;
+    }
+  }
 }
 
 __device__ __forceinline__ void consumers_sync() {
@@ -209,6 +280,8 @@ __device__ __forceinline__ unsigned d_layout(const Params& p, int e, int r0, int
 // ---------------------------------------------------------------- compute items
 // Gate/up item: rows [a, a+cnt) of the chunk (local index), every pair of the
 // expert. Lane owns half-blocks hb = lane + 32j (16 elements, 8 code bytes).
+// Products E2M1 x E4M3 are exact in f16; each f16x2 half sums 8 of them
+// (|sum| <= 8*6*448 = 21504) before the fp32 block-scale FMA.
 __device__ __forceinline__ void gu_item(const Params& p, const GuChunk& ch, int a, int cnt, int n0,
                                         int pb, int pe, const int* s_pm, const uint8_t* act,
                                         const float* s_xs) {
@@ -242,16 +315,20 @@ __device__ __forceinline__ void gu_item(const Params& p, const GuChunk& ch, int 
           e2m1x8_to_f16x2x4(cg.y, wg + 4);
           e2m1x8_to_f16x2x4(cu.x, wu);
           e2m1x8_to_f16x2x4(cu.y, wu + 4);
-          __half2 hg = __float2half2_rn(0.f), hu = __float2half2_rn(0.f);
+          __half2 hg0 = __float2half2_rn(0.f), hu0 = hg0, hg1 = hg0, hu1 = hg0;
 #pragma unroll
-          for (int t = 0; t < 8; ++t) {
-            const __half2 av = *reinterpret_cast<const __half2*>(&a2[t]);
-            hg = __hfma2(*reinterpret_cast<const __half2*>(&wg[t]), av, hg);
-            hu = __hfma2(*reinterpret_cast<const __half2*>(&wu[t]), av, hu);
+          for (int t = 0; t < 4; ++t) {
+            const __half2 av0 = *reinterpret_cast<const __half2*>(&a2[t]);
+            const __half2 av1 = *reinterpret_cast<const __half2*>(&a2[t + 4]);
+            hg0 = __hfma2(*reinterpret_cast<const __half2*>(&wg[t]), av0, hg0);
+            hu0 = __hfma2(*reinterpret_cast<const __half2*>(&wu[t]), av0, hu0);
+            hg1 = __hfma2(*reinterpret_cast<const __half2*>(&wg[t + 4]), av1, hg1);
+            hu1 = __hfma2(*reinterpret_cast<const __half2*>(&wu[t + 4]), av1, hu1);
           }
-          const float2 fg = __half22float2(hg), fu = __half22float2(hu);
-          ag[r] = fmaf(sg, fg.x + fg.y, ag[r]);
-          au[r] = fmaf(su, fu.x + fu.y, au[r]);
+          const float2 fg0 = __half22float2(hg0), fu0 = __half22float2(hu0);
+          const float2 fg1 = __half22float2(hg1), fu1 = __half22float2(hu1);
+          ag[r] = fmaf(sg, (fg0.x + fg0.y) + (fg1.x + fg1.y), ag[r]);
+          au[r] = fmaf(su, (fu0.x + fu0.y) + (fu1.x + fu1.y), au[r]);
         }
       }
     }
@@ -264,78 +341,123 @@ __device__ __forceinline__ void gu_item(const Params& p, const GuChunk& ch, int 
   }
 }
 
-// Down item: output rows [a, a+cnt) of the chunk, every pair of the expert.
-// h (fp32, L2) is rescaled by 2^t per pair so max|h| maps to <= 2^9 and
-// converted to f16; each f16 partial sums 8 products of E2M1 (<= 6) by
-// |h'| <= 2^9 (<= 24576, no overflow) before the fp32 combine.
-__device__ __forceinline__ void d_item(const Params& p, const DChunk& ch, int a, int cnt, int pb, int pe,
-                                       float* dsm, int rpc) {
+// Power-of-two rescale that maps max|h| of one pair vector below 2^9, so
+// f16 partial sums of 8 E2M1 x h' products stay below 8*6*2^9 = 24576.
+__device__ __forceinline__ int h_rescale_exp(float mx) {
+  int ex = 0;
+  if (mx > 0.f) frexpf(mx, &ex);  // mx in [2^(ex-1), 2^ex)
+  return min(126, 9 - ex);
+}
+
+// Stage h of the pairs [pb, pe) of one expert (pe - pb <= kHPairs) into
+// shared memory as f16, each pair vector rescaled by 2^t, with 2^-t kept in
+// hscale. One warp; h is read from L2 (written by other CTAs).
+__device__ __forceinline__ void stage_h(const Params& p, int pb, int pe, __half2* hbuf, float* hscale) {
+  const int lane = threadIdx.x & 31;
+  const int I = p.I;
+  for (int pp = pb; pp < pe; ++pp) {
+    const int j = pp - pb;
+    const uint4* hp = reinterpret_cast<const uint4*>(p.ws.h + (size_t)pp * I);
+    float mx = 0.f;
+    for (int q = lane; q < I / 4; q += 32) {
+      const uint4 v = ld_cg_u4(hp + q);
+      mx = fmaxf(mx, fmaxf(fmaxf(fabsf(__uint_as_float(v.x)), fabsf(__uint_as_float(v.y))),
+                           fmaxf(fabsf(__uint_as_float(v.z)), fabsf(__uint_as_float(v.w)))));
+    }
+    const int t = h_rescale_exp(warp_max(mx));
+    const float up = ldexpf(1.f, t);
+    __half2* dst = hbuf + (size_t)j * (I / 2);
+    for (int q = lane; q < I / 4; q += 32) {
+      const uint4 v = ld_cg_u4(hp + q);
+      dst[2 * q] = __floats2half2_rn(__uint_as_float(v.x) * up, __uint_as_float(v.y) * up);
+      dst[2 * q + 1] = __floats2half2_rn(__uint_as_float(v.z) * up, __uint_as_float(v.w) * up);
+    }
+    if (lane == 0) hscale[j] = ldexpf(1.f, -t);
+  }
+}
+
+// Down rows [a, a+cnt) of one chunk for one pair, given the lane's block of
+// the pair's rescaled h (h2, 16 f16x2) and its inverse scale; accumulates
+// into dsm[pp][row] (fresh when `first`).
+__device__ __forceinline__ void d_rows(const Params& p, const DChunk& ch, int a, int cnt, int blk, const uint32_t* h2,
+                                       float down, float* dsm_pp, bool first) {
   const int lane = threadIdx.x & 31;
   const int I = p.I, nblk = I / 32;
+  for (int r = 0; r < cnt; ++r) {
+    const int row = a + r;
+    float part = 0.f;
+    if (blk < nblk) {
+      const uint4 c = *reinterpret_cast<const uint4*>(ch.c + (size_t)row * (I / 2) + blk * 16);
+      const float sc = e8m0_to_f32(ch.s[(size_t)row * (I / 32) + blk]);
+      const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
+      __half2 acc0 = __float2half2_rn(0.f), acc1 = acc0;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint32_t w[4];
+        e2m1x8_to_f16x2x4(cw[q], w);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const __half2 wv = *reinterpret_cast<const __half2*>(&w[j]);
+          const __half2 hv = *reinterpret_cast<const __half2*>(&h2[q * 4 + j]);
+          if (q < 2) acc0 = __hfma2(wv, hv, acc0); else acc1 = __hfma2(wv, hv, acc1);
+        }
+      }
+      const float2 f0 = __half22float2(acc0), f1 = __half22float2(acc1);
+      part = sc * ((f0.x + f0.y) + (f1.x + f1.y));
+    }
+    part = warp_sum(part);
+    if (lane == 0) dsm_pp[row] = (first ? 0.f : dsm_pp[row]) + part * down;
+  }
+}
+
+// Down item: rows [a, a+cnt) for every pair of the expert; h from the staged
+// shared-memory copy when the expert has at most `hpairs` pairs, else read
+// and rescaled here from L2.
+__device__ __forceinline__ void d_item(const Params& p, const DChunk& ch, int a, int cnt, int pb, int pe,
+                                       const __half2* hbuf, const float* hscale, int hpairs, float* dsm, int rpc) {
+  const int lane = threadIdx.x & 31;
+  const int I = p.I, nblk = I / 32;
+  const bool staged = (pe - pb) <= hpairs;
   for (int pp = pb; pp < pe; ++pp) {
-    const float* hp = p.ws.h + (size_t)pp * I;
     for (int b0 = 0; b0 < nblk; b0 += 32) {
-      // (I <= 1024 covers every shape with one pass; larger I loops)
       const int blk = b0 + lane;
-      float hv[32];
-      float mx = 0.f;
-      if (blk < nblk) {
+      uint32_t h2[16];
+      float down;
+      if (staged) {
+        const uint4* src = reinterpret_cast<const uint4*>(hbuf + (size_t)(pp - pb) * (I / 2)) + blk * 4;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint4 v = (blk < nblk) ? src[q] : make_uint4(0u, 0u, 0u, 0u);
+          h2[4 * q] = v.x; h2[4 * q + 1] = v.y; h2[4 * q + 2] = v.z; h2[4 * q + 3] = v.w;
+        }
+        down = hscale[pp - pb];
+      } else {
+        const float* hp = p.ws.h + (size_t)pp * I;
+        float hv[32];
+        float mx = 0.f;
 #pragma unroll
         for (int t = 0; t < 8; ++t) {
-          const uint4 q = ld_cg_u4(hp + blk * 32 + t * 4);
-          hv[4 * t] = __uint_as_float(q.x);
-          hv[4 * t + 1] = __uint_as_float(q.y);
-          hv[4 * t + 2] = __uint_as_float(q.z);
-          hv[4 * t + 3] = __uint_as_float(q.w);
+          const uint4 q = (blk < nblk) ? ld_cg_u4(hp + blk * 32 + t * 4) : make_uint4(0u, 0u, 0u, 0u);
+          hv[4 * t] = __uint_as_float(q.x); hv[4 * t + 1] = __uint_as_float(q.y);
+          hv[4 * t + 2] = __uint_as_float(q.z); hv[4 * t + 3] = __uint_as_float(q.w);
         }
-#pragma unroll
-        for (int t = 0; t < 32; ++t) mx = fmaxf(mx, fabsf(hv[t]));
-      } else {
-#pragma unroll
-        for (int t = 0; t < 32; ++t) hv[t] = 0.f;
-      }
-      // one scale for the whole pair vector: max over all lanes and passes
-      // (single pass when I <= 1024)
-      mx = warp_max(mx);
-      int ex = 0;
-      if (mx > 0.f) frexpf(mx, &ex);  // mx in [2^(ex-1), 2^ex)
-      const int t = min(126, 9 - ex);   // max|h * 2^t| < 2^9
-      const float up = ldexpf(1.f, t), down = ldexpf(1.f, -t);
-      uint32_t h2[16];
-#pragma unroll
-      for (int q = 0; q < 16; ++q) {
-        __half2 v = __floats2half2_rn(hv[2 * q] * up, hv[2 * q + 1] * up);
-        h2[q] = *reinterpret_cast<uint32_t*>(&v);
-      }
-      for (int r = 0; r < cnt; ++r) {
-        const int row = a + r;
-        float part = 0.f;
-        if (blk < nblk) {
-          const uint4 c = *reinterpret_cast<const uint4*>(ch.c + (size_t)row * (I / 2) + blk * 16);
-          const float sc = e8m0_to_f32(ch.s[(size_t)row * (I / 32) + blk]);
-          const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
-          __half2 acc0 = __float2half2_rn(0.f), acc1 = __float2half2_rn(0.f);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            uint32_t w[4];
-            e2m1x8_to_f16x2x4(cw[q], w);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const __half2 wv = *reinterpret_cast<const __half2*>(&w[j]);
-              const __half2 hvv = *reinterpret_cast<const __half2*>(&h2[q * 4 + j]);
-              if (q < 2) acc0 = __hfma2(wv, hvv, acc0); else acc1 = __hfma2(wv, hvv, acc1);
-            }
-          }
-          const float2 f0 = __half22float2(acc0), f1 = __half22float2(acc1);
-          part = sc * ((f0.x + f0.y) + (f1.x + f1.y));
+        // the rescale must cover the whole vector: reduce over all passes
+        for (int b1 = 0; b1 < nblk; b1 += 32) {
+          const int bk = b1 + lane;
+          if (bk < nblk)
+            for (int t = 0; t < 32; ++t) mx = fmaxf(mx, fabsf(__ldcg(hp + bk * 32 + t)));
         }
-        part = warp_sum(part);
-        if (lane == 0) {
-          float* dst = dsm + (size_t)pp * rpc + row;
-          *dst = (b0 == 0 ? 0.f : *dst) + part * down;
+        const int t = h_rescale_exp(warp_max(mx));
+        const float up = ldexpf(1.f, t);
+        down = ldexpf(1.f, -t);
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+          __half2 v = __floats2half2_rn(hv[2 * q] * up, hv[2 * q + 1] * up);
+          h2[q] = *reinterpret_cast<uint32_t*>(&v);
         }
-        __syncwarp();
       }
+      d_rows(p, ch, a, cnt, blk, h2, down, dsm + (size_t)pp * rpc, b0 == 0);
+      __syncwarp();
     }
   }
 }
@@ -348,57 +470,84 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
   const int H = p.H, I = p.I, E = p.E, K = p.K, M = p.M;
 
   uint64_t* full_gu = reinterpret_cast<uint64_t*>(smem + pl.o_bar);
-  uint64_t* empty_gu = full_gu + pl.ns_gu;
-  uint64_t* full_d = empty_gu + pl.ns_gu;
-  uint64_t* empty_d = full_d + pl.ns_d;
-  uint64_t* wr_bar = empty_d + pl.ns_d;
+  uint64_t* empty_gu = full_gu + kMaxSlots;
+  uint64_t* full_d = empty_gu + kMaxSlots;
+  uint64_t* empty_d = full_d + kMaxSlots;
+  uint64_t* h_bar = empty_d + kMaxSlots;
+  uint64_t* wr_bar = h_bar + kMaxSlots;
+  // items finished per ring slot (all uses): an item of use k waits until use
+  // k-1 of its slot is fully consumed before any parity wait, so a parity
+  // wait can never see a barrier two phases behind and pass early
+  unsigned* done_gu = reinterpret_cast<unsigned*>(wr_bar + 1);
+  unsigned* done_d = done_gu + kMaxSlots;
   float* s_amax = reinterpret_cast<float*>(smem + pl.o_misc);  // [32]
   float* s_xs = s_amax + kMaxTokens;                           // [32] per-token scales
   float* s_red = s_xs + kMaxTokens;                            // [kFusedWarps][4]
-  int* s_int = reinterpret_cast<int*>(s_red + kFusedWarps * 4);  // [0] U, [1] epoch
+  int* s_int = reinterpret_cast<int*>(s_red + kFusedWarps * 4);  // [0] U, [1] epoch, [2] work queue head
   int* s_ids = reinterpret_cast<int*>(smem + pl.o_ids);
   float* s_w = reinterpret_cast<float*>(smem + pl.o_w);
   int* s_pm = reinterpret_cast<int*>(smem + pl.o_pm);
   int* s_ppos = reinterpret_cast<int*>(smem + pl.o_ppos);
   int* s_union = reinterpret_cast<int*>(smem + pl.o_union);
   int* s_poff = reinterpret_cast<int*>(smem + pl.o_poff);
-  int* s_cnt = reinterpret_cast<int*>(smem + pl.o_cnt);  // [E] scratch, then per-union counters
+  int* s_cnt = reinterpret_cast<int*>(smem + pl.o_cnt);  // [E] union scratch, then per-entry item counters
   uint8_t* act = smem + pl.o_act;
   float* dsm = reinterpret_cast<float*>(smem + pl.o_dsm);
+  uint8_t* hstage = smem + pl.o_h;
   uint8_t* ring_gu = smem + pl.o_ring_gu;
   uint8_t* ring_d = smem + pl.o_ring_d;
-  float* wr_s = reinterpret_cast<float*>(ring_gu);  // router rows alias the ring
+  float* wr_s = reinterpret_cast<float*>(ring_gu);       // router rows (routing phase only)
+  float* s_logit = reinterpret_cast<float*>(ring_gu);    // gathered logits (after the router rows)
+  uint4* x_s = reinterpret_cast<uint4*>(ring_d);         // staged bf16 x (routing phase only)
 
   const int e0 = (int)((long long)E * b / G), e1 = (int)((long long)E * (b + 1) / G), ne = e1 - e0;
   // this CTA's share of every union expert (independent of the routing)
   const int n0 = (int)((long long)I * b / G), nr = (int)((long long)I * (b + 1) / G) - n0;
   const int r0 = (int)((long long)H * b / G), nrd = (int)((long long)H * (b + 1) / G) - r0;
-  const int gu_items = (nr + kGuRowsPerItem - 1) / kGuRowsPerItem;  // items per gate/up chunk
-  const int d_items = (nrd + kDownRowsPerItem - 1) / kDownRowsPerItem;
-  const uint64_t pol = l2_evict_first_policy();
+  const int gu_items = (nr > 0) ? (nr + kGuRowsPerItem - 1) / kGuRowsPerItem : 0;  // per expert
+  const int d_items = (nrd > 0) ? (nrd + kDownRowsPerItem - 1) / kDownRowsPerItem : 0;
 
   if (tid == 0) {
     for (int i = 0; i < pl.ns_gu; ++i) { mbar_init(full_gu + i, 1); mbar_init(empty_gu + i, max(1, gu_items)); }
-    for (int i = 0; i < pl.ns_d; ++i) { mbar_init(full_d + i, 1); mbar_init(empty_d + i, max(1, d_items)); }
+    for (int i = 0; i < pl.ns_d; ++i) {
+      mbar_init(full_d + i, 1);
+      mbar_init(empty_d + i, max(1, d_items));
+      mbar_init(h_bar + i, 1);
+    }
     mbar_init(wr_bar, 1);
+    for (int i = 0; i < kMaxSlots; ++i) done_gu[i] = done_d[i] = 0u;
     fence_mbar_init();
     if (ne > 0) {
       mbar_expect_tx(wr_bar, (unsigned)(ne * H * 4));
-      tma_load_1d(wr_s, p.wr + (size_t)e0 * H, (unsigned)(ne * H * 4), wr_bar, pol);
+      tma_load_1d(wr_s, p.wr + (size_t)e0 * H, (unsigned)(ne * H * 4), wr_bar);
     }
   }
   // Everything above is independent of the previous kernel on the stream.
   pdl_wait();
-  if (tid == 0) s_int[1] = (int)(ld_relaxed_u32(fw.epoch) + 1u);
+  if (tid == 0) {
+    s_int[1] = (int)(ld_relaxed_u32(fw.epoch) + 1u);
+    s_int[2] = 0;
+  }
+  unsigned* s_amax_u = reinterpret_cast<unsigned*>(s_amax);
+  if (tid < M) s_amax_u[tid] = 0u;
   __syncthreads();
   const unsigned epoch = (unsigned)s_int[1];
 
-  // ---- A1: per-token amax and E4M3 codes into shared memory (every CTA)
-  for (int m = warp; m < M; m += kFusedWarps) {
-    const uint4* xm = reinterpret_cast<const uint4*>(p.x + (size_t)m * H);
+  // ---- A1: per-token amax (unsigned max of |x| bit patterns) and, when it
+  //          fits, a shared-memory copy of x for the router
+  {
+    const uint4* x16 = reinterpret_cast<const uint4*>(p.x);
+    int mcur = -1;
     float a = 0.f;
-    for (int i = lane; i < H / 8; i += 32) {
-      const uint4 v = ld_cg_u4(xm + i);
+    for (int i = tid; i < M * H / 8; i += kFusedThreads) {
+      const int m = (i * 8) / H;
+      if (m != mcur) {
+        if (mcur >= 0) atomicMax(&s_amax_u[mcur], __float_as_uint(a));
+        mcur = m;
+        a = 0.f;
+      }
+      const uint4 v = __ldcg(x16 + i);
+      if (pl.x_staged) x_s[i] = v;
       const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
@@ -406,20 +555,21 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
         a = fmaxf(a, fmaxf(fabsf(f.x), fabsf(f.y)));
       }
     }
-    a = warp_max(a);
-    if (lane == 0) {
-      s_amax[m] = a;
-      s_xs[m] = (a == 0.f) ? 1.f : __fdiv_rn(a, 448.f);
-    }
+    if (mcur >= 0) atomicMax(&s_amax_u[mcur], __float_as_uint(a));
   }
   __syncthreads();
+  const uint4* xsrc = pl.x_staged ? x_s : reinterpret_cast<const uint4*>(p.x);
+  if (tid < M) {
+    const float a = s_amax[tid];
+    s_xs[tid] = (a == 0.f) ? 1.f : __fdiv_rn(a, 448.f);
+  }
   for (int i = tid; i < M * H / 8; i += kFusedThreads) {
     const int m = (i * 8) / H;
     const float a = s_amax[m];
     uint2 out = make_uint2(0u, 0u);
     if (a != 0.f) {
       const float inv = __fdiv_rn(448.f, a);
-      const uint4 v = ld_cg_u4(reinterpret_cast<const uint4*>(p.x) + i);
+      const uint4 v = pl.x_staged ? xsrc[i] : __ldcg(xsrc + i);
       const uint32_t w[4] = {v.x, v.y, v.z, v.w};
       uint32_t q[2] = {0u, 0u};
 #pragma unroll
@@ -433,9 +583,10 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
     *reinterpret_cast<uint2*>(act + (size_t)i * 8) = out;
     if (b == 0 && p.out_xq) *reinterpret_cast<uint2*>(p.out_xq + (size_t)i * 8) = out;
   }
+  __syncthreads();
   if (b == 0 && p.out_xscale && tid < M) p.out_xscale[tid] = s_xs[tid];
 
-  // ---- A2: logits of this CTA's router rows, published with the epoch tag
+  // ---- A2: logits of this CTA's router rows
   if (ne > 0) mbar_wait(wr_bar, 0, p);
   for (int el = 0; el < ne; ++el) {
     const float4* wrow = reinterpret_cast<const float4*>(wr_s + (size_t)el * H);
@@ -446,10 +597,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
           if (m0 + t < M) {
-            uint2 xv;
-            asm volatile("ld.global.cg.v2.u32 {%0,%1}, [%2];"
-                         : "=r"(xv.x), "=r"(xv.y)
-                         : "l"(reinterpret_cast<const uint2*>(p.x + (size_t)(m0 + t) * H) + i));
+            const uint2* xrow = reinterpret_cast<const uint2*>(xsrc) + (size_t)(m0 + t) * (H / 4);
+            const uint2 xv = pl.x_staged ? xrow[i] : __ldcg(xrow + i);
             const float2 x01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xv.x));
             const float2 x23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xv.y));
             acc[t] = fmaf(x01.x, wv.x, acc[t]);
@@ -469,39 +618,31 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
       if (tid < 4 && m0 + tid < M) {
         float s = 0.f;
         for (int w = 0; w < kFusedWarps; ++w) s += s_red[w * 4 + tid];
-        const unsigned long long word =
-            ((unsigned long long)epoch << 32) | (unsigned long long)__float_as_uint(s);
-        st_relaxed_u64(fw.logits64 + (size_t)(m0 + tid) * E + e0 + el, word);
+        fw.logits[(size_t)(m0 + tid) * E + e0 + el] = s;
       }
       __syncthreads();
     }
   }
+  __syncthreads();
+  // grid-wide: every CTA's logits are in L2 once the router count reaches
+  // epoch * G (the last arrival publishes the epoch to the flag copies)
+  if (tid == 0) {
+    grid_arrive(fw.route_cnt, fw.route_done, (unsigned long long)epoch * G, epoch);
+    grid_wait(fw.route_done, b, p.force_stall ? epoch + 0x40000000u : epoch, p);
+  }
   pdl_launch_dependents();
+  __syncthreads();
 
-  // ---- A3: every CTA reads all logits (spinning on the epoch tags) and
-  //          selects the top-k of each token
-  const unsigned want = p.force_stall ? epoch + 0x40000000u : epoch;
+  // ---- A3: gather all M*E logits into shared memory; one warp per token
+  //          selects the top-k (ties to the lower index) and its softmax
+  for (int i = tid; i < M * E; i += kFusedThreads) s_logit[i] = __ldcg(fw.logits + i);
+  __syncthreads();
   for (int m = warp; m < M; m += kFusedWarps) {
-    const unsigned long long* lrow = fw.logits64 + (size_t)m * E;
     float v[kMaxExperts / 32];
 #pragma unroll
     for (int j = 0; j < kMaxExperts / 32; ++j) {
       const int e = lane + 32 * j;
-      v[j] = 0.f;
-      if (e < E) {
-        unsigned long long wd = ld_relaxed_u64(lrow + e);
-        if ((unsigned)(wd >> 32) != want) {
-          const long long t0 = clock64();
-          do {
-            wd = ld_relaxed_u64(lrow + e);
-            if (clock64() - t0 > p.spin_limit) {
-              atomicOr(p.ws.ctrl, kStatusTimeout);
-              break;
-            }
-          } while ((unsigned)(wd >> 32) != want);
-        }
-        v[j] = __uint_as_float((unsigned)wd);
-      }
+      v[j] = (e < E) ? s_logit[m * E + e] : 0.f;
     }
     uint32_t taken = 0;
     float sel_v = 0.f, top = 0.f;
@@ -545,13 +686,14 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
   }
   __syncthreads();
 
-  // ---- A4: expert union (ascending ids) and the pairs of each entry
+  // ---- A4: expert union (ascending ids) and the (token, slot) pairs of each
+  //          entry in (token, slot) order; one warp, no block barriers
   const int np = M * K;
-  for (int e = tid; e < E; e += kFusedThreads) s_cnt[e] = 0;
-  __syncthreads();
-  for (int i = tid; i < np; i += kFusedThreads) atomicAdd(&s_cnt[s_ids[i]], 1);
-  __syncthreads();
   if (warp == 0) {
+    for (int e = lane; e < E; e += 32) s_cnt[e] = 0;
+    __syncwarp();
+    for (int i = lane; i < np; i += 32) atomicAdd(&s_cnt[s_ids[i]], 1);
+    __syncwarp();
     const int per = (E + 31) / 32;
     const int ea = min(E, lane * per), eb = min(E, ea + per);
     int nz = 0, cs = 0;
@@ -565,6 +707,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
     }
     nz_ex -= nz;
     cs_ex -= cs;
+    __syncwarp();
     for (int e = ea; e < eb; ++e) {
       const int c = s_cnt[e];
       if (c > 0) {
@@ -573,86 +716,98 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
         ++nz_ex;
         cs_ex += c;
       }
-      s_cnt[e] = cs_ex - c;
+      s_cnt[e] = cs_ex - c;  // first pair position of expert e
     }
     if (lane == 31) {
       s_poff[nz_ex] = cs_ex;
       s_int[0] = nz_ex;
     }
+    __syncwarp();
+    // stable placement: rank within each 32-pair batch by matching experts
+    for (int base = 0; base < np; base += 32) {
+      const int i = base + lane;
+      const int e = (i < np) ? s_ids[i] : -1 - lane;
+      const unsigned same = __match_any_sync(0xffffffffu, e);
+      const int rank = __popc(same & ((1u << lane) - 1u));
+      int pos = 0;
+      if (i < np) {
+        pos = s_cnt[e] + rank;
+        s_pm[pos] = i / K;
+        s_ppos[i] = pos;
+      }
+      __syncwarp();
+      if (i < np && rank == 0) s_cnt[e] += __popc(same);
+      __syncwarp();
+    }
+    const int U = s_int[0];
+    __syncwarp();
+    for (int u = lane; u < U; u += 32) s_cnt[u] = 0;  // per-entry gate/up item counters
   }
   __syncthreads();
-  for (int i = tid; i < np; i += kFusedThreads) {
-    const int e = s_ids[i];
-    int before = 0;
-    for (int j = 0; j < i; ++j) before += (s_ids[j] == e);
-    const int pos = s_cnt[e] + before;
-    s_pm[pos] = i / K;
-    s_ppos[i] = pos;
-  }
   const int U = s_int[0];
-  __syncthreads();
-  // s_cnt is reused below as per-union-entry completion counters
-  for (int u = tid; u < U; u += kFusedThreads) s_cnt[u] = 0;
-
-  __syncthreads();
 
   if (warp == 0) {
-    // ---------------- producer
+    // ---------------- producer: gate/up then down slice of each entry, in
+    //                  the order the consumers take them
     if (lane == 0) {
-      // the router rows were read through the generic proxy from ring_gu;
-      // order those reads before the async-proxy (TMA) writes below
+      // ring_gu and ring_d were read and written through the generic proxy
+      // during routing; order that before the async-proxy (TMA) writes
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      if (nr > 0) {
-        for (int u = 0; u < U; ++u) {
+      for (int u = 0; u < U; ++u) {
+        const int e = s_union[u];
+        if (nr > 0) {
           const int slot = u % pl.ns_gu, use = u / pl.ns_gu;
           if (use > 0) mbar_wait(empty_gu + slot, (use - 1) & 1, p);
           uint8_t* sp = ring_gu + (size_t)slot * pl.slot_gu;
           GuChunk ch;
           size_t ga0, ua0;
           unsigned gn, un;
-          const int e = s_union[u];
           const unsigned bytes = gu_layout(p, e, n0, nr, sp, &ch, &ga0, &gn, &ua0, &un);
           mbar_expect_tx(full_gu + slot, bytes);
           const size_t grow = (size_t)e * 2 * I + n0, urow = grow + I;
           const unsigned codes = (unsigned)(nr * H / 2);
-          tma_load_1d(sp, p.w13c + grow * (H / 2), codes, full_gu + slot, pol);
-          tma_load_1d(sp + codes, p.w13c + urow * (H / 2), codes, full_gu + slot, pol);
-          tma_load_1d(sp + 2 * codes, p.w13s + ga0, gn, full_gu + slot, pol);
-          tma_load_1d(sp + 2 * codes + gn, p.w13s + ua0, un, full_gu + slot, pol);
+          tma_load_1d(sp, p.w13c + grow * (H / 2), codes, full_gu + slot);
+          tma_load_1d(sp + codes, p.w13c + urow * (H / 2), codes, full_gu + slot);
+          tma_load_1d(sp + 2 * codes, p.w13s + ga0, gn, full_gu + slot);
+          tma_load_1d(sp + 2 * codes + gn, p.w13s + ua0, un, full_gu + slot);
         }
-      }
-      if (nrd > 0) {
-        for (int u = 0; u < U; ++u) {
+        if (nrd > 0) {
           const int slot = u % pl.ns_d, use = u / pl.ns_d;
           if (use > 0) mbar_wait(empty_d + slot, (use - 1) & 1, p);
           uint8_t* sp = ring_d + (size_t)slot * pl.slot_d;
           DChunk ch;
           size_t sa0;
           unsigned sn;
-          const int e = s_union[u];
           const unsigned bytes = d_layout(p, e, r0, nrd, sp, &ch, &sa0, &sn);
           mbar_expect_tx(full_d + slot, bytes);
           const unsigned codes = (unsigned)(nrd * I / 2);
-          tma_load_1d(sp, p.w2c + ((size_t)e * H + r0) * (I / 2), codes, full_d + slot, pol);
-          tma_load_1d(sp + codes, p.w2s + sa0, sn, full_d + slot, pol);
+          tma_load_1d(sp, p.w2c + ((size_t)e * H + r0) * (I / 2), codes, full_d + slot);
+          tma_load_1d(sp + codes, p.w2s + sa0, sn, full_d + slot);
         }
       }
     }
     return;
   }
 
-  // ---------------- consumers (warps 1..15)
-  const int c = warp - 1;
-  const int n_gu = (nr > 0) ? U * gu_items : 0;
-  const int n_d = (nrd > 0) ? U * d_items : 0;
-  if (nr == 0) {
-    // nothing to compute for gate/up: publish completion for every entry
-    for (int u = c * 32 + lane; u < U; u += kConsumers * 32) st_relaxed_u32(fw.guflag + (size_t)u * G + b, epoch);
+  // ---------------- consumers (warps 1..15): one in-order work queue
+  //   entry u contributes gu_items gate/up items, then d_items down items
+  const int per_u = gu_items + d_items;
+  const int total = U * per_u;
+  const unsigned long long tgt = (unsigned long long)epoch * G;
+  if (gu_items == 0 && warp == 1 && lane == 0) {
+    // no gate/up rows here: this CTA's part of every entry is trivially done
+    for (int u = 0; u < U; ++u) grid_arrive(fw.gu_cnt + u, fw.gu_done + (size_t)u * kFlagCopies * kFlagStride, tgt, epoch);
   }
-  for (int it = c; it < n_gu + n_d; it += kConsumers) {
-    if (it < n_gu) {
-      const int u = it / gu_items, g = it % gu_items;
+  for (;;) {
+    int it = 0;
+    if (lane == 0) it = atomicAdd(&s_int[2], 1);
+    it = __shfl_sync(0xffffffffu, it, 0);
+    if (it >= total) break;
+    const int u = it / per_u, g = it % per_u;
+    if (g < gu_items) {
       const int slot = u % pl.ns_gu, use = u / pl.ns_gu;
+      if (use > 0 && lane == 0) smem_count_wait(done_gu + slot, (unsigned)(use * gu_items), p);
+      __syncwarp();
       mbar_wait(full_gu + slot, use & 1, p);
       GuChunk ch;
       size_t ga0, ua0;
@@ -663,43 +818,47 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(empty_gu + slot);
-        __threadfence();
-        const int done = atomicAdd(&s_cnt[u], 1) + 1;
-        if (done == gu_items) {
-          __threadfence();
-          st_relaxed_u32(fw.guflag + (size_t)u * G + b, epoch);
-        }
+        atomicAdd(done_gu + slot, 1u);
+        // acq_rel at CTA scope: the warp completing the entry sees every
+        // other warp's h stores, then releases them GPU-wide
+        const unsigned done = atom_add_acqrel_cta_smem(reinterpret_cast<unsigned*>(s_cnt + u), 1u) + 1u;
+        if ((int)done == gu_items)
+          grid_arrive(fw.gu_cnt + u, fw.gu_done + (size_t)u * kFlagCopies * kFlagStride, tgt, epoch);
       }
       __syncwarp();
     } else {
-      const int id = it - n_gu;
-      const int u = id / d_items, g = id % d_items;
-      // wait until every CTA has finished gate/up of union entry u
-      const unsigned* fl = fw.guflag + (size_t)u * G;
-      {
-        const long long t0 = clock64();
-        bool ok;
-        do {
-          ok = true;
-          for (int j = lane; j < G; j += 32) ok &= (ld_relaxed_u32(fl + j) == epoch);
-          ok = __all_sync(0xffffffffu, ok);
-          if (!ok && clock64() - t0 > p.spin_limit) {
-            if (lane == 0) atomicOr(p.ws.ctrl, kStatusTimeout);
-            break;
-          }
-        } while (!ok);
-        __threadfence();
-      }
+      const int gd = g - gu_items;
       const int slot = u % pl.ns_d, use = u / pl.ns_d;
+      const int pb = s_poff[u], pe = s_poff[u + 1];
+      __half2* hbuf = reinterpret_cast<__half2*>(hstage + (size_t)slot * pl.hslot);
+      float* hscale = reinterpret_cast<float*>(hstage + (size_t)slot * pl.hslot + (size_t)pl.hpairs * I * 2);
+      // every down item of the slot's previous use is finished (so its
+      // staged h and data may be replaced, and parity waits are unambiguous)
+      if (use > 0 && lane == 0) smem_count_wait(done_d + slot, (unsigned)(use * d_items), p);
+      __syncwarp();
+      if (gd == 0) {
+        // first down item of the entry: wait for gate/up of the entry on all
+        // CTAs, then stage h once for the CTA
+        if (lane == 0) grid_wait(fw.gu_done + (size_t)u * kFlagCopies * kFlagStride, b, epoch, p);
+        __syncwarp();
+        if (pe - pb <= pl.hpairs) stage_h(p, pb, pe, hbuf, hscale);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(h_bar + slot);
+      } else {
+        mbar_wait(h_bar + slot, use & 1, p);
+      }
       mbar_wait(full_d + slot, use & 1, p);
       DChunk ch;
       size_t sa0;
       unsigned sn;
       d_layout(p, s_union[u], r0, nrd, ring_d + (size_t)slot * pl.slot_d, &ch, &sa0, &sn);
-      const int a = g * kDownRowsPerItem, cnt = min(kDownRowsPerItem, nrd - a);
-      d_item(p, ch, a, cnt, s_poff[u], s_poff[u + 1], dsm, pl.rpc_max);
+      const int a = gd * kDownRowsPerItem, cnt = min(kDownRowsPerItem, nrd - a);
+      d_item(p, ch, a, cnt, pb, pe, hbuf, hscale, pl.hpairs, dsm, pl.rpc_max);
       __syncwarp();
-      if (lane == 0) mbar_arrive(empty_d + slot);
+      if (lane == 0) {
+        mbar_arrive(empty_d + slot);
+        atomicAdd(done_d + slot, 1u);
+      }
     }
   }
   consumers_sync();
@@ -711,7 +870,11 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
     for (int s = 0; s < K; ++s) acc = fmaf(s_w[m * K + s], dsm[(size_t)s_ppos[m * K + s] * pl.rpc_max + rl], acc);
     p.y[(size_t)m * H + r0 + rl] = __float2bfloat16_rn(acc);
   }
-  if (b == 0 && ct == 0) st_relaxed_u32(fw.epoch, epoch);
+  if (b == 0 && ct == 0) {
+    // keep every entry's counter at epoch * G for the next launch
+    for (int u = U; u < pl.max_union; ++u) atom_add_acqrel_u64(fw.gu_cnt + u, (unsigned long long)G);
+    st_relaxed_u32(fw.epoch, epoch);
+  }
 }
 
 }  // namespace moe

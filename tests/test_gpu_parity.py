@@ -77,6 +77,18 @@ def test_zipf_sweep_sampled(M):
     compare(L, split, L.oracle(tokens=sample), tokens=sample)
 
 
+@pytest.mark.parametrize("M,mode", [(1, "gap"), (2, "zipf"), (4, "gap"), (3, "shared")])
+def test_deep_ring_reuse(M, mode):
+    """A context sized for 32 tokens leaves 4 ring slots, so every slot is
+    reused several times per step even at M=1; every token checked in full."""
+    L = Layer(2560, 768, 256, 8, M, seed=2, mode=mode)
+    ctx = L.make_ctx(0, max_tokens=32)
+    got = L.run(ctx)
+    compare(L, got, L.oracle())
+    again = L.run(ctx)
+    assert torch.equal(got["y"], again["y"])
+
+
 def test_max_tokens_all_checked_small_layer():
     L = Layer(256, 64, 16, 4, 32, seed=4, mode="gap")
     got = L.run(L.make_ctx(0))
