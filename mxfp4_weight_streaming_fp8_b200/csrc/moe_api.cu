@@ -70,7 +70,7 @@ bool make_plan(const moe_config& c, int sm_count, size_t smem_limit, moe::FusedP
   size_t off = 0;
   auto take = [&](size_t bytes, size_t a) { off = align_up(off, a); size_t o = off; off += bytes; return o; };
   pl->o_bar = (int)take((5 * kMaxSlots + 1) * 8 + 2 * kMaxSlots * 4, 16);
-  pl->o_misc = (int)take((2 * moe::kMaxTokens + 4 * moe::kFusedWarps + 8) * 4, 16);
+  pl->o_misc = (int)take((2 * moe::kMaxTokens + moe::kFusedWarps * moe::kMaxRowsPerCta * 4 + 8) * 4, 16);
   pl->o_ids = (int)take(NP * 4, 16);
   pl->o_w = (int)take(NP * 4, 16);
   pl->o_pm = (int)take(NP * 4, 16);
@@ -104,6 +104,7 @@ bool make_plan(const moe_config& c, int sm_count, size_t smem_limit, moe::FusedP
   // ring_gu also holds the router rows of the CTA and then the gathered
   // logits [M][E] fp32 between routing and the first weight chunk
   pl->wr_bytes_max = (int)(((E + G - 1) / G) * H * 4);
+  if ((E + G - 1) / G > (size_t)moe::kMaxRowsPerCta) return false;  // router rows per CTA
   const size_t staged = std::max((size_t)pl->wr_bytes_max, MM * E * 4);
   const size_t ring_gu_bytes = align_up(std::max(ns_gu * (size_t)pl->slot_gu, staged), 128);
   pl->o_ring_gu = (int)off;
@@ -197,9 +198,7 @@ moe_status moe_create(const moe_config* cfg, moe_ctx** out) {
   const size_t o_h = take(NP * I * sizeof(float));
   const size_t o_flog = take(MM * E * sizeof(float));
   const size_t o_rcnt = take(sizeof(unsigned long long));
-  const size_t o_rdone = take(moe::kFlagCopies * moe::kFlagStride * sizeof(unsigned));
   const size_t o_gcnt = take(UMAX * sizeof(unsigned long long));
-  const size_t o_gdone = take(UMAX * moe::kFlagCopies * moe::kFlagStride * sizeof(unsigned));
   ctx->ws_bytes = off;
   if (cudaMalloc(&ctx->ws_base, ctx->ws_bytes) != cudaSuccess) {
     cudaGetLastError();
@@ -228,9 +227,7 @@ moe_status moe_create(const moe_config* cfg, moe_ctx** out) {
   w.h = reinterpret_cast<float*>(b + o_h);
   ctx->fws.logits = reinterpret_cast<float*>(b + o_flog);
   ctx->fws.route_cnt = reinterpret_cast<unsigned long long*>(b + o_rcnt);
-  ctx->fws.route_done = reinterpret_cast<unsigned*>(b + o_rdone);
   ctx->fws.gu_cnt = reinterpret_cast<unsigned long long*>(b + o_gcnt);
-  ctx->fws.gu_done = reinterpret_cast<unsigned*>(b + o_gdone);
   ctx->fws.epoch = w.ctrl + 5;
 
   // launch shapes

@@ -50,8 +50,9 @@ constexpr int kConsumers = kFusedWarps - 1;  // warp 0 produces
 constexpr int kGuRowsPerItem = 2;           // intermediate rows per gate/up item
 constexpr int kDownRowsPerItem = 6;         // output rows per down item
 constexpr int kHPairs = 4;                  // (token, slot) pairs of one expert whose h is staged in smem
-constexpr int kFlagCopies = 8;              // completion flags are replicated over this many L2 lines
-constexpr int kFlagStride = 32;             // u32 words between copies (one 128-byte line)
+constexpr int kGuWarps = 8;                 // consumer warps 1..8 take gate/up items
+constexpr int kDownWarps = kConsumers - kGuWarps;  // warps 9..15 take down items
+constexpr int kMaxRowsPerCta = 8;           // router rows a CTA may own (E <= 8 * G)
 constexpr int kMaxSlots = 64;
 
 // Launch-invariant plan computed on the host at moe_create.
@@ -74,9 +75,7 @@ struct FusedPlan {
 struct FusedWs {
   float* logits;                  // [maxM][E]
   unsigned long long* route_cnt;  // router arrivals; += G per launch
-  unsigned* route_done;           // [kFlagCopies * kFlagStride] epoch of the last complete router phase
   unsigned long long* gu_cnt;     // [max_union] gate/up arrivals per union entry; += G per launch
-  unsigned* gu_done;              // [max_union][kFlagCopies * kFlagStride]
   unsigned* epoch;                // launch counter
 };
 
@@ -172,29 +171,30 @@ __device__ __forceinline__ unsigned atom_add_acqrel_cta_smem(unsigned* p, unsign
   return old;
 }
 
-// Arrive on a grid-wide completion point: a monotonic counter that gains G
-// per launch. The CTA whose arrival completes the launch's count publishes
-// `epoch` to kFlagCopies flag words on separate L2 lines (release), so
-// waiters spread their polling instead of hammering one line.
-__device__ __forceinline__ void grid_arrive(unsigned long long* cnt, unsigned* done, unsigned long long target,
-                                            unsigned epoch) {
-  const unsigned long long old = atom_add_acqrel_u64(cnt, 1ull);
-  if (old + 1 == target) {
-#pragma unroll
-    for (int k = 0; k < kFlagCopies; ++k) st_release_u32(done + k * kFlagStride, epoch);
-  }
+__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.acquire.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void red_release_add_u64(unsigned long long* p, unsigned long long v) {
+  asm volatile("red.release.gpu.global.add.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
 
-// Wait (one thread) until flag copy `which` reads `want` (acquire), with a
-// growing sleep between polls; bounded by the wait budget.
-__device__ __forceinline__ void grid_wait(const unsigned* done, int which, unsigned want, const Params& p) {
-  const unsigned* f = done + (which % kFlagCopies) * kFlagStride;
-  if (ld_acquire_u32(f) == want) return;
+// Grid-wide completion points are monotonic 64-bit counters that gain G per
+// launch: a CTA arrives with a fire-and-forget release add, and a waiter
+// polls the counter with acquire loads until it reaches epoch * G. (Measured
+// on B200 with 148 CTAs: about 1.35 us per barrier. A returning acq_rel
+// atomic with a last-arriver flag took about 4.7 us; per-CTA flag words
+// polled by a warp took about 2.4 us.)
+__device__ __forceinline__ void grid_arrive(unsigned long long* cnt) { red_release_add_u64(cnt, 1ull); }
+
+// One thread waits until *cnt >= target, with a short sleep between polls;
+// bounded by the wait budget.
+__device__ __forceinline__ void grid_wait(const unsigned long long* cnt, unsigned long long target, const Params& p) {
+  if (ld_acquire_u64(cnt) >= target) return;
   const long long t0 = clock64();
-  unsigned ns = 32;
-  while (ld_acquire_u32(f) != want) {
-    __nanosleep(ns);
-    if (ns < 256) ns <<= 1;
+  while (ld_acquire_u64(cnt) < target) {
+    __nanosleep(32);
     if (clock64() - t0 > p.spin_limit) {
       atomicOr(p.ws.ctrl, kStatusTimeout);
       return;
@@ -334,8 +334,16 @@ __device__ __forceinline__ void gu_item(const Params& p, const GuChunk& ch, int 
     }
     const float s = s_xs[m];
 #pragma unroll
+    for (int o = 16; o; o >>= 1) {
+#pragma unroll
+      for (int r = 0; r < kGuRowsPerItem; ++r) {
+        ag[r] += __shfl_xor_sync(0xffffffffu, ag[r], o);
+        au[r] += __shfl_xor_sync(0xffffffffu, au[r], o);
+      }
+    }
+#pragma unroll
     for (int r = 0; r < kGuRowsPerItem; ++r) {
-      const float g = warp_sum(ag[r]) * s, u = warp_sum(au[r]) * s;
+      const float g = ag[r] * s, u = au[r] * s;
       if (lane == 0 && r < cnt) p.ws.h[(size_t)pp * p.I + n0 + a + r] = g / (1.f + expf(-g)) * u;
     }
   }
@@ -383,10 +391,12 @@ __device__ __forceinline__ void d_rows(const Params& p, const DChunk& ch, int a,
                                        float down, float* dsm_pp, bool first) {
   const int lane = threadIdx.x & 31;
   const int I = p.I, nblk = I / 32;
-  for (int r = 0; r < cnt; ++r) {
-    const int row = a + r;
-    float part = 0.f;
-    if (blk < nblk) {
+  float part[kDownRowsPerItem];
+#pragma unroll
+  for (int r = 0; r < kDownRowsPerItem; ++r) {
+    part[r] = 0.f;
+    if (r < cnt && blk < nblk) {
+      const int row = a + r;
       const uint4 c = *reinterpret_cast<const uint4*>(ch.c + (size_t)row * (I / 2) + blk * 16);
       const float sc = e8m0_to_f32(ch.s[(size_t)row * (I / 32) + blk]);
       const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
@@ -403,10 +413,19 @@ __device__ __forceinline__ void d_rows(const Params& p, const DChunk& ch, int a,
         }
       }
       const float2 f0 = __half22float2(acc0), f1 = __half22float2(acc1);
-      part = sc * ((f0.x + f0.y) + (f1.x + f1.y));
+      part[r] = sc * ((f0.x + f0.y) + (f1.x + f1.y));
     }
-    part = warp_sum(part);
-    if (lane == 0) dsm_pp[row] = (first ? 0.f : dsm_pp[row]) + part * down;
+  }
+  // the rows' reductions are independent: interleave their shuffle rounds
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+#pragma unroll
+    for (int r = 0; r < kDownRowsPerItem; ++r) part[r] += __shfl_xor_sync(0xffffffffu, part[r], o);
+  }
+  if (lane == 0) {
+#pragma unroll
+    for (int r = 0; r < kDownRowsPerItem; ++r)
+      if (r < cnt) dsm_pp[a + r] = (first ? 0.f : dsm_pp[a + r]) + part[r] * down;
   }
 }
 
@@ -462,6 +481,88 @@ __device__ __forceinline__ void d_item(const Params& p, const DChunk& ch, int a,
   }
 }
 
+// ---------------------------------------------------------------- routing
+// One warp: top-k of E logits (shared memory), ranked by value with ties to
+// the lower index, and the softmax over the k kept. Lane l holds experts
+// l + 32j, j < NJ (NJ = ceil(E/32) rounded up to a power of two).
+template <int NJ>
+__device__ __forceinline__ void topk_warp(const float* l, int E, int K, int* ids, float* w) {
+  const int lane = threadIdx.x & 31;
+  float v[NJ];
+#pragma unroll
+  for (int j = 0; j < NJ; ++j) {
+    const int e = lane + 32 * j;
+    v[j] = (e < E) ? l[e] : -INFINITY;
+  }
+  uint32_t taken = 0;
+  float sel_v = 0.f, top = 0.f;
+  int sel_i = 0;
+  for (int r = 0; r < K; ++r) {
+    // lane-local best among the lane's untaken experts (ascending index, so
+    // a strictly greater value is needed to replace)
+    float bv = -INFINITY;
+    int bi = 0x7fffffff;
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) {
+      const int e = lane + 32 * j;
+      const bool ok = e < E && !((taken >> j) & 1u);
+      if (ok && (v[j] > bv || bi == 0x7fffffff)) {
+        bv = v[j];
+        bi = e;
+      }
+    }
+    // warp-wide: largest value (order-preserving integer image of the
+    // float), then the lowest expert index holding it
+    const unsigned u = __float_as_uint(bv);
+    const unsigned key = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+    const unsigned kmax = __reduce_max_sync(0xffffffffu, key);
+    const int win = (int)__reduce_min_sync(0xffffffffu, (unsigned)((key == kmax) ? bi : 0x7fffffff));
+    const unsigned ub = (kmax & 0x80000000u) ? (kmax & 0x7fffffffu) : ~kmax;
+    const float wv = __uint_as_float(ub);
+    if ((win & 31) == lane) taken |= 1u << (win >> 5);
+    if (r == 0) top = wv;
+    if (lane == r) {
+      sel_v = wv;
+      sel_i = win;
+    }
+  }
+  const float ex = (lane < K) ? expf(sel_v - top) : 0.f;
+  const float z = warp_sum(ex);
+  if (lane < K) {
+    ids[lane] = sel_i;
+    w[lane] = ex / z;
+  }
+}
+
+// One warp, M*K <= 32 pairs: the expert union (ascending ids) and the pairs
+// grouped by expert in (token, slot) order, from ranks computed with
+// shuffles (no shared-memory scratch). Pair i = (i / K, i % K).
+__device__ __forceinline__ int union_small(const int* s_ids, int np, int K, int* s_union, int* s_poff, int* s_pm,
+                                           int* s_ppos) {
+  const int lane = threadIdx.x & 31;
+  const int id = (lane < np) ? s_ids[lane] : 0x7fffffff;
+  int rank = 0, urank = 0;
+  const unsigned same = __match_any_sync(0xffffffffu, id);
+  const bool leader = (lane < np) && (__ffs(same) - 1 == lane);
+  for (int j = 0; j < np; ++j) {
+    const int oj = __shfl_sync(0xffffffffu, id, j);
+    const bool lj = __shfl_sync(0xffffffffu, leader, j);
+    rank += (oj < id) || (oj == id && j < lane);
+    urank += lj && (oj < id);
+  }
+  const int U = __popc(__ballot_sync(0xffffffffu, leader));
+  if (lane < np) {
+    s_pm[rank] = lane / K;
+    s_ppos[lane] = rank;
+    if (leader) {
+      s_union[urank] = id;
+      s_poff[urank] = rank;
+    }
+  }
+  if (lane == 0) s_poff[U] = np;
+  return U;
+}
+
 // ---------------------------------------------------------------- the kernel
 __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw, FusedPlan pl) {
   extern __shared__ __align__(128) unsigned char smem[];
@@ -482,8 +583,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
   unsigned* done_d = done_gu + kMaxSlots;
   float* s_amax = reinterpret_cast<float*>(smem + pl.o_misc);  // [32]
   float* s_xs = s_amax + kMaxTokens;                           // [32] per-token scales
-  float* s_red = s_xs + kMaxTokens;                            // [kFusedWarps][4]
-  int* s_int = reinterpret_cast<int*>(s_red + kFusedWarps * 4);  // [0] U, [1] epoch, [2] work queue head
+  float* s_red = s_xs + kMaxTokens;                            // [kFusedWarps][kMaxRowsPerCta * 4]
+  int* s_int = reinterpret_cast<int*>(s_red + kFusedWarps * kMaxRowsPerCta * 4);  // [0] U, [1] epoch, [2..3] queue heads
   int* s_ids = reinterpret_cast<int*>(smem + pl.o_ids);
   float* s_w = reinterpret_cast<float*>(smem + pl.o_w);
   int* s_pm = reinterpret_cast<int*>(smem + pl.o_pm);
@@ -507,15 +608,18 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
   const int gu_items = (nr > 0) ? (nr + kGuRowsPerItem - 1) / kGuRowsPerItem : 0;  // per expert
   const int d_items = (nrd > 0) ? (nrd + kDownRowsPerItem - 1) / kDownRowsPerItem : 0;
 
-  if (tid == 0) {
-    for (int i = 0; i < pl.ns_gu; ++i) { mbar_init(full_gu + i, 1); mbar_init(empty_gu + i, max(1, gu_items)); }
-    for (int i = 0; i < pl.ns_d; ++i) {
-      mbar_init(full_d + i, 1);
-      mbar_init(empty_d + i, max(1, d_items));
-      mbar_init(h_bar + i, 1);
+  if (tid < kMaxSlots) {
+    if (tid < pl.ns_gu) { mbar_init(full_gu + tid, 1); mbar_init(empty_gu + tid, max(1, gu_items)); }
+    if (tid < pl.ns_d) {
+      mbar_init(full_d + tid, 1);
+      mbar_init(empty_d + tid, max(1, d_items));
+      mbar_init(h_bar + tid, 1);
     }
+    done_gu[tid] = done_d[tid] = 0u;
+    fence_mbar_init();
+  }
+  if (tid == 0) {
     mbar_init(wr_bar, 1);
-    for (int i = 0; i < kMaxSlots; ++i) done_gu[i] = done_d[i] = 0u;
     fence_mbar_init();
     if (ne > 0) {
       mbar_expect_tx(wr_bar, (unsigned)(ne * H * 4));
@@ -526,7 +630,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
   pdl_wait();
   if (tid == 0) {
     s_int[1] = (int)(ld_relaxed_u32(fw.epoch) + 1u);
-    s_int[2] = 0;
+    s_int[2] = 0;  // gate/up queue head
+    s_int[3] = 0;  // down queue head
   }
   unsigned* s_amax_u = reinterpret_cast<unsigned*>(s_amax);
   if (tid < M) s_amax_u[tid] = 0u;
@@ -586,39 +691,68 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
   __syncthreads();
   if (b == 0 && p.out_xscale && tid < M) p.out_xscale[tid] = s_xs[tid];
 
-  // ---- A2: logits of this CTA's router rows
+  // ---- A2: logits of this CTA's router rows (ne <= kMaxRowsPerCta), four
+  //          tokens per pass, one block reduction per pass
   if (ne > 0) mbar_wait(wr_bar, 0, p);
-  for (int el = 0; el < ne; ++el) {
-    const float4* wrow = reinterpret_cast<const float4*>(wr_s + (size_t)el * H);
+  if (ne > 0) {
     for (int m0 = 0; m0 < M; m0 += 4) {
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      const int mt = min(4, M - m0);
+      float acc[kMaxRowsPerCta][4];
+#pragma unroll
+      for (int el = 0; el < kMaxRowsPerCta; ++el)
+#pragma unroll
+        for (int t = 0; t < 4; ++t) acc[el][t] = 0.f;
       for (int i = tid; i < H / 4; i += kFusedThreads) {
-        const float4 wv = wrow[i];
+        float xv[4][4];
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
-          if (m0 + t < M) {
+          if (t < mt) {
             const uint2* xrow = reinterpret_cast<const uint2*>(xsrc) + (size_t)(m0 + t) * (H / 4);
-            const uint2 xv = pl.x_staged ? xrow[i] : __ldcg(xrow + i);
-            const float2 x01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xv.x));
-            const float2 x23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xv.y));
-            acc[t] = fmaf(x01.x, wv.x, acc[t]);
-            acc[t] = fmaf(x01.y, wv.y, acc[t]);
-            acc[t] = fmaf(x23.x, wv.z, acc[t]);
-            acc[t] = fmaf(x23.y, wv.w, acc[t]);
+            const uint2 q = pl.x_staged ? xrow[i] : __ldcg(xrow + i);
+            const float2 x01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&q.x));
+            const float2 x23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&q.y));
+            xv[t][0] = x01.x; xv[t][1] = x01.y; xv[t][2] = x23.x; xv[t][3] = x23.y;
+          }
+        }
+#pragma unroll
+        for (int el = 0; el < kMaxRowsPerCta; ++el) {
+          if (el < ne) {
+            const float4 wv = reinterpret_cast<const float4*>(wr_s + (size_t)el * H)[i];
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+              if (t < mt) {
+                acc[el][t] = fmaf(xv[t][0], wv.x, acc[el][t]);
+                acc[el][t] = fmaf(xv[t][1], wv.y, acc[el][t]);
+                acc[el][t] = fmaf(xv[t][2], wv.z, acc[el][t]);
+                acc[el][t] = fmaf(xv[t][3], wv.w, acc[el][t]);
+              }
+            }
           }
         }
       }
 #pragma unroll
-      for (int t = 0; t < 4; ++t) acc[t] = warp_sum(acc[t]);
+      for (int o = 16; o; o >>= 1) {
+#pragma unroll
+        for (int el = 0; el < kMaxRowsPerCta; ++el)
+#pragma unroll
+          for (int t = 0; t < 4; ++t)
+            if (el < ne && t < mt) acc[el][t] += __shfl_xor_sync(0xffffffffu, acc[el][t], o);
+      }
       if (lane == 0) {
 #pragma unroll
-        for (int t = 0; t < 4; ++t) s_red[warp * 4 + t] = acc[t];
+        for (int el = 0; el < kMaxRowsPerCta; ++el)
+#pragma unroll
+          for (int t = 0; t < 4; ++t)
+            if (el < ne && t < mt) s_red[warp * (kMaxRowsPerCta * 4) + el * 4 + t] = acc[el][t];
       }
       __syncthreads();
-      if (tid < 4 && m0 + tid < M) {
-        float s = 0.f;
-        for (int w = 0; w < kFusedWarps; ++w) s += s_red[w * 4 + tid];
-        fw.logits[(size_t)(m0 + tid) * E + e0 + el] = s;
+      if (tid < ne * 4) {
+        const int el = tid >> 2, t = tid & 3;
+        if (t < mt) {
+          float sum = 0.f;
+          for (int w = 0; w < kFusedWarps; ++w) sum += s_red[w * (kMaxRowsPerCta * 4) + el * 4 + t];
+          fw.logits[(size_t)(m0 + t) * E + e0 + el] = sum;
+        }
       }
       __syncthreads();
     }
@@ -627,8 +761,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
   // grid-wide: every CTA's logits are in L2 once the router count reaches
   // epoch * G (the last arrival publishes the epoch to the flag copies)
   if (tid == 0) {
-    grid_arrive(fw.route_cnt, fw.route_done, (unsigned long long)epoch * G, epoch);
-    grid_wait(fw.route_done, b, p.force_stall ? epoch + 0x40000000u : epoch, p);
+    grid_arrive(fw.route_cnt);
+    grid_wait(fw.route_cnt, (unsigned long long)(p.force_stall ? epoch + 0x40000000u : epoch) * G, p);
   }
   pdl_launch_dependents();
   __syncthreads();
@@ -638,50 +772,19 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
   for (int i = tid; i < M * E; i += kFusedThreads) s_logit[i] = __ldcg(fw.logits + i);
   __syncthreads();
   for (int m = warp; m < M; m += kFusedWarps) {
-    float v[kMaxExperts / 32];
-#pragma unroll
-    for (int j = 0; j < kMaxExperts / 32; ++j) {
-      const int e = lane + 32 * j;
-      v[j] = (e < E) ? s_logit[m * E + e] : 0.f;
-    }
-    uint32_t taken = 0;
-    float sel_v = 0.f, top = 0.f;
-    int sel_i = 0;
-    for (int r = 0; r < K; ++r) {
-      float bv = -INFINITY;
-      int bi = 0x7fffffff;
-#pragma unroll
-      for (int j = 0; j < kMaxExperts / 32; ++j) {
-        const int e = lane + 32 * j;
-        if (e < E && !((taken >> j) & 1u) && (v[j] > bv || bi == 0x7fffffff)) {
-          bv = v[j];
-          bi = e;
-        }
-      }
-#pragma unroll
-      for (int o = 16; o; o >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-        if (ov > bv || (ov == bv && oi < bi)) {
-          bv = ov;
-          bi = oi;
-        }
-      }
-      if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-      if (r == 0) top = bv;
-      if (lane == r) {
-        sel_v = bv;
-        sel_i = bi;
-      }
-    }
-    const float ex = (lane < K) ? expf(sel_v - top) : 0.f;
-    const float z = warp_sum(ex);
-    if (lane < K) {
-      const float w = ex / z;
-      s_ids[m * K + lane] = sel_i;
-      s_w[m * K + lane] = w;
-      if (b == 0 && p.out_ids) p.out_ids[m * K + lane] = sel_i;
-      if (b == 0 && p.out_w) p.out_w[m * K + lane] = w;
+    const float* lrow = s_logit + (size_t)m * E;
+    int* ids = s_ids + m * K;
+    float* ws = s_w + m * K;
+    if (E <= 32) topk_warp<1>(lrow, E, K, ids, ws);
+    else if (E <= 64) topk_warp<2>(lrow, E, K, ids, ws);
+    else if (E <= 128) topk_warp<4>(lrow, E, K, ids, ws);
+    else if (E <= 256) topk_warp<8>(lrow, E, K, ids, ws);
+    else if (E <= 512) topk_warp<16>(lrow, E, K, ids, ws);
+    else topk_warp<32>(lrow, E, K, ids, ws);
+    __syncwarp();
+    if (b == 0 && lane < K) {
+      if (p.out_ids) p.out_ids[m * K + lane] = ids[lane];
+      if (p.out_w) p.out_w[m * K + lane] = ws[lane];
     }
   }
   __syncthreads();
@@ -689,7 +792,11 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
   // ---- A4: expert union (ascending ids) and the (token, slot) pairs of each
   //          entry in (token, slot) order; one warp, no block barriers
   const int np = M * K;
-  if (warp == 0) {
+  if (warp == 0 && np <= 32) {
+    const int Us = union_small(s_ids, np, K, s_union, s_poff, s_pm, s_ppos);
+    if (lane == 0) s_int[0] = Us;
+    for (int u = lane; u < Us; u += 32) s_cnt[u] = 0;  // per-entry gate/up item counters
+  } else if (warp == 0) {
     for (int e = lane; e < E; e += 32) s_cnt[e] = 0;
     __syncwarp();
     for (int i = lane; i < np; i += 32) atomicAdd(&s_cnt[s_ids[i]], 1);
@@ -789,22 +896,25 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
     return;
   }
 
-  // ---------------- consumers (warps 1..15): one in-order work queue
-  //   entry u contributes gu_items gate/up items, then d_items down items
-  const int per_u = gu_items + d_items;
-  const int total = U * per_u;
+  // ---------------- consumers. Two groups with their own in-order queues, so
+  //   a down item waiting on other CTAs never holds up gate/up work:
+  //   warps 1..kGuWarps take gate/up items (entry-major), the rest take down
+  //   items (entry-major). Gate/up items depend only on their chunk; down
+  //   items on their chunk and on gate/up of the entry on every CTA, which
+  //   never waits on down work, so neither queue can deadlock.
   const unsigned long long tgt = (unsigned long long)epoch * G;
-  if (gu_items == 0 && warp == 1 && lane == 0) {
-    // no gate/up rows here: this CTA's part of every entry is trivially done
-    for (int u = 0; u < U; ++u) grid_arrive(fw.gu_cnt + u, fw.gu_done + (size_t)u * kFlagCopies * kFlagStride, tgt, epoch);
-  }
-  for (;;) {
-    int it = 0;
-    if (lane == 0) it = atomicAdd(&s_int[2], 1);
-    it = __shfl_sync(0xffffffffu, it, 0);
-    if (it >= total) break;
-    const int u = it / per_u, g = it % per_u;
-    if (g < gu_items) {
+  if (warp <= kGuWarps) {
+    const int total = U * gu_items;
+    if (gu_items == 0 && warp == 1 && lane == 0) {
+      // no gate/up rows here: this CTA's part of every entry is trivially done
+      for (int u = 0; u < U; ++u) grid_arrive(fw.gu_cnt + u);
+    }
+    for (;;) {
+      int it = 0;
+      if (lane == 0) it = atomicAdd(&s_int[2], 1);
+      it = __shfl_sync(0xffffffffu, it, 0);
+      if (it >= total) break;
+      const int u = it / gu_items, g = it % gu_items;
       const int slot = u % pl.ns_gu, use = u / pl.ns_gu;
       if (use > 0 && lane == 0) smem_count_wait(done_gu + slot, (unsigned)(use * gu_items), p);
       __syncwarp();
@@ -822,12 +932,18 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
         // acq_rel at CTA scope: the warp completing the entry sees every
         // other warp's h stores, then releases them GPU-wide
         const unsigned done = atom_add_acqrel_cta_smem(reinterpret_cast<unsigned*>(s_cnt + u), 1u) + 1u;
-        if ((int)done == gu_items)
-          grid_arrive(fw.gu_cnt + u, fw.gu_done + (size_t)u * kFlagCopies * kFlagStride, tgt, epoch);
+        if ((int)done == gu_items) grid_arrive(fw.gu_cnt + u);
       }
       __syncwarp();
-    } else {
-      const int gd = g - gu_items;
+    }
+  } else {
+    const int total = U * d_items;
+    for (;;) {
+      int it = 0;
+      if (lane == 0) it = atomicAdd(&s_int[3], 1);
+      it = __shfl_sync(0xffffffffu, it, 0);
+      if (it >= total) break;
+      const int u = it / d_items, gd = it % d_items;
       const int slot = u % pl.ns_d, use = u / pl.ns_d;
       const int pb = s_poff[u], pe = s_poff[u + 1];
       __half2* hbuf = reinterpret_cast<__half2*>(hstage + (size_t)slot * pl.hslot);
@@ -839,7 +955,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
       if (gd == 0) {
         // first down item of the entry: wait for gate/up of the entry on all
         // CTAs, then stage h once for the CTA
-        if (lane == 0) grid_wait(fw.gu_done + (size_t)u * kFlagCopies * kFlagStride, b, epoch, p);
+        if (lane == 0) grid_wait(fw.gu_cnt + u, tgt, p);
         __syncwarp();
         if (pe - pb <= pl.hpairs) stage_h(p, pb, pe, hbuf, hscale);
         __syncwarp();
@@ -872,7 +988,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
   }
   if (b == 0 && ct == 0) {
     // keep every entry's counter at epoch * G for the next launch
-    for (int u = U; u < pl.max_union; ++u) atom_add_acqrel_u64(fw.gu_cnt + u, (unsigned long long)G);
+    for (int u = U; u < pl.max_union; ++u) red_release_add_u64(fw.gu_cnt + u, (unsigned long long)G);
     st_relaxed_u32(fw.epoch, epoch);
   }
 }
