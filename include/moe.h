@@ -149,6 +149,44 @@ moe_status moe_plan_query(const moe_config* cfg, int32_t sm_count, size_t smem_l
  * reports MOE_ERR_TIMEOUT. Returns INVALID_ARG for a NULL ctx. */
 moe_status moe_debug_set_wait(moe_ctx* ctx, long long budget_cycles, int force_stall);
 
+/* Size of the fixed device scratch array behind moe_decode_static. */
+#define MOE_STATIC_SCRATCH_BYTES ((size_t)4 << 20)
+
+/* One decode step that allocates nothing. The paper has no counterpart: this
+ * is an interface for callers that cannot allocate device memory, such as a
+ * plugin hosted by a runtime that owns all device memory, or a serving loop
+ * that must never call cudaMalloc (the call can synchronise the device).
+ *
+ * It computes what moe_decode computes, with the three-kernel form of the
+ * step (the MOE_FLAG_SPLIT_KERNELS path). There is no context. The layer's
+ * shapes come from cfg (flags, max_tokens and device are ignored), and the
+ * weights, x and y are passed in directly with the layouts, alignment and
+ * optional outputs of moe_load_experts and moe_decode. The scale bytes are not
+ * scanned for 0xFF.
+ *
+ * Scratch is one file-scope device array of MOE_STATIC_SCRATCH_BYTES (4 MiB),
+ * held by every GPU that loads the library until the process exits. A call
+ * needs about M*(E*4 + H) + M*top_k*(4*I + 32) bytes of it. Larger shapes
+ * return MOE_ERR_UNSUPPORTED, as do calls whose M*H*2 bytes of f16
+ * activations exceed the gate/up kernel's shared memory. The first call on a
+ * device, made with that device current, does that device's set-up (it finds
+ * the array's device address and reads the device's limits). Make that first
+ * call before any stream capture.
+ *
+ * Every call shares the array, which keeps what the last call left in it.
+ * Each call clears the words that must start at zero. Calls that overlap on
+ * the GPU (different streams or host threads) race on the array and corrupt
+ * each other's results.
+ *
+ * No cudaMalloc, cudaFree or other allocating routine is called. Returns
+ * INVALID_ARG (null/misaligned/bad size), UNSUPPORTED (device or shape),
+ * CUDA (launch). */
+moe_status moe_decode_static(const moe_config* cfg, const float* router_w,
+                             const uint8_t* w13_codes, const uint8_t* w13_scales,
+                             const uint8_t* w2_codes, const uint8_t* w2_scales,
+                             const void* x_bf16, int32_t M, void* y_bf16, void* stream,
+                             int32_t* topk_ids, float* topk_w, uint8_t* xq, float* xscale);
+
 /* Static string naming a status code. */
 const char* moe_status_string(moe_status s);
 

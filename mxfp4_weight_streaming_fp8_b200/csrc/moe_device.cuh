@@ -188,7 +188,7 @@ __device__ __forceinline__ uint4 ldg_stream(const void* p) {
 // Per-token E4M3 quantisation, one CTA per token: amax = max|x|,
 // inv = fl32(448/amax), code = E4M3_rne_sat(fl32(x*inv)), s = fl32(amax/448);
 // amax == 0 gives all-zero codes and s = 1.
-__device__ void quantize_token(const Params& p, int m, float* red) {
+static __device__ void quantize_token(const Params& p, int m, float* red) {
   const __nv_bfloat16* xm = p.x + (size_t)m * p.H;
   float a = 0.f;
   for (int h = threadIdx.x; h < p.H; h += blockDim.x) a = fmaxf(a, fabsf(__bfloat162float(xm[h])));
@@ -210,7 +210,7 @@ __device__ void quantize_token(const Params& p, int m, float* red) {
 // ---------------------------------------------------------------- A2
 // One warp computes logits[m][e] for all M tokens of one router row e (fp32
 // accumulation of bf16 x times fp32 weights), four tokens per pass.
-__device__ void router_row(const Params& p, int e) {
+static __device__ void router_row(const Params& p, int e) {
   const int lane = threadIdx.x & 31;
   const float4* w = reinterpret_cast<const float4*>(p.wr + (size_t)e * p.H);
   const int n4 = p.H / 4;
@@ -243,7 +243,7 @@ __device__ void router_row(const Params& p, int e) {
 // One warp: top-k of token m's E logits (ranked by value, ties to the lower
 // index) and the softmax over the kept logits. Lane e%32 holds logit e.
 // Writes ws.ids/ws.wts (and the optional outputs).
-__device__ void topk_token(const Params& p, int m) {
+static __device__ void topk_token(const Params& p, int m) {
   const int lane = threadIdx.x & 31;
   const float* l = p.ws.logits + (size_t)m * p.E;
   float v[kMaxExperts / 32];
@@ -298,7 +298,7 @@ __device__ void topk_token(const Params& p, int m) {
 // (token, slot) pairs of each union entry, in (token, slot) order. Reads
 // ws.ids / ws.wts written earlier by this CTA (after __syncthreads).
 // `cnt` is shared scratch of kMaxExperts ints.
-__device__ void build_union(const Params& p, int* cnt, int* s_u) {
+static __device__ void build_union(const Params& p, int* cnt, int* s_u) {
   const int tid = threadIdx.x, lane = tid & 31;
   const int np = p.M * p.K;
   for (int e = tid; e < p.E; e += blockDim.x) cnt[e] = 0;

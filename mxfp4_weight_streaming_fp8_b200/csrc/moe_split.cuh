@@ -2,7 +2,8 @@
 //
 // This is the plain, launch-per-phase form of the step. It is kept beside the
 // persistent kernel as a second path that the tests compare against, and it
-// is selected with MOE_FLAG_SPLIT_KERNELS.
+// is selected with MOE_FLAG_SPLIT_KERNELS. The kernels have internal linkage:
+// each translation unit that launches them gets its own copy.
 //   k_route   quantise (A1), router logits (A2); the last CTA to finish does
 //             top-k (A3) and the union (A4)
 //   k_gateup  gate/up GEMV with in-register MXFP4 decode (A5) and SwiGLU (A6)
@@ -13,7 +14,7 @@
 
 namespace moe {
 
-__global__ void __launch_bounds__(kThreads) k_route(Params p) {
+static __global__ void __launch_bounds__(kThreads) k_route(Params p) {
   __shared__ float red[kWarps];
   __shared__ int s_last, s_u;
   __shared__ int cnt[kMaxExperts];
@@ -43,7 +44,7 @@ __global__ void __launch_bounds__(kThreads) k_route(Params p) {
 // gate row n and the up row I+n of expert union_ids[u]; for each (token, slot)
 // pair routed to the expert, h = silu(s*<gate,q>) * s*<up,q>.
 // Activations are decoded once per CTA into shared memory as f16.
-__global__ void __launch_bounds__(kThreads) k_gateup(Params p) {
+static __global__ void __launch_bounds__(kThreads) k_gateup(Params p) {
   extern __shared__ __align__(128) unsigned char smem[];
   uint32_t* act2 = reinterpret_cast<uint32_t*>(smem);  // [M][H/2] f16x2
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -93,7 +94,7 @@ __global__ void __launch_bounds__(kThreads) k_gateup(Params p) {
 // Down + combine: one warp per output row r; for each union expert (ascending
 // id) and each of its (token, slot) pairs, d = <W2[e][r], h_pair>, and
 // y[m][r] accumulates w_pair * d in that order (deterministic, no atomics).
-__global__ void __launch_bounds__(kThreads) k_down(Params p) {
+static __global__ void __launch_bounds__(kThreads) k_down(Params p) {
   __shared__ float yacc[kWarps][kMaxTokens];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int H = p.H, I = p.I, nblk = I / 32;
@@ -134,7 +135,7 @@ __global__ void __launch_bounds__(kThreads) k_down(Params p) {
 }
 
 // Scan scale bytes for the E8M0 NaN encoding (0xFF); counts into *bad.
-__global__ void k_scan_scales(const uint8_t* s, size_t n, unsigned* bad) {
+static __global__ void k_scan_scales(const uint8_t* s, size_t n, unsigned* bad) {
   unsigned c = 0;
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
     c += (s[i] == 0xFF);

@@ -65,6 +65,8 @@ def lib() -> ctypes.CDLL:
         L.moe_plan_query.argtypes = [ctypes.POINTER(moe_config), ctypes.c_int32, ctypes.c_size_t,
                                      ctypes.c_char_p, ctypes.c_size_t]
         L.moe_plan_query.restype = ctypes.c_int
+        L.moe_decode_static.argtypes = [ctypes.POINTER(moe_config)] + [_vp] * 6 + [ctypes.c_int32] + [_vp] * 6
+        L.moe_decode_static.restype = ctypes.c_int
         L.moe_debug_set_wait.argtypes = [_vp, ctypes.c_longlong, ctypes.c_int]
         L.moe_debug_set_wait.restype = ctypes.c_int
         _lib = L
@@ -88,6 +90,16 @@ def plan_query(hidden, inter, num_experts, top_k, max_tokens, flags=0, sm_count=
     buf = ctypes.create_string_buffer(1024)
     st = lib().moe_plan_query(ctypes.byref(cfg), sm_count, smem_limit, buf, len(buf))
     return st, (json.loads(buf.value.decode()) if buf.value else None)
+
+
+def decode_static(hidden, inter, num_experts, top_k, router_w, w13_codes, w13_scales, w2_codes, w2_scales, x, M, y,
+                  stream=None, topk_ids=None, topk_w=None, xq=None, xscale=None) -> int:
+    """moe_decode_static: one step with no context and no allocation; returns
+    the status code. Scratch is the library's fixed device array."""
+    cfg = moe_config(hidden, inter, num_experts, top_k, max(1, int(M)), 0, 0)
+    return lib().moe_decode_static(ctypes.byref(cfg), _ptr(router_w), _ptr(w13_codes), _ptr(w13_scales),
+                                   _ptr(w2_codes), _ptr(w2_scales), _ptr(x), int(M), _ptr(y),
+                                   _stream_handle(stream), _ptr(topk_ids), _ptr(topk_w), _ptr(xq), _ptr(xscale))
 
 
 def status_string(s: int) -> str:
