@@ -293,6 +293,7 @@ __device__ __forceinline__ void gu_item(const Params& p, const GuChunk& ch, int 
     float ag[kGuRowsPerItem], au[kGuRowsPerItem];
 #pragma unroll
     for (int r = 0; r < kGuRowsPerItem; ++r) ag[r] = au[r] = 0.f;
+#pragma unroll 2
     for (int hb = lane; hb < nhb; hb += 32) {
       const uint4 aq = *reinterpret_cast<const uint4*>(am + hb * 16);  // 16 E4M3 codes
       uint32_t a2[8];
@@ -363,24 +364,51 @@ __device__ __forceinline__ int h_rescale_exp(float mx) {
 __device__ __forceinline__ void stage_h(const Params& p, int pb, int pe, __half2* hbuf, float* hscale) {
   const int lane = threadIdx.x & 31;
   const int I = p.I;
+  constexpr int kQ = 8;  // uint4 per lane kept in registers: one L2 pass when I <= 1024
   for (int pp = pb; pp < pe; ++pp) {
     const int j = pp - pb;
     const uint4* hp = reinterpret_cast<const uint4*>(p.ws.h + (size_t)pp * I);
-    float mx = 0.f;
-    for (int q = lane; q < I / 4; q += 32) {
-      const uint4 v = ld_cg_u4(hp + q);
-      mx = fmaxf(mx, fmaxf(fmaxf(fabsf(__uint_as_float(v.x)), fabsf(__uint_as_float(v.y))),
-                           fmaxf(fabsf(__uint_as_float(v.z)), fabsf(__uint_as_float(v.w)))));
-    }
-    const int t = h_rescale_exp(warp_max(mx));
-    const float up = ldexpf(1.f, t);
     __half2* dst = hbuf + (size_t)j * (I / 2);
-    for (int q = lane; q < I / 4; q += 32) {
-      const uint4 v = ld_cg_u4(hp + q);
-      dst[2 * q] = __floats2half2_rn(__uint_as_float(v.x) * up, __uint_as_float(v.y) * up);
-      dst[2 * q + 1] = __floats2half2_rn(__uint_as_float(v.z) * up, __uint_as_float(v.w) * up);
+    if (I / 4 <= 32 * kQ) {
+      uint4 v[kQ];
+      float mx = 0.f;
+#pragma unroll
+      for (int k = 0; k < kQ; ++k) {
+        const int q = lane + 32 * k;
+        v[k] = (q < I / 4) ? ld_cg_u4(hp + q) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int k = 0; k < kQ; ++k)
+        mx = fmaxf(mx, fmaxf(fmaxf(fabsf(__uint_as_float(v[k].x)), fabsf(__uint_as_float(v[k].y))),
+                             fmaxf(fabsf(__uint_as_float(v[k].z)), fabsf(__uint_as_float(v[k].w)))));
+      const int t = h_rescale_exp(warp_max(mx));
+      const float up = ldexpf(1.f, t);
+#pragma unroll
+      for (int k = 0; k < kQ; ++k) {
+        const int q = lane + 32 * k;
+        if (q < I / 4) {
+          dst[2 * q] = __floats2half2_rn(__uint_as_float(v[k].x) * up, __uint_as_float(v[k].y) * up);
+          dst[2 * q + 1] = __floats2half2_rn(__uint_as_float(v[k].z) * up, __uint_as_float(v[k].w) * up);
+        }
+      }
+      if (lane == 0) hscale[j] = ldexpf(1.f, -t);
+    } else {
+      // wide intermediate: one pass for the max, one to convert
+      float mx = 0.f;
+      for (int q = lane; q < I / 4; q += 32) {
+        const uint4 v = ld_cg_u4(hp + q);
+        mx = fmaxf(mx, fmaxf(fmaxf(fabsf(__uint_as_float(v.x)), fabsf(__uint_as_float(v.y))),
+                             fmaxf(fabsf(__uint_as_float(v.z)), fabsf(__uint_as_float(v.w)))));
+      }
+      const int t = h_rescale_exp(warp_max(mx));
+      const float up = ldexpf(1.f, t);
+      for (int q = lane; q < I / 4; q += 32) {
+        const uint4 v = ld_cg_u4(hp + q);
+        dst[2 * q] = __floats2half2_rn(__uint_as_float(v.x) * up, __uint_as_float(v.y) * up);
+        dst[2 * q + 1] = __floats2half2_rn(__uint_as_float(v.z) * up, __uint_as_float(v.w) * up);
+      }
+      if (lane == 0) hscale[j] = ldexpf(1.f, -t);
     }
-    if (lane == 0) hscale[j] = ldexpf(1.f, -t);
   }
 }
 
@@ -692,18 +720,16 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
   if (b == 0 && p.out_xscale && tid < M) p.out_xscale[tid] = s_xs[tid];
 
   // ---- A2: logits of this CTA's router rows (ne <= kMaxRowsPerCta), four
-  //          tokens per pass, one block reduction per pass
+  //          tokens per pass; warp partials go to shared memory and one block
+  //          barrier per pass ends it
   if (ne > 0) mbar_wait(wr_bar, 0, p);
-  if (ne > 0) {
-    for (int m0 = 0; m0 < M; m0 += 4) {
-      const int mt = min(4, M - m0);
-      float acc[kMaxRowsPerCta][4];
-#pragma unroll
-      for (int el = 0; el < kMaxRowsPerCta; ++el)
-#pragma unroll
-        for (int t = 0; t < 4; ++t) acc[el][t] = 0.f;
+  for (int m0 = 0; m0 < M && ne > 0; m0 += 4) {
+    const int mt = min(4, M - m0);
+    for (int el = 0; el < ne; ++el) {
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      const float4* wrow = reinterpret_cast<const float4*>(wr_s + (size_t)el * H);
       for (int i = tid; i < H / 4; i += kFusedThreads) {
-        float xv[4][4];
+        const float4 wv = wrow[i];
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
           if (t < mt) {
@@ -711,53 +737,39 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
             const uint2 q = pl.x_staged ? xrow[i] : __ldcg(xrow + i);
             const float2 x01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&q.x));
             const float2 x23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&q.y));
-            xv[t][0] = x01.x; xv[t][1] = x01.y; xv[t][2] = x23.x; xv[t][3] = x23.y;
-          }
-        }
-#pragma unroll
-        for (int el = 0; el < kMaxRowsPerCta; ++el) {
-          if (el < ne) {
-            const float4 wv = reinterpret_cast<const float4*>(wr_s + (size_t)el * H)[i];
-#pragma unroll
-            for (int t = 0; t < 4; ++t) {
-              if (t < mt) {
-                acc[el][t] = fmaf(xv[t][0], wv.x, acc[el][t]);
-                acc[el][t] = fmaf(xv[t][1], wv.y, acc[el][t]);
-                acc[el][t] = fmaf(xv[t][2], wv.z, acc[el][t]);
-                acc[el][t] = fmaf(xv[t][3], wv.w, acc[el][t]);
-              }
-            }
+            acc[t] = fmaf(x01.x, wv.x, acc[t]);
+            acc[t] = fmaf(x01.y, wv.y, acc[t]);
+            acc[t] = fmaf(x23.x, wv.z, acc[t]);
+            acc[t] = fmaf(x23.y, wv.w, acc[t]);
           }
         }
       }
+      if (mt == 1) {
+        acc[0] = warp_sum(acc[0]);
+      } else {
 #pragma unroll
-      for (int o = 16; o; o >>= 1) {
+        for (int o = 16; o; o >>= 1) {
 #pragma unroll
-        for (int el = 0; el < kMaxRowsPerCta; ++el)
-#pragma unroll
-          for (int t = 0; t < 4; ++t)
-            if (el < ne && t < mt) acc[el][t] += __shfl_xor_sync(0xffffffffu, acc[el][t], o);
+          for (int t = 0; t < 4; ++t) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], o);
+        }
       }
       if (lane == 0) {
 #pragma unroll
-        for (int el = 0; el < kMaxRowsPerCta; ++el)
-#pragma unroll
-          for (int t = 0; t < 4; ++t)
-            if (el < ne && t < mt) s_red[warp * (kMaxRowsPerCta * 4) + el * 4 + t] = acc[el][t];
+        for (int t = 0; t < 4; ++t)
+          if (t < mt) s_red[warp * (kMaxRowsPerCta * 4) + el * 4 + t] = acc[t];
       }
-      __syncthreads();
-      if (tid < ne * 4) {
-        const int el = tid >> 2, t = tid & 3;
-        if (t < mt) {
-          float sum = 0.f;
-          for (int w = 0; w < kFusedWarps; ++w) sum += s_red[w * (kMaxRowsPerCta * 4) + el * 4 + t];
-          fw.logits[(size_t)(m0 + t) * E + e0 + el] = sum;
-        }
-      }
-      __syncthreads();
     }
+    __syncthreads();
+    if (tid < ne * 4) {
+      const int el = tid >> 2, t = tid & 3;
+      if (t < mt) {
+        float sum = 0.f;
+        for (int w = 0; w < kFusedWarps; ++w) sum += s_red[w * (kMaxRowsPerCta * 4) + el * 4 + t];
+        fw.logits[(size_t)(m0 + t) * E + e0 + el] = sum;
+      }
+    }
+    __syncthreads();
   }
-  __syncthreads();
   // grid-wide: every CTA's logits are in L2 once the router count reaches
   // epoch * G (the last arrival publishes the epoch to the flag copies)
   if (tid == 0) {
