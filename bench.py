@@ -170,16 +170,23 @@ def sum_over_ranks(value: float, ws: int, device=None) -> float:
 
 
 # ------------------------------------------------------------------ workload
-def build_pool(device, M, mode, layers=POOL_LAYERS, seed=SEED, flags=0):
+def build_pool(device, M, mode, layers=POOL_LAYERS, seed=SEED, flags=0, stack=False):
+    """One context per layer of the pool. With stack=True, layers after the
+    first normalise their input (RMSNorm) and take the previous output."""
     import torch
     from mxfp4_weight_streaming_fp8_b200 import moe, synth
     x = synth.gen_x(seed, M, H)
     ctxs, weights = [], []
     for l in range(layers):
-        wr = synth.force_router(x, synth.gen_router(seed, l, E, H), K, mode, seed=seed, layer=l)
+        # routing forced against the shared input (a stacked layer's input is
+        # the previous output, so its routing stays natural)
+        wr = synth.gen_router(seed, l, E, H)
+        if not (stack and l > 0):
+            wr = synth.force_router(x, wr, K, mode, seed=seed, layer=l)
         ex = synth.layer_experts_torch(seed, l, E, H, I, device)
         wr_d = torch.from_numpy(wr).to(device)
-        ctx = moe.MoELayer(H, I, E, K, M, flags=flags, device=device.index)
+        lflags = flags | (moe.MOE_FLAG_PRE_RMSNORM if (stack and l > 0) else 0)
+        ctx = moe.MoELayer(H, I, E, K, M, flags=lflags, device=device.index)
         ctx.load_experts(wr_d, *ex, validate=False)
         ctxs.append(ctx)
         weights.append((wr_d, ex))
@@ -200,16 +207,18 @@ def run_ours(args):
     M = args.tokens
     L = args.layers
     flags = moe.MOE_FLAG_SPLIT_KERNELS if args.variant == "split" else 0
-    x, ctxs, _weights = build_pool(device, M, args.routing, layers=L, flags=flags)
+    x, ctxs, _weights = build_pool(device, M, args.routing, layers=L, flags=flags, stack=args.stack)
     info = ctxs[0].query()
     x_d = x.to(device)
     ys = [torch.empty_like(x_d) for _ in range(L)]
+    # layer l reads x (independent layer-steps) or, stacked, the previous output
+    inputs = [x_d if (l == 0 or not args.stack) else ys[l - 1] for l in range(L)]
 
     # union size of each layer (from the kernel's own routing outputs)
     Us = []
     for l in range(L):
-        y, ids, _, _, _ = ctxs[l].decode(x_d, routing=True)
-        Us.append(len(set(ids.cpu().numpy().ravel().tolist())))
+        out = ctxs[l].decode(inputs[l], y=ys[l], routing=True)
+        Us.append(len(set(out[1].cpu().numpy().ravel().tolist())))
     torch.cuda.synchronize()
     for c in ctxs:
         st = c.sync_status()
@@ -221,13 +230,13 @@ def run_ours(args):
     stream.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(stream):
         for l in range(L):
-            assert ctxs[l].decode_raw(x_d, M, ys[l], stream=stream) == moe.MOE_OK
+            assert ctxs[l].decode_raw(inputs[l], M, ys[l], stream=stream) == moe.MOE_OK
     torch.cuda.current_stream().wait_stream(stream)
     torch.cuda.synchronize()
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph, stream=stream):
         for l in range(L):
-            st = ctxs[l].decode_raw(x_d, M, ys[l], stream=stream)
+            st = ctxs[l].decode_raw(inputs[l], M, ys[l], stream=stream)
             assert st == moe.MOE_OK, moe.status_string(st)
 
     cur = torch.cuda.current_stream()
@@ -265,11 +274,11 @@ def run_ours(args):
     exp_b = U_mean * expert_bytes()
     peak, peak_kind = load_peaks()
     achieved = alg / (us_per_layer * 1e-6) / 1e9
-    workload = f"ling_layer_M{M}_{args.routing}"
+    workload = (f"ling_stack{L}_rmsnorm_M{M}" if args.stack else f"ling_layer_M{M}_{args.routing}")
     traffic = recorded_traffic("k_fused", workload)
 
     # ---- end to end through the public API with host buffers
-    e2e = run_e2e(args, ctxs, x, device, M, L)
+    e2e = run_e2e(args, ctxs, x, device, M, L, stack=args.stack)
 
     # ---- CPU oracle baseline (rank 0 only)
     cpu = run_cpu_baseline(args, M) if rank == 0 and not args.no_cpu else None
@@ -283,7 +292,8 @@ def run_ours(args):
         "config": {"workload": workload, "hidden": H, "inter": I, "num_experts": E, "top_k": K, "tokens": M,
                    "routing": args.routing, "layers_in_pool": L, "pool_weight_bytes": L * E * expert_bytes(),
                    "l2": "inputs larger than L2: each layer-step reads a different layer of the pool",
-                   "step": f"{L} layer-steps in one CUDA graph", "parallelism": f"replicas x{ws}",
+                   "step": (f"{L}-layer stack (RMSNorm between layers) in one CUDA graph" if args.stack
+                            else f"{L} layer-steps in one CUDA graph"), "parallelism": f"replicas x{ws}",
                    "variant": info["variant"]},
         "us_per_layer_step": round(us_per_layer, 3),
         "union_experts": U_mean,
@@ -297,6 +307,9 @@ def run_ours(args):
         "clocks": clk.summary(),
         "e2e": e2e,
     }
+    if args.stack:
+        line["stack_tokens_per_s"] = round(ws * M * args.steps / (ms / 1e3), 1)
+        line["us_per_stack_step"] = round(ms * 1e3 / args.steps, 2)
     if cpu is not None:
         line["cpu_baseline"] = cpu
     if rank == 0:
@@ -308,7 +321,7 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
-def run_e2e(args, ctxs, x_cpu, device, M, L):
+def run_e2e(args, ctxs, x_cpu, device, M, L, stack=False):
     """Per step: pinned-host x -> device, L moe_decode calls through the
     Python/C-ABI API, final y -> pinned host; timed with events."""
     import torch
@@ -322,7 +335,7 @@ def run_e2e(args, ctxs, x_cpu, device, M, L):
     def step():
         xd.copy_(xh, non_blocking=True)
         for l in range(L):
-            ctxs[l].decode_raw(xd, M, ys[l], stream=cur)
+            ctxs[l].decode_raw(ys[l - 1] if (stack and l > 0) else xd, M, ys[l], stream=cur)
         yh.copy_(ys[-1], non_blocking=True)
 
     for _ in range(args.warmup):
@@ -419,6 +432,8 @@ def main():
     ap.add_argument("--ref-layers", type=int, default=4)
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--variant", choices=["fused", "split"], default="fused")
+    ap.add_argument("--stack", action="store_true",
+                    help="chain the pool as a stack: layer l+1 takes RMSNorm(y_l)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3

@@ -66,8 +66,11 @@ typedef enum {
 /* moe_config.flags */
 #define MOE_FLAG_SPLIT_KERNELS 0x1u /* run the step as three kernels (route, gate/up,
                                        down) instead of one persistent kernel */
-#define MOE_FLAG_PRE_RMSNORM  0x2u  /* x <- bf16(x / sqrt(mean(x^2) + 1e-6)) before
-                                       A1/A2 (unit-weight RMSNorm between layers) */
+#define MOE_FLAG_PRE_RMSNORM  0x2u  /* x <- bf16(x / sqrt(mean(x^2) + 1e-6)) per token
+                                       before A1/A2 (unit-weight RMSNorm between
+                                       stacked layers, fp32); persistent kernel
+                                       only: with MOE_FLAG_SPLIT_KERNELS,
+                                       moe_create returns MOE_ERR_UNSUPPORTED */
 
 typedef struct {
   int32_t hidden;      /* H: multiple of 32, 32..8192                        */
@@ -112,10 +115,11 @@ moe_status moe_load_experts(moe_ctx* ctx, const float* router_w,
  *   topk_w   [M][top_k] fp32 routing weights in the same order
  *   xq       [M][H] uint8 E4M3 activation codes
  *   xscale   [M] fp32 per-token activation scales
+ *   xnorm    [M][H] bf16 normalised input (only with MOE_FLAG_PRE_RMSNORM)
  * Returns INVALID_ARG (null/misaligned/size), NOT_LOADED, CUDA (launch). */
 moe_status moe_decode(moe_ctx* ctx, const void* x_bf16, int32_t M, void* y_bf16,
                       void* stream, int32_t* topk_ids, float* topk_w, uint8_t* xq,
-                      float* xscale);
+                      float* xscale, void* xnorm_bf16);
 
 /* Synchronise `stream`, then read and clear the context's device status word.
  * Returns MOE_ERR_TIMEOUT if a device-side wait gave up since the last call,

@@ -46,7 +46,7 @@ moe_status validate_config(const moe_config& c) {
   if (c.top_k < 1 || c.top_k > c.num_experts || c.top_k > moe::kMaxTopK) return MOE_ERR_INVALID_ARG;
   if (c.max_tokens < 1 || c.max_tokens > moe::kMaxTokens) return MOE_ERR_INVALID_ARG;
   if (c.flags & ~(MOE_FLAG_SPLIT_KERNELS | MOE_FLAG_PRE_RMSNORM)) return MOE_ERR_INVALID_ARG;
-  if (c.flags & MOE_FLAG_PRE_RMSNORM) return MOE_ERR_UNSUPPORTED;
+  if ((c.flags & MOE_FLAG_PRE_RMSNORM) && (c.flags & MOE_FLAG_SPLIT_KERNELS)) return MOE_ERR_UNSUPPORTED;
   return MOE_OK;
 }
 
@@ -70,7 +70,7 @@ bool make_plan(const moe_config& c, int sm_count, size_t smem_limit, moe::FusedP
   size_t off = 0;
   auto take = [&](size_t bytes, size_t a) { off = align_up(off, a); size_t o = off; off += bytes; return o; };
   pl->o_bar = (int)take((5 * kMaxSlots + 1) * 8 + 2 * kMaxSlots * 4, 16);
-  pl->o_misc = (int)take((2 * moe::kMaxTokens + moe::kFusedWarps * moe::kMaxRowsPerCta * 4 + 8) * 4, 16);
+  pl->o_misc = (int)take((3 * moe::kMaxTokens + moe::kFusedWarps * moe::kMaxRowsPerCta * 4 + 8) * 4, 16);
   pl->o_ids = (int)take(NP * 4, 16);
   pl->o_w = (int)take(NP * 4, 16);
   pl->o_pm = (int)take(NP * 4, 16);
@@ -303,7 +303,7 @@ moe_status moe_load_experts(moe_ctx* ctx, const float* router_w, const uint8_t* 
 }
 
 moe_status moe_decode(moe_ctx* ctx, const void* x_bf16, int32_t M, void* y_bf16, void* stream,
-                      int32_t* topk_ids, float* topk_w, uint8_t* xq, float* xscale) {
+                      int32_t* topk_ids, float* topk_w, uint8_t* xq, float* xscale, void* xnorm_bf16) {
   if (!ctx) return MOE_ERR_INVALID_ARG;
   const moe_config& c = ctx->cfg;
   if (M < 0 || M > c.max_tokens) return MOE_ERR_INVALID_ARG;
@@ -315,8 +315,9 @@ moe_status moe_decode(moe_ctx* ctx, const void* x_bf16, int32_t M, void* y_bf16,
   if (xb < yb + xbytes && yb < xb + xbytes) return MOE_ERR_INVALID_ARG;  // aliasing
   if ((xq && !aligned16(xq)) || (topk_ids && (reinterpret_cast<uintptr_t>(topk_ids) & 3)) ||
       (topk_w && (reinterpret_cast<uintptr_t>(topk_w) & 3)) ||
-      (xscale && (reinterpret_cast<uintptr_t>(xscale) & 3)))
+      (xscale && (reinterpret_cast<uintptr_t>(xscale) & 3)) || (xnorm_bf16 && !aligned16(xnorm_bf16)))
     return MOE_ERR_INVALID_ARG;
+  if (xnorm_bf16 && !(c.flags & MOE_FLAG_PRE_RMSNORM)) return MOE_ERR_INVALID_ARG;
   if (!ctx->loaded) return MOE_ERR_NOT_LOADED;
   DeviceGuard guard(ctx->dev);
   if (!guard.ok) return MOE_ERR_CUDA;
@@ -340,6 +341,8 @@ moe_status moe_decode(moe_ctx* ctx, const void* x_bf16, int32_t M, void* y_bf16,
   p.out_xscale = xscale;
   p.spin_limit = ctx->spin_limit;
   p.force_stall = ctx->force_stall;
+  p.pre_rmsnorm = (c.flags & MOE_FLAG_PRE_RMSNORM) ? 1 : 0;
+  p.out_xn = static_cast<__nv_bfloat16*>(xnorm_bf16);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (ctx->variant == kSplit) {
     moe::k_route<<<ctx->grid_route, moe::kThreads, 0, st>>>(p);
@@ -423,10 +426,11 @@ moe_status moe_query(const moe_ctx* ctx, char* buf, size_t len) {
     n = snprintf(buf, len,
                  "{\"lib\": \"libmoe\", \"arch\": \"sm_100a\", \"device\": %d, \"sm_count\": %d, "
                  "\"variant\": \"fused\", \"kernels\": [\"k_fused\"], \"grid\": [%d], \"threads\": %d, "
-                 "\"smem\": %d, \"ring_gu\": [%d, %d], \"ring_d\": [%d, %d], \"pdl\": true, "
+                 "\"smem\": %d, \"ring_gu\": [%d, %d], \"ring_d\": [%d, %d], \"pdl\": true, \"pre_rmsnorm\": %s, "
                  "\"hidden\": %d, \"inter\": %d, \"num_experts\": %d, \"top_k\": %d, \"max_tokens\": %d}",
                  ctx->dev, ctx->sm_count, pl.G, moe::kFusedThreads, pl.smem_bytes, pl.ns_gu, pl.slot_gu, pl.ns_d,
-                 pl.slot_d, c.hidden, c.inter, c.num_experts, c.top_k, c.max_tokens);
+                 pl.slot_d, (c.flags & MOE_FLAG_PRE_RMSNORM) ? "true" : "false", c.hidden, c.inter, c.num_experts,
+                 c.top_k, c.max_tokens);
   }
   if (n < 0 || (size_t)n >= len) return MOE_ERR_INVALID_ARG;
   return MOE_OK;

@@ -57,6 +57,8 @@ struct Params {
   float* out_xscale;
   long long spin_limit;  // device-side wait budget in clock64 cycles
   int force_stall;       // test hook: the logits wait targets a tag nobody writes
+  int pre_rmsnorm;       // x <- bf16(x * rsqrt(mean(x^2) + eps)) before A1/A2
+  __nv_bfloat16* out_xn; // optional [M][H] normalised input
 };
 
 // ---------------------------------------------------------------- formats

@@ -97,13 +97,15 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
+// try_wait with a suspend-time hint: a waiting thread is parked (up to the
+// hint) until the phase completes instead of spinning on issue slots.
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, unsigned parity) {
   uint32_t ok;
   asm volatile(
       "{.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;}"
-      : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+      : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity), "r"(20000u) : "memory");
   return ok != 0;
 }
 
@@ -692,6 +694,58 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
   }
   __syncthreads();
   const uint4* xsrc = pl.x_staged ? x_s : reinterpret_cast<const uint4*>(p.x);
+  // ---- A9 (stacked layers): x <- bf16(x / sqrt(mean(x^2) + 1e-6)) per token.
+  //      One warp per token sums x^2 in a fixed order with IEEE fp32 ops, so
+  //      every CTA derives the same factor. Rounding is monotonic and
+  //      symmetric, so the new amax is bf16(fl32(amax * r)).
+  float* s_rn = reinterpret_cast<float*>(s_int + 8);  // [32] per-token RMSNorm factors
+  if (p.pre_rmsnorm) {
+    for (int m = warp; m < M; m += kFusedWarps) {
+      float ss = 0.f;
+      for (int i = lane; i < H / 8; i += 32) {
+        const uint4 v = pl.x_staged ? xsrc[(size_t)m * (H / 8) + i] : __ldcg(xsrc + (size_t)m * (H / 8) + i);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[t]));
+          ss = __fmaf_rn(f.x, f.x, ss);
+          ss = __fmaf_rn(f.y, f.y, ss);
+        }
+      }
+      ss = warp_sum(ss);
+      if (lane == 0) {
+        const float r = __fdiv_rn(1.f, __fsqrt_rn(__fadd_rn(__fdiv_rn(ss, (float)H), 1e-6f)));
+        s_rn[m] = r;
+        s_amax[m] = __bfloat162float(__float2bfloat16_rn(__fmul_rn(s_amax[m], r)));
+      }
+    }
+    __syncthreads();
+    // normalise the staged copy in place (bf16); unstaged reads apply it on use
+    for (int i = tid; i < M * H / 8; i += kFusedThreads) {
+      const int m = (i * 8) / H;
+      const float r = s_rn[m];
+      uint4 v = pl.x_staged ? x_s[i] : __ldcg(reinterpret_cast<const uint4*>(p.x) + i);
+      uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[t]));
+        const __nv_bfloat162 o = __floats2bfloat162_rn(__fmul_rn(f.x, r), __fmul_rn(f.y, r));
+        w[t] = *reinterpret_cast<const uint32_t*>(&o);
+      }
+      v = make_uint4(w[0], w[1], w[2], w[3]);
+      if (pl.x_staged) x_s[i] = v;
+      if (b == 0 && p.out_xn) reinterpret_cast<uint4*>(p.out_xn)[i] = v;
+    }
+    __syncthreads();
+  }
+  // normalised value of one bf16 pair read from global x (unstaged case)
+  auto xn2 = [&](uint32_t raw, int m) -> uint32_t {
+    if (!p.pre_rmsnorm || pl.x_staged) return raw;
+    const float r = s_rn[m];
+    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw));
+    const __nv_bfloat162 o = __floats2bfloat162_rn(__fmul_rn(f.x, r), __fmul_rn(f.y, r));
+    return *reinterpret_cast<const uint32_t*>(&o);
+  };
   if (tid < M) {
     const float a = s_amax[tid];
     s_xs[tid] = (a == 0.f) ? 1.f : __fdiv_rn(a, 448.f);
@@ -703,7 +757,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
     if (a != 0.f) {
       const float inv = __fdiv_rn(448.f, a);
       const uint4 v = pl.x_staged ? xsrc[i] : __ldcg(xsrc + i);
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+      const uint32_t w[4] = {xn2(v.x, m), xn2(v.y, m), xn2(v.z, m), xn2(v.w, m)};
       uint32_t q[2] = {0u, 0u};
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
@@ -734,7 +788,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
         for (int t = 0; t < 4; ++t) {
           if (t < mt) {
             const uint2* xrow = reinterpret_cast<const uint2*>(xsrc) + (size_t)(m0 + t) * (H / 4);
-            const uint2 q = pl.x_staged ? xrow[i] : __ldcg(xrow + i);
+            uint2 q = pl.x_staged ? xrow[i] : __ldcg(xrow + i);
+            q.x = xn2(q.x, m0 + t);
+            q.y = xn2(q.y, m0 + t);
             const float2 x01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&q.x));
             const float2 x23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&q.y));
             acc[t] = fmaf(x01.x, wv.x, acc[t]);

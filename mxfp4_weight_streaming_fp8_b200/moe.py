@@ -52,7 +52,7 @@ def lib() -> ctypes.CDLL:
         L.moe_create.restype = ctypes.c_int
         L.moe_load_experts.argtypes = [_vp] * 6 + [ctypes.c_uint32]
         L.moe_load_experts.restype = ctypes.c_int
-        L.moe_decode.argtypes = [_vp, _vp, ctypes.c_int32, _vp, _vp, _vp, _vp, _vp, _vp]
+        L.moe_decode.argtypes = [_vp, _vp, ctypes.c_int32, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
         L.moe_decode.restype = ctypes.c_int
         L.moe_sync_status.argtypes = [_vp, _vp]
         L.moe_sync_status.restype = ctypes.c_int
@@ -130,13 +130,15 @@ class MoELayer:
             raise MoEError(st, "moe_load_experts")
         self._weights = (router_w, w13_codes, w13_scales, w2_codes, w2_scales)
 
-    def decode_raw(self, x, M: int, y, stream=None, topk_ids=None, topk_w=None, xq=None, xscale=None) -> int:
+    def decode_raw(self, x, M: int, y, stream=None, topk_ids=None, topk_w=None, xq=None, xscale=None,
+                   xnorm=None) -> int:
         """moe_decode with explicit buffers; returns the status code."""
         return lib().moe_decode(self._ctx, _ptr(x), int(M), _ptr(y), _stream_handle(stream), _ptr(topk_ids),
-                                _ptr(topk_w), _ptr(xq), _ptr(xscale))
+                                _ptr(topk_w), _ptr(xq), _ptr(xscale), _ptr(xnorm))
 
     def decode(self, x, y=None, stream=None, routing: bool = False):
-        """x: bf16 [M, H] on the device. Returns y (and the routing outputs if asked)."""
+        """x: bf16 [M, H] on the device. Returns y, or with routing=True
+        (y, topk_ids, topk_w, xq, xscale[, xnorm when the context normalises])."""
         import torch
         M = x.shape[0]
         if y is None:
@@ -148,6 +150,8 @@ class MoELayer:
                      torch.empty((M, self.top_k), dtype=torch.float32, device=dev),
                      torch.empty((M, self.hidden), dtype=torch.uint8, device=dev),
                      torch.empty((M,), dtype=torch.float32, device=dev)]
+            if self.cfg.flags & MOE_FLAG_PRE_RMSNORM:
+                extra.append(torch.empty_like(x))
         st = self.decode_raw(x, M, y, stream, *extra)
         if st != MOE_OK:
             raise MoEError(st, "moe_decode")

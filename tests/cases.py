@@ -64,11 +64,15 @@ class Layer:
         return ctx
 
     def run(self, ctx):
-        y, ids, w, xq, xs = ctx.decode(self.x_d, routing=True)
+        out = ctx.decode(self.x_d, routing=True)
+        y, ids, w, xq, xs = out[:5]
         torch.cuda.synchronize()
         st = ctx.sync_status()
         assert st == moe.MOE_OK, moe.status_string(st)
-        return dict(y=y, ids=ids.cpu().numpy(), w=w.cpu().numpy(), q=xq.cpu().numpy(), s=xs.cpu().numpy())
+        res = dict(y=y, ids=ids.cpu().numpy(), w=w.cpu().numpy(), q=xq.cpu().numpy(), s=xs.cpu().numpy())
+        if len(out) > 5:
+            res["xn"] = out[5]
+        return res
 
 
 def min_gap(logits: np.ndarray, k: int) -> float:

@@ -60,7 +60,7 @@ def test_create_rejects_bad_config_without_gpu(L):
 
 
 def test_null_context_calls(L):
-    assert L.moe_decode(None, None, 1, None, None, None, None, None, None) == 1
+    assert L.moe_decode(None, None, 1, None, None, None, None, None, None, None) == 1
     assert L.moe_sync_status(None, None) == 1
     buf = ctypes.create_string_buffer(64)
     assert L.moe_query(None, buf, 64) == 1
