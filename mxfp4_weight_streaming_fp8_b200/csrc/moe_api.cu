@@ -198,7 +198,7 @@ moe_status moe_create(const moe_config* cfg, moe_ctx** out) {
   const size_t o_h = take(NP * I * sizeof(float));
   const size_t o_flog = take(MM * E * sizeof(float));
   const size_t o_rcnt = take(sizeof(unsigned long long));
-  const size_t o_gcnt = take(UMAX * sizeof(unsigned long long));
+  const size_t o_gcnt = take(UMAX * moe::kCounterStride * sizeof(unsigned long long));
   ctx->ws_bytes = off;
   if (cudaMalloc(&ctx->ws_base, ctx->ws_bytes) != cudaSuccess) {
     cudaGetLastError();

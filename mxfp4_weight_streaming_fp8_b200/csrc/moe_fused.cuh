@@ -19,21 +19,22 @@
 //     with back-off.
 //  3. Every CTA gathers all the logits and, redundantly, computes top-k,
 //     softmax and the expert union (A3, A4) in shared memory.
-//  4. Warp 0, lane 0 is the producer. It issues TMA bulk copies of this CTA's
-//     share of every union expert into two shared-memory rings:
+//  4. The CTA streams its share of every union expert into two
+//     shared-memory rings with TMA bulk copies:
 //       - gate/up: intermediate rows [I*b/G, I*(b+1)/G) of each expert, i.e.
 //         gate rows, up rows and their E8M0 scale bytes
 //       - down: output rows [H*b/G, H*(b+1)/G) of each expert, with scales
-//     Each active weight byte is read from HBM once, by one CTA.
-//  5. Warps 1..15 take items from one in-order queue: the gate/up items of
-//     entry u, then its down items, then entry u+1, in the order the
-//     producer issues the chunks, which rules out deadlock. For gate/up
-//     items (A5, A6) they decode E2M1 in registers, run f16x2 FMAs on exact
-//     products, apply the E8M0 scale in fp32, then SwiGLU, and write h to L2.
-//     When a CTA has finished entry u, it arrives on that entry's grid
-//     counter. The first down item of u (A7) waits on the counter's flag and
-//     stages h once into shared memory for the CTA, so down work on early
-//     experts overlaps gate/up work on later ones.
+//     Each active weight byte is read from HBM once, by one CTA. A bulk copy
+//     costs its issuing thread about a hundred nanoseconds, so the first use
+//     of every slot is issued by all 16 warps at once; refills of a drained
+//     slot come from warp 0 (lane 0 gate/up, lane 1 down).
+//  5. Warps 1..15 first drain an in-order queue of gate/up items (A5, A6):
+//     they decode E2M1 in registers, run f16x2 FMAs on exact products, apply
+//     the E8M0 scale in fp32, then SwiGLU, and write h to L2. When a CTA has
+//     finished entry u, it arrives on that entry's grid counter. Then they
+//     drain an in-order queue of down items (A7). The first down item of u
+//     waits on the counter and stages h once into shared memory for the CTA;
+//     the other items of u wait for that.
 //  6. Each CTA combines its output rows in slot order (A8) and writes bf16 y.
 //
 // Every wait is bounded: on timeout the kernel sets the status word and goes
@@ -50,10 +51,9 @@ constexpr int kConsumers = kFusedWarps - 1;  // warp 0 produces
 constexpr int kGuRowsPerItem = 2;           // intermediate rows per gate/up item
 constexpr int kDownRowsPerItem = 6;         // output rows per down item
 constexpr int kHPairs = 4;                  // (token, slot) pairs of one expert whose h is staged in smem
-constexpr int kGuWarps = 8;                 // consumer warps 1..8 take gate/up items
-constexpr int kDownWarps = kConsumers - kGuWarps;  // warps 9..15 take down items
 constexpr int kMaxRowsPerCta = 8;           // router rows a CTA may own (E <= 8 * G)
 constexpr int kMaxSlots = 64;
+constexpr int kCounterStride = 16;          // u64 words between per-entry counters (one 128-byte line)
 
 // Launch-invariant plan computed on the host at moe_create.
 struct FusedPlan {
@@ -75,9 +75,14 @@ struct FusedPlan {
 struct FusedWs {
   float* logits;                  // [maxM][E]
   unsigned long long* route_cnt;  // router arrivals; += G per launch
-  unsigned long long* gu_cnt;     // [max_union] gate/up arrivals per union entry; += G per launch
+  unsigned long long* gu_cnt;     // [max_union][kCounterStride] gate/up arrivals per entry; += G per launch
   unsigned* epoch;                // launch counter
 };
+
+// Counter of union entry u, alone on its L2 line.
+__host__ __device__ __forceinline__ unsigned long long* gu_counter(const FusedWs& fw, int u) {
+  return fw.gu_cnt + (size_t)u * kCounterStride;
+}
 
 // ---------------------------------------------------------------- PTX helpers
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -490,11 +495,16 @@ __device__ __forceinline__ void d_item(const Params& p, const DChunk& ch, int a,
           hv[4 * t] = __uint_as_float(q.x); hv[4 * t + 1] = __uint_as_float(q.y);
           hv[4 * t + 2] = __uint_as_float(q.z); hv[4 * t + 3] = __uint_as_float(q.w);
         }
-        // the rescale must cover the whole vector: reduce over all passes
-        for (int b1 = 0; b1 < nblk; b1 += 32) {
-          const int bk = b1 + lane;
-          if (bk < nblk)
-            for (int t = 0; t < 32; ++t) mx = fmaxf(mx, fabsf(__ldcg(hp + bk * 32 + t)));
+        if (nblk <= 32) {
+#pragma unroll
+          for (int t = 0; t < 32; ++t) mx = fmaxf(mx, fabsf(hv[t]));
+        } else {
+          // the rescale must cover the whole vector: reduce over all passes
+          for (int b1 = 0; b1 < nblk; b1 += 32) {
+            const int bk = b1 + lane;
+            if (bk < nblk)
+              for (int t = 0; t < 32; ++t) mx = fmaxf(mx, fabsf(__ldcg(hp + bk * 32 + t)));
+          }
         }
         const int t = h_rescale_exp(warp_max(mx));
         const float up = ldexpf(1.f, t);
@@ -921,61 +931,82 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
   __syncthreads();
   const int U = s_int[0];
 
+  // ---------------- weight stream. Each bulk copy costs its issuing thread
+  //   about a hundred nanoseconds, so the first use of every ring slot is
+  //   issued by all warps in parallel (lane 0 of warp w takes entries w, w+16,
+  //   ...; gate/up chunks first, then down chunks); later uses wait for their
+  //   slot to drain and are issued by warp 0: lane 0 for gate/up, lane 1 for
+  //   down, so a full down ring never holds back gate/up data.
+  auto issue_gu = [&](int u) {
+    const int e = s_union[u];
+    const int slot = u % pl.ns_gu;
+    uint8_t* sp = ring_gu + (size_t)slot * pl.slot_gu;
+    GuChunk ch;
+    size_t ga0, ua0;
+    unsigned gn, un;
+    const unsigned bytes = gu_layout(p, e, n0, nr, sp, &ch, &ga0, &gn, &ua0, &un);
+    mbar_expect_tx(full_gu + slot, bytes);
+    const size_t grow = (size_t)e * 2 * I + n0, urow = grow + I;
+    const unsigned codes = (unsigned)(nr * H / 2);
+    tma_load_1d(sp, p.w13c + grow * (H / 2), codes, full_gu + slot);
+    tma_load_1d(sp + codes, p.w13c + urow * (H / 2), codes, full_gu + slot);
+    tma_load_1d(sp + 2 * codes, p.w13s + ga0, gn, full_gu + slot);
+    tma_load_1d(sp + 2 * codes + gn, p.w13s + ua0, un, full_gu + slot);
+  };
+  auto issue_d = [&](int u) {
+    const int e = s_union[u];
+    const int slot = u % pl.ns_d;
+    uint8_t* sp = ring_d + (size_t)slot * pl.slot_d;
+    DChunk ch;
+    size_t sa0;
+    unsigned sn;
+    const unsigned bytes = d_layout(p, e, r0, nrd, sp, &ch, &sa0, &sn);
+    mbar_expect_tx(full_d + slot, bytes);
+    const unsigned codes = (unsigned)(nrd * I / 2);
+    tma_load_1d(sp, p.w2c + ((size_t)e * H + r0) * (I / 2), codes, full_d + slot);
+    tma_load_1d(sp + codes, p.w2s + sa0, sn, full_d + slot);
+  };
+  const int n_gu0 = (nr > 0) ? min(U, pl.ns_gu) : 0;
+  const int n_d0 = (nrd > 0) ? min(U, pl.ns_d) : 0;
+  if (lane == 0 && (warp < n_gu0 || warp < n_d0)) {
+    // ring_gu and ring_d were read and written through the generic proxy
+    // during routing; order that before the async-proxy (TMA) writes
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    for (int u = warp; u < n_gu0; u += kFusedWarps) issue_gu(u);
+    for (int u = warp; u < n_d0; u += kFusedWarps) issue_d(u);
+  }
   if (warp == 0) {
-    // ---------------- producer: gate/up then down slice of each entry, in
-    //                  the order the consumers take them
-    if (lane == 0) {
-      // ring_gu and ring_d were read and written through the generic proxy
-      // during routing; order that before the async-proxy (TMA) writes
+    if (lane == 0 && nr > 0 && n_gu0 < U) {
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      for (int u = 0; u < U; ++u) {
-        const int e = s_union[u];
-        if (nr > 0) {
-          const int slot = u % pl.ns_gu, use = u / pl.ns_gu;
-          if (use > 0) mbar_wait(empty_gu + slot, (use - 1) & 1, p);
-          uint8_t* sp = ring_gu + (size_t)slot * pl.slot_gu;
-          GuChunk ch;
-          size_t ga0, ua0;
-          unsigned gn, un;
-          const unsigned bytes = gu_layout(p, e, n0, nr, sp, &ch, &ga0, &gn, &ua0, &un);
-          mbar_expect_tx(full_gu + slot, bytes);
-          const size_t grow = (size_t)e * 2 * I + n0, urow = grow + I;
-          const unsigned codes = (unsigned)(nr * H / 2);
-          tma_load_1d(sp, p.w13c + grow * (H / 2), codes, full_gu + slot);
-          tma_load_1d(sp + codes, p.w13c + urow * (H / 2), codes, full_gu + slot);
-          tma_load_1d(sp + 2 * codes, p.w13s + ga0, gn, full_gu + slot);
-          tma_load_1d(sp + 2 * codes + gn, p.w13s + ua0, un, full_gu + slot);
-        }
-        if (nrd > 0) {
-          const int slot = u % pl.ns_d, use = u / pl.ns_d;
-          if (use > 0) mbar_wait(empty_d + slot, (use - 1) & 1, p);
-          uint8_t* sp = ring_d + (size_t)slot * pl.slot_d;
-          DChunk ch;
-          size_t sa0;
-          unsigned sn;
-          const unsigned bytes = d_layout(p, e, r0, nrd, sp, &ch, &sa0, &sn);
-          mbar_expect_tx(full_d + slot, bytes);
-          const unsigned codes = (unsigned)(nrd * I / 2);
-          tma_load_1d(sp, p.w2c + ((size_t)e * H + r0) * (I / 2), codes, full_d + slot);
-          tma_load_1d(sp + codes, p.w2s + sa0, sn, full_d + slot);
-        }
+      for (int u = n_gu0; u < U; ++u) {
+        const int slot = u % pl.ns_gu, use = u / pl.ns_gu;
+        mbar_wait(empty_gu + slot, (use - 1) & 1, p);
+        issue_gu(u);
+      }
+    }
+    if (lane == 1 && nrd > 0 && n_d0 < U) {
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      for (int u = n_d0; u < U; ++u) {
+        const int slot = u % pl.ns_d, use = u / pl.ns_d;
+        mbar_wait(empty_d + slot, (use - 1) & 1, p);
+        issue_d(u);
       }
     }
     return;
   }
 
-  // ---------------- consumers. Two groups with their own in-order queues, so
-  //   a down item waiting on other CTAs never holds up gate/up work:
-  //   warps 1..kGuWarps take gate/up items (entry-major), the rest take down
-  //   items (entry-major). Gate/up items depend only on their chunk; down
-  //   items on their chunk and on gate/up of the entry on every CTA, which
-  //   never waits on down work, so neither queue can deadlock.
+  // ---------------- consumers. Two in-order queues: every consumer warp
+  //   first takes gate/up items (entry-major) until that queue is empty, then
+  //   down items (entry-major). Gate/up items depend only on their chunk, so
+  //   the first queue always drains; down items depend on their chunk and on
+  //   gate/up of the entry on every CTA, which never waits on down work, so
+  //   the second cannot deadlock either.
   const unsigned long long tgt = (unsigned long long)epoch * G;
-  if (warp <= kGuWarps) {
+  {
     const int total = U * gu_items;
     if (gu_items == 0 && warp == 1 && lane == 0) {
       // no gate/up rows here: this CTA's part of every entry is trivially done
-      for (int u = 0; u < U; ++u) grid_arrive(fw.gu_cnt + u);
+      for (int u = 0; u < U; ++u) grid_arrive(gu_counter(fw, u));
     }
     for (;;) {
       int it = 0;
@@ -1000,11 +1031,12 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
         // acq_rel at CTA scope: the warp completing the entry sees every
         // other warp's h stores, then releases them GPU-wide
         const unsigned done = atom_add_acqrel_cta_smem(reinterpret_cast<unsigned*>(s_cnt + u), 1u) + 1u;
-        if ((int)done == gu_items) grid_arrive(fw.gu_cnt + u);
+        if ((int)done == gu_items) grid_arrive(gu_counter(fw, u));
       }
       __syncwarp();
     }
-  } else {
+  }
+  {
     const int total = U * d_items;
     for (;;) {
       int it = 0;
@@ -1023,7 +1055,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
       if (gd == 0) {
         // first down item of the entry: wait for gate/up of the entry on all
         // CTAs, then stage h once for the CTA
-        if (lane == 0) grid_wait(fw.gu_cnt + u, tgt, p);
+        if (lane == 0) grid_wait(gu_counter(fw, u), tgt, p);
         __syncwarp();
         if (pe - pb <= pl.hpairs) stage_h(p, pb, pe, hbuf, hscale);
         __syncwarp();
@@ -1056,7 +1088,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
   }
   if (b == 0 && ct == 0) {
     // keep every entry's counter at epoch * G for the next launch
-    for (int u = U; u < pl.max_union; ++u) red_release_add_u64(fw.gu_cnt + u, (unsigned long long)G);
+    for (int u = U; u < pl.max_union; ++u) red_release_add_u64(gu_counter(fw, u), (unsigned long long)G);
     st_relaxed_u32(fw.epoch, epoch);
   }
 }
