@@ -64,6 +64,11 @@ bool make_plan(const moe_config& c, int sm_count, size_t smem_limit, moe::FusedP
   pl->rpc_max = (int)nrd_max;
   pl->slot_gu = (int)align_up(nr_max * H + 2 * (nr_max * H / 32 + 32), 128);
   pl->slot_d = (int)align_up(nrd_max * (I / 2) + nrd_max * (I / 32) + 32, 128);
+  // MMA partials of entries with several pairs: per gate/up slot, one float4
+  // per lane for each (K chunk = item, 8-row group, 8-pair tile)
+  const size_t gu_items_max = (nr_max + moe::kGuRowsPerItem - 1) / moe::kGuRowsPerItem;
+  pl->part_ct = (int)std::min<size_t>(moe::kMaxPairTiles, (MM + 7) / 8);
+  pl->part_slot = (MM >= (size_t)moe::kMmaMinPairs) ? (int)(gu_items_max * ((nr_max + 7) / 8) * pl->part_ct * 32 * 16) : 0;
   pl->hpairs = (int)std::min<size_t>(moe::kHPairs, MM);
   pl->hslot = (int)align_up((size_t)pl->hpairs * I * 2 + moe::kHPairs * 4, 16);
   const size_t kMaxSlots = moe::kMaxSlots;
@@ -84,7 +89,7 @@ bool make_plan(const moe_config& c, int sm_count, size_t smem_limit, moe::FusedP
   if (off >= smem_limit) return false;
   // each down slot carries its staged h
   const size_t room = smem_limit - off;
-  const size_t per = pl->slot_gu + pl->slot_d + pl->hslot;
+  const size_t per = pl->slot_gu + pl->part_slot + pl->slot_d + pl->hslot;
   size_t n_both = room / per;
   if (n_both < 2) return false;
   size_t ns_gu, ns_d;
@@ -92,7 +97,7 @@ bool make_plan(const moe_config& c, int sm_count, size_t smem_limit, moe::FusedP
     ns_gu = ns_d = UMAX;
   } else {
     ns_gu = ns_d = n_both;
-    ns_gu += (room - n_both * per) / pl->slot_gu;
+    ns_gu += (room - n_both * per) / (pl->slot_gu + pl->part_slot);
     if (ns_gu > UMAX) ns_gu = UMAX;
   }
   if (ns_gu > kMaxSlots) ns_gu = kMaxSlots;
@@ -101,6 +106,8 @@ bool make_plan(const moe_config& c, int sm_count, size_t smem_limit, moe::FusedP
   pl->ns_d = (int)ns_d;
   pl->o_h = (int)off;
   off = align_up(off + ns_d * pl->hslot, 128);
+  pl->o_part = (int)off;
+  off = align_up(off + ns_gu * (size_t)pl->part_slot, 128);
   // ring_gu also holds the router rows of the CTA and then the gathered
   // logits [M][E] fp32 between routing and the first weight chunk
   pl->wr_bytes_max = (int)(((E + G - 1) / G) * H * 4);

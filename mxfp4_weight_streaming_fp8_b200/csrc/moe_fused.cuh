@@ -53,6 +53,8 @@ constexpr int kDownRowsPerItem = 6;         // output rows per down item
 constexpr int kHPairs = 4;                  // (token, slot) pairs of one expert whose h is staged in smem
 constexpr int kMaxRowsPerCta = 8;           // router rows a CTA may own (E <= 8 * G)
 constexpr int kMaxSlots = 64;
+constexpr int kMaxPairTiles = 4;            // 8-pair MMA column tiles per entry (32 pairs)
+constexpr int kMmaMinPairs = 3;             // entries with at least this many pairs take the MMA gate/up path
 constexpr int kCounterStride = 16;          // u64 words between per-entry counters (one 128-byte line)
 
 // Launch-invariant plan computed on the host at moe_create.
@@ -65,7 +67,9 @@ struct FusedPlan {
   int hslot;            // bytes of staged h per down slot
   int hpairs;           // pairs staged per down slot (min(kHPairs, max_tokens))
   // shared memory offsets (bytes)
-  int o_bar, o_misc, o_ids, o_w, o_pm, o_ppos, o_union, o_poff, o_cnt, o_act, o_dsm, o_h, o_ring_gu, o_ring_d;
+  int o_bar, o_misc, o_ids, o_w, o_pm, o_ppos, o_union, o_poff, o_cnt, o_act, o_dsm, o_h, o_part, o_ring_gu, o_ring_d;
+  int part_slot;        // bytes of MMA partials per gate/up slot (0: one token, never used)
+  int part_ct;          // 8-pair column tiles a slot's partials hold (min(kMaxPairTiles, max_tokens / 8 rounded up))
   int smem_bytes;
   int wr_bytes_max;     // router rows staged per CTA (alias ring_gu)
   int x_staged;         // bf16 x fits in ring_d and is staged there during routing
@@ -353,6 +357,78 @@ __device__ __forceinline__ void gu_item(const Params& p, const GuChunk& ch, int 
     for (int r = 0; r < kGuRowsPerItem; ++r) {
       const float g = ag[r] * s, u = au[r] * s;
       if (lane == 0 && r < cnt) p.ws.h[(size_t)pp * p.I + n0 + a + r] = g / (1.f + expf(-g)) * u;
+    }
+  }
+}
+
+// D = A(16x16, f16, row) * B(16x8, f16, col) + C, fp32 accumulate.
+__device__ __forceinline__ void mma_f16_16816(float d[4], const uint32_t a[4], uint32_t b0, uint32_t b1,
+                                              const float c[4]) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%10,%11,%12,%13};"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(c[0]), "f"(c[1]), "f"(c[2]),
+        "f"(c[3]));
+}
+
+// Gate/up of an expert with several (token, slot) pairs: warp MMAs
+// (m16n8k16, f16 x f16 -> fp32) decode each weight once for all pairs. The
+// A tile's rows 0..7 are gate rows r0g.. of the chunk and rows 8..15 the up
+// rows with the same index (nrg <= 8 valid); the B tile's 8 columns are
+// pairs pb + 8*ct.. (up to kMaxPairTiles tiles). Within each 32-element
+// scale block lane (g, t) supplies elements 8t..8t+7: 8t+4s+{0,1} as the K
+// positions 2t, 2t+1 of step s and 8t+4s+{2,3} as 2t+8, 2t+9, for A and B
+// alike, so each product pairs the same element; E2M1 and E4M3 are exact in
+// f16. Each scale block is a fresh two-step MMA scaled in fp32 by the E8M0
+// scales of gate row g and up row g. acc[4*ct + i]: gate (i = 0, 1) and up
+// (i = 2, 3) of row g for pairs pb + 8*ct + 2t + (i & 1).
+__device__ __forceinline__ void gu_mma_slice(const Params& p, const GuChunk& ch, int r0g, int nrg, int kb0, int kb1,
+                                             int pb, int pe, const int* s_pm, const uint8_t* act,
+                                             float acc[4 * kMaxPairTiles]) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  const int H = p.H, hs = H / 32;
+  const int np = pe - pb, nct = min(kMaxPairTiles, (np + 7) >> 3);
+  const bool rv = g < nrg;
+  const uint8_t* gc = ch.gc + (size_t)(r0g + g) * (H / 2) + 4 * t;
+  const uint8_t* uc = ch.uc + (size_t)(r0g + g) * (H / 2) + 4 * t;
+  const uint8_t* gs = ch.gs + (size_t)(r0g + g) * hs;
+  const uint8_t* us = ch.us + (size_t)(r0g + g) * hs;
+  const uint8_t* br[kMaxPairTiles];
+#pragma unroll
+  for (int ct = 0; ct < kMaxPairTiles; ++ct) {
+    const int q = 8 * ct + g;
+    br[ct] = (q < np) ? act + (size_t)s_pm[pb + q] * H + 8 * t : nullptr;
+  }
+#pragma unroll
+  for (int i = 0; i < 4 * kMaxPairTiles; ++i) acc[i] = 0.f;
+  const float z[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int kb = kb0; kb < kb1; ++kb) {
+    uint32_t fg[4] = {0u, 0u, 0u, 0u}, fu[4] = {0u, 0u, 0u, 0u};
+    float sg = 0.f, su = 0.f;
+    if (rv) {
+      e2m1x8_to_f16x2x4(*reinterpret_cast<const uint32_t*>(gc + kb * 16), fg);
+      e2m1x8_to_f16x2x4(*reinterpret_cast<const uint32_t*>(uc + kb * 16), fu);
+      sg = e8m0_to_f32(gs[kb]);
+      su = e8m0_to_f32(us[kb]);
+    }
+    const uint32_t a0[4] = {fg[0], fu[0], fg[1], fu[1]};
+    const uint32_t a1[4] = {fg[2], fu[2], fg[3], fu[3]};
+#pragma unroll
+    for (int ct = 0; ct < kMaxPairTiles; ++ct) {
+      if (ct >= nct) break;
+      uint4 bv = make_uint4(0u, 0u, 0u, 0u);
+      if (br[ct]) {
+        const uint2 c = *reinterpret_cast<const uint2*>(br[ct] + kb * 32);
+        bv = make_uint4(e4m3x2_to_f16x2((uint16_t)(c.x & 0xFFFFu)), e4m3x2_to_f16x2((uint16_t)(c.x >> 16)),
+                        e4m3x2_to_f16x2((uint16_t)(c.y & 0xFFFFu)), e4m3x2_to_f16x2((uint16_t)(c.y >> 16)));
+      }
+      float d[4];
+      mma_f16_16816(d, a0, bv.x, bv.y, z);
+      mma_f16_16816(d, a1, bv.z, bv.w, d);
+      acc[4 * ct + 0] = fmaf(d[0], sg, acc[4 * ct + 0]);
+      acc[4 * ct + 1] = fmaf(d[1], sg, acc[4 * ct + 1]);
+      acc[4 * ct + 2] = fmaf(d[2], su, acc[4 * ct + 2]);
+      acc[4 * ct + 3] = fmaf(d[3], su, acc[4 * ct + 3]);
     }
   }
 }
@@ -756,33 +832,6 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
     const __nv_bfloat162 o = __floats2bfloat162_rn(__fmul_rn(f.x, r), __fmul_rn(f.y, r));
     return *reinterpret_cast<const uint32_t*>(&o);
   };
-  if (tid < M) {
-    const float a = s_amax[tid];
-    s_xs[tid] = (a == 0.f) ? 1.f : __fdiv_rn(a, 448.f);
-  }
-  for (int i = tid; i < M * H / 8; i += kFusedThreads) {
-    const int m = (i * 8) / H;
-    const float a = s_amax[m];
-    uint2 out = make_uint2(0u, 0u);
-    if (a != 0.f) {
-      const float inv = __fdiv_rn(448.f, a);
-      const uint4 v = pl.x_staged ? xsrc[i] : __ldcg(xsrc + i);
-      const uint32_t w[4] = {xn2(v.x, m), xn2(v.y, m), xn2(v.z, m), xn2(v.w, m)};
-      uint32_t q[2] = {0u, 0u};
-#pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[t]));
-        const uint32_t c2 = f32x2_to_e4m3x2(__fmul_rn(f.x, inv), __fmul_rn(f.y, inv));
-        q[t >> 1] |= c2 << (16 * (t & 1));
-      }
-      out = make_uint2(q[0], q[1]);
-    }
-    *reinterpret_cast<uint2*>(act + (size_t)i * 8) = out;
-    if (b == 0 && p.out_xq) *reinterpret_cast<uint2*>(p.out_xq + (size_t)i * 8) = out;
-  }
-  __syncthreads();
-  if (b == 0 && p.out_xscale && tid < M) p.out_xscale[tid] = s_xs[tid];
-
   // ---- A2: logits of this CTA's router rows (ne <= kMaxRowsPerCta), four
   //          tokens per pass; warp partials go to shared memory and one block
   //          barrier per pass ends it
@@ -838,10 +887,37 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
   }
   // grid-wide: every CTA's logits are in L2 once the router count reaches
   // epoch * G (the last arrival publishes the epoch to the flag copies)
-  if (tid == 0) {
-    grid_arrive(fw.route_cnt);
-    grid_wait(fw.route_cnt, (unsigned long long)(p.force_stall ? epoch + 0x40000000u : epoch) * G, p);
+  if (tid == 0) grid_arrive(fw.route_cnt);
+  // ---- A1 (second half): E4M3 codes and scales, done while the other CTAs'
+  //      logits arrive (the router works on the bf16 x, not on the codes)
+  if (tid < M) {
+    const float a = s_amax[tid];
+    s_xs[tid] = (a == 0.f) ? 1.f : __fdiv_rn(a, 448.f);
   }
+  for (int i = tid; i < M * H / 8; i += kFusedThreads) {
+    const int m = (i * 8) / H;
+    const float a = s_amax[m];
+    uint2 out = make_uint2(0u, 0u);
+    if (a != 0.f) {
+      const float inv = __fdiv_rn(448.f, a);
+      const uint4 v = pl.x_staged ? xsrc[i] : __ldcg(xsrc + i);
+      const uint32_t w[4] = {xn2(v.x, m), xn2(v.y, m), xn2(v.z, m), xn2(v.w, m)};
+      uint32_t q[2] = {0u, 0u};
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[t]));
+        const uint32_t c2 = f32x2_to_e4m3x2(__fmul_rn(f.x, inv), __fmul_rn(f.y, inv));
+        q[t >> 1] |= c2 << (16 * (t & 1));
+      }
+      out = make_uint2(q[0], q[1]);
+    }
+    *reinterpret_cast<uint2*>(act + (size_t)i * 8) = out;
+    if (b == 0 && p.out_xq) *reinterpret_cast<uint2*>(p.out_xq + (size_t)i * 8) = out;
+  }
+  if (b == 0 && p.out_xscale && tid < M) p.out_xscale[tid] = s_xs[tid];
+
+  if (tid == 0)
+    grid_wait(fw.route_cnt, (unsigned long long)(p.force_stall ? epoch + 0x40000000u : epoch) * G, p);
   pdl_launch_dependents();
   __syncthreads();
 
@@ -1022,8 +1098,64 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
       size_t ga0, ua0;
       unsigned gn, un;
       gu_layout(p, s_union[u], n0, nr, ring_gu + (size_t)slot * pl.slot_gu, &ch, &ga0, &gn, &ua0, &un);
+      const int pb = s_poff[u], pe = s_poff[u + 1];
+      if (pe - pb >= kMmaMinPairs && pl.part_slot > 0) {
+        // several pairs: the entry's items split K; each runs warp MMAs over
+        // all rows and pairs, and the last one to finish sums the partials
+        // in chunk order (deterministic), applies SwiGLU and writes h
+        const int nkb = H / 32, nrg = (nr + 7) >> 3, nct = min(pl.part_ct, (pe - pb + 7) >> 3);
+        const int kb0 = g * nkb / gu_items, kb1 = (g + 1) * nkb / gu_items;
+        float4* part = reinterpret_cast<float4*>(smem + pl.o_part + (size_t)slot * pl.part_slot);
+        for (int rg = 0; rg < nrg; ++rg) {
+          float acc[4 * kMaxPairTiles];
+          gu_mma_slice(p, ch, 8 * rg, min(8, nr - 8 * rg), kb0, kb1, pb, pe, s_pm, act, acc);
+#pragma unroll
+          for (int ct = 0; ct < kMaxPairTiles; ++ct)
+            if (ct < nct)
+              part[((g * nrg + rg) * pl.part_ct + ct) * 32 + lane] =
+                  make_float4(acc[4 * ct], acc[4 * ct + 1], acc[4 * ct + 2], acc[4 * ct + 3]);
+        }
+        __syncwarp();
+        unsigned done = 0;
+        if (lane == 0) done = atom_add_acqrel_cta_smem(reinterpret_cast<unsigned*>(s_cnt + u), 1u) + 1u;
+        done = __shfl_sync(0xffffffffu, done, 0);
+        if ((int)done == gu_items) {
+          const int gq = lane >> 2, tq = lane & 3;
+          for (int rg = 0; rg < nrg; ++rg) {
+            const int row = 8 * rg + gq;
+            for (int ct = 0; ct < nct; ++ct) {
+              float4 v = part[(rg * pl.part_ct + ct) * 32 + lane];
+              for (int c = 1; c < gu_items; ++c) {
+                const float4 w = part[((c * nrg + rg) * pl.part_ct + ct) * 32 + lane];
+                v.x += w.x; v.y += w.y; v.z += w.z; v.w += w.w;
+              }
+              const float gg[2] = {v.x, v.y}, uu[2] = {v.z, v.w};
+#pragma unroll
+              for (int i = 0; i < 2; ++i) {
+                const int q = 8 * ct + 2 * tq + i;
+                if (q < pe - pb && row < nr) {
+                  const float sx = s_xs[s_pm[pb + q]];
+                  const float gv = gg[i] * sx, uv = uu[i] * sx;
+                  p.ws.h[(size_t)(pb + q) * I + n0 + row] = gv / (1.f + expf(-gv)) * uv;
+                }
+              }
+            }
+          }
+          __syncwarp();
+          // orders the warp's h stores (through the warp barrier) before the
+          // GPU-wide arrival for the entry
+          if (lane == 0) grid_arrive(gu_counter(fw, u));
+        }
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(empty_gu + slot);
+          atomicAdd(done_gu + slot, 1u);
+        }
+        __syncwarp();
+        continue;
+      }
       const int a = g * kGuRowsPerItem, cnt = min(kGuRowsPerItem, nr - a);
-      gu_item(p, ch, a, cnt, n0, s_poff[u], s_poff[u + 1], s_pm, act, s_xs);
+      gu_item(p, ch, a, cnt, n0, pb, pe, s_pm, act, s_xs);
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(empty_gu + slot);
