@@ -26,11 +26,15 @@
 //       - down: output rows [H*b/G, H*(b+1)/G) of each expert, with scales
 //     Each active weight byte is read from HBM once, by one CTA. A bulk copy
 //     costs its issuing thread about a hundred nanoseconds, so the first use
-//     of every slot is issued by all 16 warps at once; refills of a drained
-//     slot come from warp 0 (lane 0 gate/up, lane 1 down).
+//     of every slot is issued by all 16 warps at once; refills of drained
+//     slots come from one thread of warp 0 that polls both rings.
 //  5. Warps 1..15 first drain an in-order queue of gate/up items (A5, A6):
-//     they decode E2M1 in registers, run f16x2 FMAs on exact products, apply
-//     the E8M0 scale in fp32, then SwiGLU, and write h to L2. When a CTA has
+//     for an expert with one or two (token, slot) pairs they decode E2M1 in
+//     registers, run f16x2 FMAs on exact products per pair, apply
+//     the E8M0 scale in fp32, then SwiGLU, and write h to L2. An expert
+//     with three or more pairs splits K over its items instead: each runs
+//     warp MMAs (m16n8k16, f16) over all rows and pairs, so a weight is
+//     decoded once, and the last item sums the partials. When a CTA has
 //     finished entry u, it arrives on that entry's grid counter. Then they
 //     drain an in-order queue of down items (A7). The first down item of u
 //     waits on the counter and stages h once into shared memory for the CTA;
@@ -115,6 +119,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, unsigned parity) {
       "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;}"
       : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity), "r"(20000u) : "memory");
+  return ok != 0;
+}
+
+// Non-blocking test of an mbarrier phase (no suspension).
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, unsigned parity) {
+  uint32_t ok;
+  asm volatile(
+      "{.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;}"
+      : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
   return ok != 0;
 }
 
@@ -1011,8 +1026,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
   //   about a hundred nanoseconds, so the first use of every ring slot is
   //   issued by all warps in parallel (lane 0 of warp w takes entries w, w+16,
   //   ...; gate/up chunks first, then down chunks); later uses wait for their
-  //   slot to drain and are issued by warp 0: lane 0 for gate/up, lane 1 for
-  //   down, so a full down ring never holds back gate/up data.
+  //   slot to drain and are issued by lane 0 of warp 0.
   auto issue_gu = [&](int u) {
     const int e = s_union[u];
     const int slot = u % pl.ns_gu;
@@ -1052,20 +1066,34 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
     for (int u = warp; u < n_d0; u += kFusedWarps) issue_d(u);
   }
   if (warp == 0) {
-    if (lane == 0 && nr > 0 && n_gu0 < U) {
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      for (int u = n_gu0; u < U; ++u) {
-        const int slot = u % pl.ns_gu, use = u / pl.ns_gu;
-        mbar_wait(empty_gu + slot, (use - 1) & 1, p);
-        issue_gu(u);
-      }
-    }
-    if (lane == 1 && nrd > 0 && n_d0 < U) {
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      for (int u = n_d0; u < U; ++u) {
-        const int slot = u % pl.ns_d, use = u / pl.ns_d;
-        mbar_wait(empty_d + slot, (use - 1) & 1, p);
-        issue_d(u);
+    // refills of drained slots (more union entries than slots): one thread
+    // polls both rings without suspending and issues whichever slot drains
+    // first, in entry order per ring, so neither ring waits behind the other
+    if (lane == 0) {
+      int ug = (nr > 0) ? n_gu0 : U, ud = (nrd > 0) ? n_d0 : U;
+      if (ug < U || ud < U) {
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        long long t0 = clock64();
+        while (ug < U || ud < U) {
+          bool moved = false;
+          if (ug < U && mbar_test(empty_gu + ug % pl.ns_gu, (ug / pl.ns_gu - 1) & 1)) {
+            issue_gu(ug++);
+            moved = true;
+          }
+          if (ud < U && mbar_test(empty_d + ud % pl.ns_d, (ud / pl.ns_d - 1) & 1)) {
+            issue_d(ud++);
+            moved = true;
+          }
+          if (moved) {
+            t0 = clock64();
+          } else {
+            __nanosleep(64);
+            if (clock64() - t0 > p.spin_limit) {
+              atomicOr(p.ws.ctrl, kStatusTimeout);
+              break;
+            }
+          }
+        }
       }
     }
     return;
