@@ -428,7 +428,7 @@ def main():
     ap.add_argument("--tokens", type=int, default=1)
     ap.add_argument("--routing", default="gap", choices=["gap", "zipf", "distinct", "shared", "natural"])
     ap.add_argument("--layers", type=int, default=POOL_LAYERS)
-    ap.add_argument("--cpu-layers", type=int, default=6)
+    ap.add_argument("--cpu-layers", type=int, default=16)
     ap.add_argument("--ref-layers", type=int, default=4)
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--variant", choices=["fused", "split"], default="fused")

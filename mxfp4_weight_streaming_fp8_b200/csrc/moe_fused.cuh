@@ -59,6 +59,7 @@ constexpr int kMaxRowsPerCta = 8;           // router rows a CTA may own (E <= 8
 constexpr int kMaxSlots = 64;
 constexpr int kMaxPairTiles = 4;            // 8-pair MMA column tiles per entry (32 pairs)
 constexpr int kMmaMinPairs = 3;             // entries with at least this many pairs take the MMA gate/up path
+constexpr int kDownLag = 8;                 // down items of entry k follow the gate/up items of entry k + kDownLag
 constexpr int kCounterStride = 16;          // u64 words between per-entry counters (one 128-byte line)
 
 // Launch-invariant plan computed on the host at moe_create.
@@ -1106,18 +1107,42 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
   //   gate/up of the entry on every CTA, which never waits on down work, so
   //   the second cannot deadlock either.
   const unsigned long long tgt = (unsigned long long)epoch * G;
-  {
-    const int total = U * gu_items;
-    if (gu_items == 0 && warp == 1 && lane == 0) {
-      // no gate/up rows here: this CTA's part of every entry is trivially done
-      for (int u = 0; u < U; ++u) grid_arrive(gu_counter(fw, u));
+  if (gu_items == 0 && warp == 1 && lane == 0) {
+    // no gate/up rows here: this CTA's part of every entry is trivially done
+    for (int u = 0; u < U; ++u) grid_arrive(gu_counter(fw, u));
+  }
+  // One in-order queue: round k holds the gate/up items of entry k, then the
+  // down items of entry k - kDownLag, so down work on early entries overlaps
+  // gate/up work on later ones. Gate/up items wait only for their chunk, and
+  // a down item is handed out only after every gate/up item of its entry,
+  // here and (by the same order) on every CTA, so the queue cannot deadlock.
+  const int DL = min(kDownLag, U);
+  const int n1 = DL * gu_items, per2 = gu_items + d_items, n2 = (U - DL) * per2;
+  const int total = U * (gu_items + d_items);
+  for (;;) {
+    int it = 0;
+    if (lane == 0) it = atomicAdd(&s_int[2], 1);
+    it = __shfl_sync(0xffffffffu, it, 0);
+    if (it >= total) break;
+    bool is_down;
+    int u, sub;
+    if (it < n1) {
+      is_down = false;
+      u = it / gu_items;
+      sub = it - u * gu_items;
+    } else if (it < n1 + n2) {
+      const int r = (it - n1) / per2, w = (it - n1) - r * per2;
+      is_down = w >= gu_items;
+      u = is_down ? r : DL + r;
+      sub = is_down ? w - gu_items : w;
+    } else {
+      const int q = it - n1 - n2;
+      is_down = true;
+      u = U - DL + q / d_items;
+      sub = q % d_items;
     }
-    for (;;) {
-      int it = 0;
-      if (lane == 0) it = atomicAdd(&s_int[2], 1);
-      it = __shfl_sync(0xffffffffu, it, 0);
-      if (it >= total) break;
-      const int u = it / gu_items, g = it % gu_items;
+    if (!is_down) {
+      const int g = sub;
       const int slot = u % pl.ns_gu, use = u / pl.ns_gu;
       if (use > 0 && lane == 0) smem_count_wait(done_gu + slot, (unsigned)(use * gu_items), p);
       __syncwarp();
@@ -1194,16 +1219,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
         if ((int)done == gu_items) grid_arrive(gu_counter(fw, u));
       }
       __syncwarp();
-    }
-  }
-  {
-    const int total = U * d_items;
-    for (;;) {
-      int it = 0;
-      if (lane == 0) it = atomicAdd(&s_int[3], 1);
-      it = __shfl_sync(0xffffffffu, it, 0);
-      if (it >= total) break;
-      const int u = it / d_items, gd = it % d_items;
+    } else {
+      const int gd = sub;
       const int slot = u % pl.ns_d, use = u / pl.ns_d;
       const int pb = s_poff[u], pe = s_poff[u + 1];
       __half2* hbuf = reinterpret_cast<__half2*>(hstage + (size_t)slot * pl.hslot);

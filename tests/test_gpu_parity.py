@@ -77,6 +77,18 @@ def test_zipf_sweep_sampled(M):
     compare(L, split, L.oracle(tokens=sample), tokens=sample)
 
 
+@pytest.mark.parametrize("M", [16, 32])
+def test_shared_experts_many_pairs(M):
+    """Every token routes to the same 8 experts, so each expert has M pairs:
+    the tensor-core gate/up path runs two to four 8-pair column tiles, and
+    the down path reads h of more pairs than it stages."""
+    L = Layer(2560, 768, 256, 8, M, seed=12, mode="shared")
+    got = L.run(L.make_ctx(0, max_tokens=32))
+    assert len(set(got["ids"].ravel().tolist())) == 8
+    sample = sorted({0, M // 3, M - 1})
+    compare(L, got, L.oracle(tokens=sample), tokens=sample)
+
+
 @pytest.mark.parametrize("M,mode", [(1, "gap"), (2, "zipf"), (4, "gap"), (3, "shared")])
 def test_deep_ring_reuse(M, mode):
     """A context sized for 32 tokens leaves 4 ring slots, so every slot is
