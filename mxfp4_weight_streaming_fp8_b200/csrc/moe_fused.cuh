@@ -53,7 +53,7 @@ constexpr int kFusedThreads = 512;
 constexpr int kFusedWarps = kFusedThreads / 32;
 constexpr int kConsumers = kFusedWarps - 1;  // warp 0 produces
 constexpr int kGuRowsPerItem = 2;           // intermediate rows per gate/up item
-constexpr int kDownRowsPerItem = 6;         // output rows per down item
+constexpr int kDownRowsPerItem = 9;         // output rows per down item (two items per expert at 17-18 rows per CTA)
 constexpr int kHPairs = 4;                  // (token, slot) pairs of one expert whose h is staged in smem
 constexpr int kMaxRowsPerCta = 8;           // router rows a CTA may own (E <= 8 * G)
 constexpr int kMaxSlots = 64;
