@@ -57,6 +57,8 @@ def lib():
                                         [_u8p, _f32p, _f64p, _i32p, _f64p, _f64p, _u16p])
         L.oracle_moe_dense.argtypes = [ctypes.c_int] * 5 + [_u16p, _f32p] + [_u8pp] * 4 + [_f64p]
         L.oracle_rmsnorm.argtypes = [ctypes.c_int, ctypes.c_int, _u16p, ctypes.c_double, _u16p]
+        L.oracle_lm_quantize.argtypes = [ctypes.c_int, ctypes.c_int, _u16p, _u8p, _f32p]
+        L.oracle_lm_head.argtypes = [ctypes.c_int] * 3 + [_u8p, _f32p, _u16p, _f64p]
         _lib = L
     return _lib
 
@@ -202,4 +204,26 @@ def rmsnorm(y_bits, eps=1e-6):
     M, H = y.shape
     out = np.zeros((M, H), np.uint16)
     _check(lib().oracle_rmsnorm(M, H, _p(y, _u16p), float(eps), _p(out, _u16p)), "rmsnorm")
+    return out
+
+
+def lm_quantize(w_bits: np.ndarray):
+    """FP8 LM head weights: uint16 bf16 [V,H] -> (codes uint8 [V,H], scales float32 [V])."""
+    w = np.ascontiguousarray(w_bits, dtype=np.uint16)
+    V, H = w.shape
+    codes = np.zeros((V, H), np.uint8)
+    scales = np.zeros(V, np.float32)
+    _check(lib().oracle_lm_quantize(V, H, _p(w, _u16p), _p(codes, _u8p), _p(scales, _f32p)), "lm_quantize")
+    return codes, scales
+
+
+def lm_head(codes: np.ndarray, scales: np.ndarray, x_bits: np.ndarray) -> np.ndarray:
+    """fp64 logits [M,V] of the FP8 LM head for bf16 activations x [M,H]."""
+    c = np.ascontiguousarray(codes, dtype=np.uint8)
+    s = np.ascontiguousarray(scales, dtype=np.float32)
+    x = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    V, H = c.shape
+    M = x.shape[0]
+    out = np.zeros((M, V), np.float64)
+    _check(lib().oracle_lm_head(V, H, M, _p(c, _u8p), _p(s, _f32p), _p(x, _u16p), _p(out, _f64p)), "lm_head")
     return out

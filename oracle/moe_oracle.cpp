@@ -356,4 +356,26 @@ int oracle_rmsnorm(int M, int H, const uint16_t* y, double eps, uint16_t* out) {
   return 0;
 }
 
+// FP8 LM head: per-row quantisation is the A1 rule applied to each row of
+// the output matrix (one fp32 scale per row, the reading stated in
+// moe_oracle.h).
+int oracle_lm_quantize(int V, int H, const uint16_t* w, uint8_t* codes, float* scales) {
+  if (V < 0 || H <= 0 || !w || !codes || !scales) return -1;
+  return oracle_quantize(V, H, w, codes, scales);
+}
+
+// logits[m][v] = s_v * sum_h e4m3(code[v][h]) * x[m][h], fp64.
+int oracle_lm_head(int V, int H, int M, const uint8_t* codes, const float* scales, const uint16_t* x,
+                   double* logits) {
+  if (V < 0 || H <= 0 || M < 0 || !codes || !scales || !x || !logits) return -1;
+  for (int m = 0; m < M; ++m)
+    for (int v = 0; v < V; ++v) {
+      double acc = 0.0;
+      for (int h = 0; h < H; ++h)
+        acc += oracle_e4m3_value(codes[(size_t)v * H + h]) * oracle_bf16_value(x[(size_t)m * H + h]);
+      logits[(size_t)m * V + v] = acc * (double)scales[v];
+    }
+  return 0;
+}
+
 }  // extern "C"

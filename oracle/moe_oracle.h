@@ -99,6 +99,21 @@ int oracle_moe_dense(int H, int I, int E, int k, int M,
  * out = bf16(y / sqrt(mean(y^2) + eps)), per token, fp64. */
 int oracle_rmsnorm(int M, int H, const uint16_t* y, double eps, uint16_t* out);
 
+/* FP8 LM head ("NVIDIA Shows 3 Ways to Speed Up MoE Inference on DGX Spark",
+ * MarkTechPost, item 2 "Online FP8 LM head": the 157,184 x 2,560 BF16 output
+ * matrix is quantised to FP8 once at load, halving the bytes each token
+ * reads). The pages do not give the scale granularity; the reading here is
+ * one fp32 scale per output row, set by the same rule as the activation
+ * quantiser A1 applied to each row (amax, fp32 448/amax, E4M3
+ * round-to-nearest-even with saturation, scale amax/448; an all-zero row
+ * gives zero codes and scale 1). w [V][H] bf16 bits -> codes [V][H], scales
+ * [V]. */
+int oracle_lm_quantize(int V, int H, const uint16_t* w, uint8_t* codes, float* scales);
+/* logits[m][v] = scales[v] * sum_h e4m3(codes[v][h]) * bf16(x[m][h]) in fp64
+ * (weights FP8, activations kept in BF16). x [M][H], logits [M][V]. */
+int oracle_lm_head(int V, int H, int M, const uint8_t* codes, const float* scales, const uint16_t* x,
+                   double* logits);
+
 #ifdef __cplusplus
 }
 #endif

@@ -350,3 +350,73 @@ def test_rmsnorm_matches_torch_and_closed_form(oracle_mod):
     assert torch.all((gv - rv).abs() <= rv.abs() * 2 ** -8)
     const = np.full((1, 64), 0x4040, np.uint16)  # 3.0 everywhere -> 3/sqrt(9+eps) ~ 1
     assert np.all(oracle_mod.rmsnorm(const, 1e-6) == 0x3F80)
+
+
+# ---------------------------------------------------------------- FP8 LM head
+def _f8_codes(v32: torch.Tensor) -> np.ndarray:
+    """torch's own float32 -> float8_e4m3fn conversion (round to nearest even)."""
+    return v32.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def test_lm_quantize_hand_row(oracle_mod):
+    # row [1, 2, 3, 4]: amax 4, inv = 448/4 = 112 -> 112, 224, 336, 448.
+    # OFP8 E4M3: 112 = 1.75*2^6 -> 0x6E; 224 = 1.75*2^7 -> 0x76; 336 = 1.3125*2^8
+    # lies halfway between 1.25 and 1.375 and rounds to the even 1.25 -> 0x7A;
+    # 448 = 1.75*2^8 -> 0x7E. Scale fl32(4/448).
+    w = bf16_bits(torch.tensor([[1.0, 2.0, 3.0, 4.0], [0.0, 0.0, 0.0, 0.0]], dtype=torch.bfloat16))
+    codes, scales = oracle_mod.lm_quantize(w)
+    assert codes[0].tolist() == [0x6E, 0x76, 0x7A, 0x7E]
+    assert codes[1].tolist() == [0, 0, 0, 0] and scales[1] == 1.0
+    assert scales[0] == np.float32(4.0) / np.float32(448.0)
+    # x = [1, -1, 0.5, 2]: 112 - 224 + 0.5*320 + 2*448 = 944 (in units of the scale)
+    x = bf16_bits(torch.tensor([[1.0, -1.0, 0.5, 2.0]], dtype=torch.bfloat16))
+    lg = oracle_mod.lm_head(codes, scales, x)
+    assert lg[0, 0] == 944.0 * float(scales[0]) and lg[0, 1] == 0.0
+
+
+def test_lm_quantize_matches_torch_float8(oracle_mod):
+    g = torch.Generator().manual_seed(5)
+    w = torch.randn(37, 96, generator=g) * torch.logspace(-3, 3, 37).unsqueeze(1)
+    w[3] = 0.0
+    w[7] = 0.0
+    w[7, 11] = -0.75
+    wb = w.to(torch.bfloat16)
+    codes, scales = oracle_mod.lm_quantize(bf16_bits(wb))
+    w32 = wb.float()
+    amax = w32.abs().amax(dim=1)
+    for v in range(w.shape[0]):
+        if amax[v] == 0:
+            assert np.all(codes[v] == 0) and scales[v] == 1.0
+            continue
+        inv = torch.tensor(448.0, dtype=torch.float32) / amax[v]
+        assert np.array_equal(codes[v], _f8_codes(w32[v] * inv)), v
+        assert scales[v] == (amax[v] / torch.tensor(448.0)).item()
+
+
+def test_lm_head_one_hot_reads_a_column(oracle_mod):
+    rng = np.random.default_rng(6)
+    codes = rng.integers(0, 256, (23, 64)).astype(np.uint8)
+    codes[(codes & 0x7F) == 0x7F] = 0x01  # no NaN codes
+    scales = (2.0 ** rng.integers(-8, 8, 23)).astype(np.float32) * np.float32(1.5)
+    dec = torch.from_numpy(codes.copy()).view(torch.float8_e4m3fn).float().numpy().astype(np.float64)
+    for h in (0, 17, 63):
+        x = np.zeros((1, 64), np.float32)
+        x[0, h] = 1.0
+        lg = oracle_mod.lm_head(codes, scales, bf16_bits(torch.from_numpy(x).to(torch.bfloat16)))
+        assert np.array_equal(lg[0], dec[:, h] * scales.astype(np.float64)), h
+
+
+def test_lm_head_linear_and_homogeneous(oracle_mod):
+    rng = np.random.default_rng(7)
+    codes = rng.integers(0, 0x7E, (19, 128)).astype(np.uint8)
+    scales = rng.uniform(0.5, 2.0, 19).astype(np.float32)
+    x = torch.randn(2, 128, generator=torch.Generator().manual_seed(8)).to(torch.bfloat16)
+    a, b = x.clone(), x.clone()
+    a[:, 64:] = 0
+    b[:, :64] = 0
+    la = oracle_mod.lm_head(codes, scales, bf16_bits(a))
+    lb = oracle_mod.lm_head(codes, scales, bf16_bits(b))
+    lx = oracle_mod.lm_head(codes, scales, bf16_bits(x))
+    assert np.allclose(la + lb, lx, rtol=1e-12, atol=1e-9)
+    l2 = oracle_mod.lm_head(codes, scales, bf16_bits(x * 2))
+    assert np.array_equal(l2, 2 * lx)
