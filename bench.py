@@ -60,12 +60,18 @@ def load_peaks():
         return 6650.0, "fallback"
 
 
-def kernel_source_hash():
+KERNEL_SOURCES = {
+    # the device code each kernel is compiled from
+    "k_fused": ("moe_fused.cuh", "moe_device.cuh"),
+    "k_lm_head": ("moe_lmhead.cu", "moe_device.cuh"),
+}
+
+
+def kernel_source_hash(kernel: str = "k_fused"):
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "mxfp4_weight_streaming_fp8_b200", "csrc")
-    for fn in sorted(os.listdir(csrc)):
-        if fn.endswith((".cu", ".cuh", ".h")):
-            h.update(open(os.path.join(csrc, fn), "rb").read())
+    for fn in KERNEL_SOURCES.get(kernel, ()):
+        h.update(open(os.path.join(csrc, fn), "rb").read())
     return h.hexdigest()[:16]
 
 
@@ -77,7 +83,7 @@ def recorded_traffic(kernel: str, workload: str):
         rec = json.load(open(path))[kernel][workload]
     except Exception:
         return None
-    if rec.get("source_hash") != kernel_source_hash():
+    if rec.get("source_hash") != kernel_source_hash(kernel):
         return None
     return rec.get("bytes_per_launch")
 
@@ -419,6 +425,112 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+LM_V, LM_H = 157184, 2560
+LM_METRIC = "FP8 LM head GEMV (157,184 x 2,560) µs/call, tokens/s; HBM GB/s as % of B200 peak"
+
+
+def run_lm_head(args):
+    """The FP8 LM head on one GPU: each step is one call for M tokens; the
+    402 MB FP8 matrix is far larger than L2, so every call streams it."""
+    import numpy as np
+    import torch
+    from mxfp4_weight_streaming_fp8_b200 import moe
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    M = args.tokens
+    g = torch.Generator(device=device).manual_seed(SEED)
+    lm = moe.LMHead(LM_V, LM_H, max_tokens=M)
+    w = (torch.randn(LM_V, LM_H, generator=g, device=device) * 0.02).to(torch.bfloat16)
+    lm.load(w)
+    w_cpu_rows = w[:65536].cpu()  # CPU baseline sample (~1-2 s of oracle work)
+    del w
+    x = torch.randn(M, LM_H, generator=g, device=device).to(torch.bfloat16)
+    logits = torch.empty((M, LM_V), dtype=torch.float32, device=device)
+    calls = 8  # calls per graph replay
+    stream = torch.cuda.Stream(device)
+    stream.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(stream):
+        assert lm.head_raw(x, M, logits, stream=stream) == moe.MOE_OK
+    torch.cuda.current_stream().wait_stream(stream)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for _ in range(calls):
+            assert lm.head_raw(x, M, logits, stream=stream) == moe.MOE_OK
+    cur = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(device.index) as clk:
+        ev0.record(cur)
+        for _ in range(args.steps):
+            graph.replay()
+        ev1.record(cur)
+        ev1.synchronize()
+    ms = ev0.elapsed_time(ev1)
+    st = lm.sync_status()
+    if st != moe.MOE_OK:
+        raise RuntimeError(f"kernel status {moe.status_string(st)}")
+    n_calls = args.steps * calls
+    us_call = ms * 1e3 / n_calls
+    alg = LM_V * LM_H + 4 * LM_V + 2 * M * LM_H + 4 * M * LM_V
+    peak, peak_kind = load_peaks()
+    achieved = alg / (us_call * 1e-6) / 1e9
+    workload = f"lm_head_fp8_V{LM_V}_H{LM_H}_M{M}"
+    # end to end: pinned x in, one call, logits out
+    xh = x.cpu().pin_memory()
+    lh = torch.empty((M, LM_V), dtype=torch.float32).pin_memory()
+    xd = torch.empty_like(x)
+    for _ in range(args.warmup):
+        xd.copy_(xh, non_blocking=True)
+        lm.head_raw(xd, M, logits, stream=cur)
+        lh.copy_(logits, non_blocking=True)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(cur)
+    for _ in range(args.steps):
+        xd.copy_(xh, non_blocking=True)
+        lm.head_raw(xd, M, logits, stream=cur)
+        lh.copy_(logits, non_blocking=True)
+    e1.record(cur)
+    e1.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    line = {
+        "metric": LM_METRIC, "value": round(M * n_calls / (ms / 1e3), 1), "unit": "tokens/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "fp8e4m3 x bf16 (f16 MMA, fp32 accumulate)", "data": "synthetic (seeded N(0,0.02) bf16 weights)",
+        "config": {"workload": workload, "vocab": LM_V, "hidden": LM_H, "tokens": M,
+                   "l2": "inputs larger than L2: every call streams the 402 MB FP8 matrix",
+                   "step": f"{calls} calls in one CUDA graph"},
+        "us_per_call": round(us_call, 3),
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
+                     "traffic": recorded_traffic("k_lm_head", workload), "kernel": "k_lm_head",
+                     "algorithmic_bytes_per_launch": alg},
+        "gpu_launches": n_calls, "clocks": clk.summary(),
+        "e2e": {"value": round(M * args.steps / (e2e_ms / 1e3), 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": M * LM_H * 2, "d2h_bytes_per_step": M * LM_V * 4,
+                "how": "per step: H2D x, one moe_lm_head call, D2H logits"},
+    }
+    if not args.no_cpu:
+        import oracle
+        rows = w_cpu_rows.shape[0]
+        codes, scales = oracle.lm_quantize(w_cpu_rows.view(torch.int16).numpy().view(np.uint16))
+        xb = x.cpu().view(torch.int16).numpy().view(np.uint16)
+        t0 = time.perf_counter()
+        oracle.lm_head(codes, scales, xb)
+        dt = time.perf_counter() - t0
+        per_call = dt * LM_V / rows
+        line["cpu_baseline"] = {"value": round(M / per_call, 4), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                                "sample": f"{rows} of {LM_V} rows for M={M} ({dt:.2f} s), scaled to the full "
+                                          "matrix; single-threaded fp64 C++ oracle"}
+    print(json.dumps(line), flush=True)
+    del graph
+    lm.close()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -434,11 +546,15 @@ def main():
     ap.add_argument("--variant", choices=["fused", "split"], default="fused")
     ap.add_argument("--stack", action="store_true",
                     help="chain the pool as a stack: layer l+1 takes RMSNorm(y_l)")
+    ap.add_argument("--op", choices=["moe", "lm_head"], default="moe",
+                    help="moe: the MoE layer step (default); lm_head: the FP8 LM head GEMV")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
     if args.impl == "reference":
         run_reference(args)
+    elif args.op == "lm_head":
+        run_lm_head(args)
     else:
         run_ours(args)
 

@@ -194,6 +194,55 @@ moe_status moe_decode_static(const moe_config* cfg, const float* router_w,
 /* Static string naming a status code. */
 const char* moe_status_string(moe_status s);
 
+/* ------------------------------------------------------------ FP8 LM head
+ * "NVIDIA Shows 3 Ways to Speed Up MoE Inference on DGX Spark"
+ * (MarkTechPost), item 2 "Online FP8 LM head": the 157,184 x 2,560 output
+ * matrix, stored in BF16, is quantised to FP8 once when it is loaded, which
+ * halves the bytes every generated token reads. The pages do not give the
+ * scale granularity; here each output row v gets one fp32 scale s_v and E4M3
+ * codes by the activation quantiser's rule applied to the row (amax over the
+ * row, fp32 448/amax, round to nearest even with saturation, s_v = amax/448;
+ * an all-zero row gets zero codes and s_v = 1). A call computes
+ *     logits[m][v] = s_v * sum_h e4m3(W[v][h]) * x[m][h]
+ * for BF16 activations x, in fp32 (weights FP8, activations BF16).
+ * The context owns the FP8 copy (V*H + 4*V bytes); it serves one matrix. */
+typedef struct moe_lm moe_lm; /* opaque */
+
+/* vocab >= 1; hidden a multiple of 64 in [64, 8192]; 1 <= max_tokens <= 16;
+ * device an sm_100 GPU. Allocates the FP8 copy and a status word.
+ * INVALID_ARG on bad arguments, UNSUPPORTED if the kernel does not fit the
+ * device, OOM if an allocation fails. */
+moe_status moe_lm_create(int32_t vocab, int32_t hidden, int32_t max_tokens, int32_t device, moe_lm** out);
+
+/* Quantise the BF16 matrix w_bf16 [vocab][hidden] (device pointer, 16-byte
+ * aligned, row-major) into the context. Synchronous; the caller may free w
+ * afterwards. INVALID_ARG on a NULL or misaligned pointer, CUDA on a launch
+ * failure. */
+moe_status moe_lm_load(moe_lm* lm, const void* w_bf16);
+
+/* logits [M][vocab] fp32 (device, 4-byte aligned) for x_bf16 [M][hidden]
+ * (device, 16-byte aligned), 0 <= M <= max_tokens; M = 0 does nothing.
+ * Asynchronous on `stream` (NULL: the legacy default stream); allocates
+ * nothing. INVALID_ARG on bad sizes, misalignment or overlapping x and
+ * logits; NOT_LOADED before moe_lm_load. A device-side wait that runs out of
+ * budget sets the status word, read by moe_lm_sync_status. */
+moe_status moe_lm_head(moe_lm* lm, const void* x_bf16, int32_t M, float* logits, void* stream);
+
+/* Synchronise `stream` and report the status word: OK, or TIMEOUT (the word
+ * is cleared). */
+moe_status moe_lm_sync_status(moe_lm* lm, void* stream);
+
+/* Copy the context's FP8 weights into caller buffers (device pointers):
+ * codes [vocab][hidden] E4M3 and scales [vocab] fp32, asynchronously on
+ * `stream`. NOT_LOADED before moe_lm_load; CUDA if a copy fails. */
+moe_status moe_lm_read_weights(const moe_lm* lm, uint8_t* codes, float* scales, void* stream);
+
+/* JSON description of the launch configuration (kernel, grid, shared memory,
+ * ring slots) into buf; INVALID_ARG if it does not fit in len. */
+moe_status moe_lm_query(const moe_lm* lm, char* buf, size_t len);
+
+void moe_lm_destroy(moe_lm* lm);
+
 #ifdef __cplusplus
 }
 #endif

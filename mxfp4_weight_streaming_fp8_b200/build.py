@@ -12,7 +12,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB_PATH = os.path.join(HERE, "libmoe.so")
-SOURCES = [os.path.join(CSRC, "moe_api.cu"), os.path.join(CSRC, "moe_static.cu")]
+SOURCES = [os.path.join(CSRC, f) for f in ("moe_api.cu", "moe_static.cu", "moe_lmhead.cu")]
 DEPS = SOURCES + [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cuh", ".h", ".cu"))] + [
     os.path.join(ROOT, "include", "moe.h")]
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",

@@ -11,33 +11,20 @@
 
 #include "../../include/moe.h"
 #include "moe_device.cuh"
+#include "moe_host.h"
 #include "moe_fused.cuh"
 #include "moe_split.cuh"
+
+using moe_host::aligned16;
+using moe_host::align_up;
+using moe_host::DeviceGuard;
+using moe_host::kDefaultSpinLimit;
 
 namespace {
 
 enum Variant { kFused = 0, kSplit = 1 };
 
-// ~0.5 s at ~2 GHz: far longer than any legitimate wait, short enough that a
-// stuck wait returns an error instead of hanging the GPU.
-constexpr long long kDefaultSpinLimit = 1000000000LL;
 
-struct DeviceGuard {
-  int prev = -1;
-  bool ok = true;
-  explicit DeviceGuard(int dev) {
-    if (cudaGetDevice(&prev) != cudaSuccess) { ok = false; return; }
-    if (prev != dev && cudaSetDevice(dev) != cudaSuccess) ok = false;
-  }
-  ~DeviceGuard() {
-    int cur;
-    if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
-  }
-};
-
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
-size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 moe_status validate_config(const moe_config& c) {
   if (c.hidden < 32 || c.hidden > 8192 || c.hidden % 32) return MOE_ERR_INVALID_ARG;

@@ -69,6 +69,21 @@ def lib() -> ctypes.CDLL:
         L.moe_decode_static.restype = ctypes.c_int
         L.moe_debug_set_wait.argtypes = [_vp, ctypes.c_longlong, ctypes.c_int]
         L.moe_debug_set_wait.restype = ctypes.c_int
+        L.moe_lm_create.argtypes = [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                    ctypes.POINTER(_vp)]
+        L.moe_lm_create.restype = ctypes.c_int
+        L.moe_lm_load.argtypes = [_vp, _vp]
+        L.moe_lm_load.restype = ctypes.c_int
+        L.moe_lm_head.argtypes = [_vp, _vp, ctypes.c_int32, _vp, _vp]
+        L.moe_lm_head.restype = ctypes.c_int
+        L.moe_lm_sync_status.argtypes = [_vp, _vp]
+        L.moe_lm_sync_status.restype = ctypes.c_int
+        L.moe_lm_read_weights.argtypes = [_vp, _vp, _vp, _vp]
+        L.moe_lm_read_weights.restype = ctypes.c_int
+        L.moe_lm_query.argtypes = [_vp, ctypes.c_char_p, ctypes.c_size_t]
+        L.moe_lm_query.restype = ctypes.c_int
+        L.moe_lm_destroy.argtypes = [_vp]
+        L.moe_lm_destroy.restype = None
         _lib = L
     return _lib
 
@@ -175,6 +190,69 @@ class MoELayer:
             lib().moe_destroy(self._ctx)
             self._ctx = _vp()
         self._weights = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+class LMHead:
+    """FP8 LM head context: moe_lm_create / moe_lm_load / moe_lm_head."""
+
+    def __init__(self, vocab: int, hidden: int, max_tokens: int = 1, device: int = 0):
+        self.vocab, self.hidden, self.max_tokens, self.device = vocab, hidden, max_tokens, device
+        self._lm = _vp()
+        st = lib().moe_lm_create(vocab, hidden, max_tokens, device, ctypes.byref(self._lm))
+        if st != MOE_OK:
+            raise MoEError(st, "moe_lm_create")
+
+    def load(self, w_bf16):
+        """Quantise the bf16 [vocab, hidden] device matrix into the context."""
+        st = lib().moe_lm_load(self._lm, _ptr(w_bf16))
+        if st != MOE_OK:
+            raise MoEError(st, "moe_lm_load")
+
+    def weights(self, stream=None):
+        """(codes uint8 [vocab, hidden], scales float32 [vocab]) as device tensors (copies)."""
+        import torch
+        dev = f"cuda:{self.device}"
+        codes = torch.empty((self.vocab, self.hidden), dtype=torch.uint8, device=dev)
+        scales = torch.empty(self.vocab, dtype=torch.float32, device=dev)
+        st = lib().moe_lm_read_weights(self._lm, _ptr(codes), _ptr(scales), _stream_handle(stream))
+        if st != MOE_OK:
+            raise MoEError(st, "moe_lm_read_weights")
+        return codes, scales
+
+    def head_raw(self, x, M: int, logits, stream=None) -> int:
+        return lib().moe_lm_head(self._lm, _ptr(x), int(M), _ptr(logits), _stream_handle(stream))
+
+    def __call__(self, x, logits=None, stream=None):
+        """x: bf16 [M, hidden] on the device -> fp32 logits [M, vocab]."""
+        import torch
+        M = x.shape[0]
+        if logits is None:
+            logits = torch.empty((M, self.vocab), dtype=torch.float32, device=x.device)
+        st = self.head_raw(x, M, logits, stream)
+        if st != MOE_OK:
+            raise MoEError(st, "moe_lm_head")
+        return logits
+
+    def sync_status(self, stream=None) -> int:
+        return lib().moe_lm_sync_status(self._lm, _stream_handle(stream))
+
+    def query(self) -> dict:
+        buf = ctypes.create_string_buffer(1024)
+        st = lib().moe_lm_query(self._lm, buf, len(buf))
+        if st != MOE_OK:
+            raise MoEError(st, "moe_lm_query")
+        return json.loads(buf.value.decode())
+
+    def close(self):
+        if self._lm:
+            lib().moe_lm_destroy(self._lm)
+            self._lm = _vp()
 
     def __del__(self):
         try:

@@ -93,3 +93,20 @@ def test_persistent_kernel_plan_fits(L, shape):
 def test_plan_rejects_what_does_not_fit(L):
     st, pl = moe.plan_query(8192, 4096, 1024, 32, 32)
     assert st == 2 and not pl["ok"]
+
+
+def test_lm_head_entry_points_reject_bad_arguments_without_a_gpu(L):
+    """The LM head entry points validate arguments before touching CUDA."""
+    import ctypes
+    out = ctypes.c_void_p()
+    assert L.moe_lm_create(0, 256, 1, 0, ctypes.byref(out)) == 1       # vocab < 1
+    assert L.moe_lm_create(1000, 100, 1, 0, ctypes.byref(out)) == 1    # hidden % 64
+    assert L.moe_lm_create(1000, 256, 17, 0, ctypes.byref(out)) == 1   # max_tokens > 16
+    assert L.moe_lm_create(1000, 256, 1, 0, None) == 1
+    assert L.moe_lm_load(None, None) == 1
+    assert L.moe_lm_head(None, None, 1, None, None) == 1
+    assert L.moe_lm_sync_status(None, None) == 1
+    assert L.moe_lm_read_weights(None, None, None, None) == 1
+    buf = ctypes.create_string_buffer(64)
+    assert L.moe_lm_query(None, buf, 64) == 1
+    L.moe_lm_destroy(None)
