@@ -295,6 +295,30 @@ int oracle_moe_decode(int H, int I, int E, int k, int M,
   return 0;
 }
 
+// The routed step, then the shared expert's output added with weight 1.
+int oracle_moe_decode_shared(int H, int I, int E, int k, int M,
+                             const uint16_t* x, const float* router_w,
+                             const uint8_t* const* w13_codes, const uint8_t* const* w13_scales,
+                             const uint8_t* const* w2_codes, const uint8_t* const* w2_scales,
+                             const uint8_t* sh_w13_codes, const uint8_t* sh_w13_scales,
+                             const uint8_t* sh_w2_codes, const uint8_t* sh_w2_scales,
+                             int32_t* ids, double* weights, double* y64) {
+  if (!sh_w13_codes || !sh_w13_scales || !sh_w2_codes || !sh_w2_scales || M < 0 || H <= 0) return -1;
+  std::vector<uint8_t> qv((size_t)M * H);
+  std::vector<float> sv(M);
+  int rc = oracle_moe_decode(H, I, E, k, M, x, router_w, w13_codes, w13_scales, w2_codes, w2_scales,
+                             qv.data(), sv.data(), nullptr, ids, weights, y64, nullptr);
+  if (rc) return rc;
+  std::vector<double> d(H);
+  for (int m = 0; m < M; ++m) {
+    rc = oracle_expert(H, I, qv.data() + (size_t)m * H, sv[m], sh_w13_codes, sh_w13_scales, sh_w2_codes,
+                       sh_w2_scales, nullptr, d.data());
+    if (rc) return rc;
+    for (int r = 0; r < H; ++r) y64[(size_t)m * H + r] += d[r];
+  }
+  return 0;
+}
+
 // Brute force over all E experts: expert e is kept for token m when fewer
 // than k experts rank above it (higher logit, or equal logit and lower index);
 // the kept experts' weights are exp(l_e - max) renormalised over the kept set.

@@ -302,6 +302,56 @@ def test_invariant_zero_codes_give_zero(oracle_mod):
         assert not out["y64"].any()
 
 
+def _shared_expert(seed=7, H=256, I=64):
+    return [np.asarray(a) for a in synth.expert_np(seed, 0, 0, H, I)]
+
+
+@pytest.mark.parametrize("M,k,mode", [(1, 2, "natural"), (3, 4, "gap")])
+def test_shared_expert_zero_w2_is_routed_only(oracle_mod, M, k, mode):
+    # A shared expert whose down weights are all zero adds nothing: the
+    # result is the routed-only step bit for bit, ids and weights included.
+    H, I, E = 256, 64, 16
+    x, wr, per = _tiny_layer(M=M, k=k, mode=mode)
+    sh = _shared_expert()
+    sh[2] = np.zeros_like(sh[2])
+    base = oracle_mod.moe_decode(x, wr, *per, H, I, E, k)
+    out = oracle_mod.moe_decode_shared(x, wr, *per, sh, H, I, E, k)
+    assert np.array_equal(out["ids"], base["ids"])
+    assert np.array_equal(out["weights"], base["weights"])
+    assert np.array_equal(out["y64"], base["y64"])
+
+
+def test_shared_expert_alone_is_one_expert_at_weight_one(oracle_mod):
+    # With every routed expert's down weights zero, the layer output is the
+    # shared expert applied to the quantised token, with weight exactly 1.
+    H, I, E, k, M = 256, 64, 16, 2, 3
+    x, wr, per = _tiny_layer(M=M, k=k, mode="gap")
+    z2 = [np.zeros_like(a) for a in per[2]]
+    sh = _shared_expert()
+    out = oracle_mod.moe_decode_shared(x, wr, per[0], per[1], z2, per[3], sh, H, I, E, k)
+    q, s = oracle_mod.quantize(x)
+    for m in range(M):
+        _, d = oracle_mod.expert(q[m], s[m], *sh, H, I)
+        assert np.array_equal(out["y64"][m], d)
+        assert np.any(d != 0)
+
+
+def test_shared_expert_is_additive_and_scales(oracle_mod):
+    # Raising every E8M0 down scale of the shared expert by one doubles its
+    # contribution exactly, and leaves the routed part untouched.
+    H, I, E, k, M = 256, 64, 16, 4, 2
+    x, wr, per = _tiny_layer(M=M, k=k, mode="gap")
+    sh = _shared_expert()
+    base = oracle_mod.moe_decode(x, wr, *per, H, I, E, k)["y64"]
+    one = oracle_mod.moe_decode_shared(x, wr, *per, sh, H, I, E, k)["y64"]
+    sh2 = list(sh)
+    sh2[3] = sh[3] + 1
+    two = oracle_mod.moe_decode_shared(x, wr, *per, sh2, H, I, E, k)["y64"]
+    scale = np.abs(one).max() + np.abs(base).max()
+    assert np.all(np.abs((two - base) - 2 * (one - base)) <= 1e-13 * scale)
+    assert np.any(one != base)
+
+
 def test_invariant_w2_scale_doubles_output(oracle_mod):
     H, I, E, k = 256, 64, 16, 2
     x, wr, per = _tiny_layer()
