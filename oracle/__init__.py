@@ -58,7 +58,7 @@ def lib():
         L.oracle_moe_dense.argtypes = [ctypes.c_int] * 5 + [_u16p, _f32p] + [_u8pp] * 4 + [_f64p]
         L.oracle_rmsnorm.argtypes = [ctypes.c_int, ctypes.c_int, _u16p, ctypes.c_double, _u16p]
         L.oracle_moe_decode_shared.argtypes = ([ctypes.c_int] * 5 + [_u16p, _f32p] + [_u8pp] * 4 + [_u8p] * 4 +
-                                               [_i32p, _f64p, _f64p])
+                                               [_u8p, _f32p, _f64p, _i32p, _f64p, _f64p])
         L.oracle_lm_quantize.argtypes = [ctypes.c_int, ctypes.c_int, _u16p, _u8p, _f32p]
         L.oracle_lm_head.argtypes = [ctypes.c_int] * 3 + [_u8p, _f32p, _u16p, _f64p]
         _lib = L
@@ -192,17 +192,19 @@ def moe_decode(x_bits, router_w, w13c, w13s, w2c, w2s, H, I, E, k):
 
 def moe_decode_shared(x_bits, router_w, w13c, w13s, w2c, w2s, shared, H, I, E, k):
     """A1-A8 plus one always-active shared expert; shared = (w13c, w13s, w2c,
-    w2s) arrays of one expert. Returns dict with ids, weights, y64."""
+    w2s) arrays of one expert. Returns dict with q, s, logits, ids, weights,
+    y64."""
     x = np.ascontiguousarray(x_bits, dtype=np.uint16)
     wr = np.ascontiguousarray(router_w, dtype=np.float32)
     M = x.shape[0]
     ptrs = [_expert_ptrs(t, E) for t in (w13c, w13s, w2c, w2s)]
     sh = [np.ascontiguousarray(a, dtype=np.uint8) for a in shared]
-    out = dict(ids=np.zeros((M, k), np.int32), weights=np.zeros((M, k), np.float64),
-               y64=np.zeros((M, H), np.float64))
+    out = dict(q=np.zeros((M, H), np.uint8), s=np.zeros(M, np.float32),
+               logits=np.zeros((M, E), np.float64), ids=np.zeros((M, k), np.int32),
+               weights=np.zeros((M, k), np.float64), y64=np.zeros((M, H), np.float64))
     _check(lib().oracle_moe_decode_shared(
         H, I, E, k, M, _p(x, _u16p), _p(wr, _f32p), *[p[0] for p in ptrs], *[_p(a, _u8p) for a in sh],
-        _p(out["ids"], _i32p), _p(out["weights"], _f64p), _p(out["y64"], _f64p)), "moe_decode_shared")
+        _p(out["q"], _u8p), _p(out["s"], _f32p), _p(out["logits"], _f64p), _p(out["ids"], _i32p), _p(out["weights"], _f64p), _p(out["y64"], _f64p)), "moe_decode_shared")
     return out
 
 

@@ -302,13 +302,16 @@ int oracle_moe_decode_shared(int H, int I, int E, int k, int M,
                              const uint8_t* const* w2_codes, const uint8_t* const* w2_scales,
                              const uint8_t* sh_w13_codes, const uint8_t* sh_w13_scales,
                              const uint8_t* sh_w2_codes, const uint8_t* sh_w2_scales,
-                             int32_t* ids, double* weights, double* y64) {
+                             uint8_t* q, float* s, double* logits, int32_t* ids, double* weights,
+                             double* y64) {
   if (!sh_w13_codes || !sh_w13_scales || !sh_w2_codes || !sh_w2_scales || M < 0 || H <= 0) return -1;
   std::vector<uint8_t> qv((size_t)M * H);
   std::vector<float> sv(M);
   int rc = oracle_moe_decode(H, I, E, k, M, x, router_w, w13_codes, w13_scales, w2_codes, w2_scales,
-                             qv.data(), sv.data(), nullptr, ids, weights, y64, nullptr);
+                             qv.data(), sv.data(), logits, ids, weights, y64, nullptr);
   if (rc) return rc;
+  if (q) std::copy(qv.begin(), qv.end(), q);
+  if (s) std::copy(sv.begin(), sv.end(), s);
   std::vector<double> d(H);
   for (int m = 0; m < M; ++m) {
     rc = oracle_expert(H, I, qv.data() + (size_t)m * H, sv[m], sh_w13_codes, sh_w13_scales, sh_w2_codes,

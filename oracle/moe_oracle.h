@@ -94,14 +94,16 @@ int oracle_moe_decode(int H, int I, int E, int k, int M,
  * and format and is always active with weight 1 (outside the router's
  * softmax); its output is added after the routed ones:
  *   y[m] = sum_j w[m][j] * expert_{ids[m][j]}(x_m) + expert_shared(x_m).
- * Outputs as oracle_moe_decode (ids/weights cover the routed experts). */
+ * Outputs as oracle_moe_decode (q, s, logits may be NULL; ids and weights
+ * cover the routed experts). */
 int oracle_moe_decode_shared(int H, int I, int E, int k, int M,
                              const uint16_t* x, const float* router_w,
                              const uint8_t* const* w13_codes, const uint8_t* const* w13_scales,
                              const uint8_t* const* w2_codes, const uint8_t* const* w2_scales,
                              const uint8_t* sh_w13_codes, const uint8_t* sh_w13_scales,
                              const uint8_t* sh_w2_codes, const uint8_t* sh_w2_scales,
-                             int32_t* ids, double* weights, double* y64);
+                             uint8_t* q, float* s, double* logits, int32_t* ids, double* weights,
+                             double* y64);
 /* Brute force: every expert for every token, masked by a rank-count top-k
  * and weighted by a softmax renormalised over the kept experts. */
 int oracle_moe_dense(int H, int I, int E, int k, int M,

@@ -316,7 +316,8 @@ def test_shared_expert_zero_w2_is_routed_only(oracle_mod, M, k, mode):
     sh[2] = np.zeros_like(sh[2])
     base = oracle_mod.moe_decode(x, wr, *per, H, I, E, k)
     out = oracle_mod.moe_decode_shared(x, wr, *per, sh, H, I, E, k)
-    assert np.array_equal(out["ids"], base["ids"])
+    for key in ("q", "s", "logits", "ids"):
+        assert np.array_equal(out[key], base[key])
     assert np.array_equal(out["weights"], base["weights"])
     assert np.array_equal(out["y64"], base["y64"])
 
