@@ -176,9 +176,10 @@ def sum_over_ranks(value: float, ws: int, device=None) -> float:
 
 
 # ------------------------------------------------------------------ workload
-def build_pool(device, M, mode, layers=POOL_LAYERS, seed=SEED, flags=0, stack=False):
+def build_pool(device, M, mode, layers=POOL_LAYERS, seed=SEED, flags=0, stack=False, shared=False):
     """One context per layer of the pool. With stack=True, layers after the
-    first normalise their input (RMSNorm) and take the previous output."""
+    first normalise their input (RMSNorm) and take the previous output. With
+    shared=True every layer has one more expert (index E), the shared one."""
     import torch
     from mxfp4_weight_streaming_fp8_b200 import moe, synth
     x = synth.gen_x(seed, M, H)
@@ -189,9 +190,10 @@ def build_pool(device, M, mode, layers=POOL_LAYERS, seed=SEED, flags=0, stack=Fa
         wr = synth.gen_router(seed, l, E, H)
         if not (stack and l > 0):
             wr = synth.force_router(x, wr, K, mode, seed=seed, layer=l)
-        ex = synth.layer_experts_torch(seed, l, E, H, I, device)
+        ex = synth.layer_experts_torch(seed, l, E + int(shared), H, I, device)
         wr_d = torch.from_numpy(wr).to(device)
         lflags = flags | (moe.MOE_FLAG_PRE_RMSNORM if (stack and l > 0) else 0)
+        lflags |= moe.MOE_FLAG_SHARED_EXPERT if shared else 0
         ctx = moe.MoELayer(H, I, E, K, M, flags=lflags, device=device.index)
         ctx.load_experts(wr_d, *ex, validate=False)
         ctxs.append(ctx)
@@ -213,7 +215,9 @@ def run_ours(args):
     M = args.tokens
     L = args.layers
     flags = moe.MOE_FLAG_SPLIT_KERNELS if args.variant == "split" else 0
-    x, ctxs, _weights = build_pool(device, M, args.routing, layers=L, flags=flags, stack=args.stack)
+    x, ctxs, _weights = build_pool(device, M, args.routing, layers=L, flags=flags, stack=args.stack,
+                                   shared=args.shared_expert)
+    n_shared = int(args.shared_expert)
     info = ctxs[0].query()
     x_d = x.to(device)
     ys = [torch.empty_like(x_d) for _ in range(L)]
@@ -276,18 +280,19 @@ def run_ours(args):
     U_mean = sum(Us) / len(Us)
     tokens_total = ws * M * layer_steps
     value = tokens_total / (ms / 1e3)
-    alg = algorithmic_bytes(M, U_mean)
-    exp_b = U_mean * expert_bytes()
+    alg = algorithmic_bytes(M, U_mean + n_shared)
+    exp_b = (U_mean + n_shared) * expert_bytes()
     peak, peak_kind = load_peaks()
     achieved = alg / (us_per_layer * 1e-6) / 1e9
     workload = (f"ling_stack{L}_rmsnorm_M{M}" if args.stack else f"ling_layer_M{M}_{args.routing}")
+    workload += "_shared1" if n_shared else ""
     traffic = recorded_traffic("k_fused", workload)
 
     # ---- end to end through the public API with host buffers
     e2e = run_e2e(args, ctxs, x, device, M, L, stack=args.stack)
 
     # ---- CPU oracle baseline (rank 0 only)
-    cpu = run_cpu_baseline(args, M) if rank == 0 and not args.no_cpu else None
+    cpu = run_cpu_baseline(args, M, shared=args.shared_expert) if rank == 0 and not args.no_cpu else None
 
     launches = layer_steps * (3 if info["variant"] == "split" else 1)
     line = {
@@ -296,7 +301,8 @@ def run_ours(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp8e4m3 x mxfp4 (f16/fp32 accumulate)",
         "data": "synthetic (seeded SplitMix64; random MXFP4 weights, N(0,1) bf16 activations)",
         "config": {"workload": workload, "hidden": H, "inter": I, "num_experts": E, "top_k": K, "tokens": M,
-                   "routing": args.routing, "layers_in_pool": L, "pool_weight_bytes": L * E * expert_bytes(),
+                   "routing": args.routing, "shared_experts": n_shared, "layers_in_pool": L,
+                   "pool_weight_bytes": L * (E + n_shared) * expert_bytes(),
                    "l2": "inputs larger than L2: each layer-step reads a different layer of the pool",
                    "step": (f"{L}-layer stack (RMSNorm between layers) in one CUDA graph" if args.stack
                             else f"{L} layer-steps in one CUDA graph"), "parallelism": f"replicas x{ws}",
@@ -362,8 +368,9 @@ def run_e2e(args, ctxs, x_cpu, device, M, L, stack=False):
             "how": f"per step: H2D x, {L} moe_decode calls (direct launches), D2H y"}
 
 
-def cpu_sample_steps(M, n_layers, seed=SEED):
-    """Inputs of a bounded oracle sample: n_layers layer-steps of the pool."""
+def cpu_sample_steps(M, n_layers, seed=SEED, shared=False):
+    """Inputs of a bounded oracle sample: n_layers layer-steps of the pool
+    (with the shared expert's arrays when shared=True)."""
     import numpy as np
     import oracle
     from mxfp4_weight_streaming_fp8_b200 import synth
@@ -378,17 +385,24 @@ def cpu_sample_steps(M, n_layers, seed=SEED):
             parts = synth.expert_np(seed, l, e, H, I)
             for t in range(4):
                 per[t][e] = parts[t]
-        steps.append((wr, per))
+        steps.append((wr, per, synth.expert_np(seed, l, E, H, I) if shared else None))
     return xb, steps
 
 
-def run_cpu_baseline(args, M, n_layers=None):
+def oracle_step(xb, step):
     import oracle
+    wr, per, sh = step
+    if sh is None:
+        return oracle.moe_decode(xb, wr, *per, H, I, E, K)
+    return oracle.moe_decode_shared(xb, wr, *per, sh, H, I, E, K)
+
+
+def run_cpu_baseline(args, M, n_layers=None, shared=False):
     n_layers = n_layers or args.cpu_layers
-    xb, steps = cpu_sample_steps(M, n_layers)
+    xb, steps = cpu_sample_steps(M, n_layers, shared=shared)
     t0 = time.perf_counter()
-    for wr, per in steps:
-        oracle.moe_decode(xb, wr, *per, H, I, E, K)
+    for st in steps:
+        oracle_step(xb, st)
     dt = time.perf_counter() - t0
     return {"value": round(M * n_layers / dt, 3), "unit": "tokens/s", "cores": 1, "kind": "oracle",
             "sample": f"{n_layers} layer-steps of the same workload (M={M}, distinct pool layers), "
@@ -400,23 +414,22 @@ def run_reference(args):
     if rank != 0:
         return
     M = args.tokens
-    import oracle
     n = max(1, args.ref_layers)
-    xb, steps = cpu_sample_steps(M, n)
+    xb, steps = cpu_sample_steps(M, n, shared=args.shared_expert)
     for _ in range(min(args.warmup, 1)):
-        oracle.moe_decode(xb, steps[0][0], *steps[0][1], H, I, E, K)
+        oracle_step(xb, steps[0])
     t0 = time.perf_counter()
     for s in range(args.steps):
-        wr, per = steps[s % n]
-        oracle.moe_decode(xb, wr, *per, H, I, E, K)
+        oracle_step(xb, steps[s % n])
     dt = time.perf_counter() - t0
     value = M * args.steps / dt
     line = {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s",
             "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(dt * 1e3 / args.steps, 3), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": f"ling_layer_M{M}_{args.routing}", "hidden": H, "inter": I,
-                       "num_experts": E, "top_k": K, "tokens": M,
+            "config": {"workload": f"ling_layer_M{M}_{args.routing}" + ("_shared1" if args.shared_expert else ""),
+                       "hidden": H, "inter": I, "num_experts": E, "top_k": K, "tokens": M,
+                       "shared_experts": int(args.shared_expert),
                        "step": "one layer-step of the CPU oracle on host cores"},
             "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": 1, "kind": "oracle",
                              "sample": f"{args.steps} layer-steps cycling over {n} pool layers"},
@@ -544,6 +557,8 @@ def main():
     ap.add_argument("--ref-layers", type=int, default=4)
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--variant", choices=["fused", "split"], default="fused")
+    ap.add_argument("--shared-expert", action="store_true",
+                    help="one always-active shared expert per layer besides the top-8 routed ones")
     ap.add_argument("--stack", action="store_true",
                     help="chain the pool as a stack: layer l+1 takes RMSNorm(y_l)")
     ap.add_argument("--op", choices=["moe", "lm_head"], default="moe",

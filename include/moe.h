@@ -71,6 +71,21 @@ typedef enum {
                                        stacked layers, fp32); persistent kernel
                                        only: with MOE_FLAG_SPLIT_KERNELS,
                                        moe_create returns MOE_ERR_UNSUPPORTED */
+#define MOE_FLAG_SHARED_EXPERT 0x4u /* one shared expert besides the routed ones
+                                       ("NVIDIA Shows 3 Ways to Speed Up MoE
+                                       Inference on DGX Spark", Ling 3.0: 8 of
+                                       512 routed experts plus 1 shared). The
+                                       four expert arrays hold E + 1 experts;
+                                       expert E (the last) is the shared one,
+                                       same shape and format, never routed
+                                       (router_w stays [E][H]). Every token
+                                       passes it with weight 1, outside the
+                                       softmax, and its output is added after
+                                       the routed ones:
+                                         y = sum_j w_j * FFN_{id_j}(x) + FFN_E(x)
+                                       Persistent kernel only: with
+                                       MOE_FLAG_SPLIT_KERNELS, moe_create
+                                       returns MOE_ERR_UNSUPPORTED */
 
 typedef struct {
   int32_t hidden;      /* H: multiple of 32, 32..8192                        */
@@ -163,7 +178,9 @@ moe_status moe_debug_set_wait(moe_ctx* ctx, long long budget_cycles, int force_s
  *
  * It computes what moe_decode computes, with the three-kernel form of the
  * step (the MOE_FLAG_SPLIT_KERNELS path). There is no context. The layer's
- * shapes come from cfg (flags, max_tokens and device are ignored), and the
+ * shapes come from cfg (max_tokens and device are ignored; of the flags,
+ * MOE_FLAG_SHARED_EXPERT and MOE_FLAG_PRE_RMSNORM return MOE_ERR_UNSUPPORTED
+ * and MOE_FLAG_SPLIT_KERNELS is ignored), and the
  * weights, x and y are passed in directly with the layouts, alignment and
  * optional outputs of moe_load_experts and moe_decode. The scale bytes are not
  * scanned for 0xFF.

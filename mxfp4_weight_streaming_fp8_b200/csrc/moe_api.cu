@@ -32,16 +32,29 @@ moe_status validate_config(const moe_config& c) {
   if (c.num_experts < 1 || c.num_experts > moe::kMaxExperts) return MOE_ERR_INVALID_ARG;
   if (c.top_k < 1 || c.top_k > c.num_experts || c.top_k > moe::kMaxTopK) return MOE_ERR_INVALID_ARG;
   if (c.max_tokens < 1 || c.max_tokens > moe::kMaxTokens) return MOE_ERR_INVALID_ARG;
-  if (c.flags & ~(MOE_FLAG_SPLIT_KERNELS | MOE_FLAG_PRE_RMSNORM)) return MOE_ERR_INVALID_ARG;
-  if ((c.flags & MOE_FLAG_PRE_RMSNORM) && (c.flags & MOE_FLAG_SPLIT_KERNELS)) return MOE_ERR_UNSUPPORTED;
+  if (c.flags & ~(MOE_FLAG_SPLIT_KERNELS | MOE_FLAG_PRE_RMSNORM | MOE_FLAG_SHARED_EXPERT)) return MOE_ERR_INVALID_ARG;
+  if ((c.flags & (MOE_FLAG_PRE_RMSNORM | MOE_FLAG_SHARED_EXPERT)) && (c.flags & MOE_FLAG_SPLIT_KERNELS))
+    return MOE_ERR_UNSUPPORTED;
   return MOE_OK;
+}
+
+// Union entries and (token, slot) pairs a call can have; a shared expert adds
+// one entry holding one pair per token.
+void union_bounds(const moe_config& c, size_t* np, size_t* umax) {
+  const size_t E = c.num_experts, NP = (size_t)c.max_tokens * c.top_k;
+  const size_t sh = (c.flags & MOE_FLAG_SHARED_EXPERT) ? 1 : 0;
+  *np = NP + sh * c.max_tokens;
+  *umax = (E < NP ? E : NP) + sh;
 }
 
 // Shared-memory plan of the persistent kernel (mirrors k_fused's carving).
 bool make_plan(const moe_config& c, int sm_count, size_t smem_limit, moe::FusedPlan* pl) {
-  const size_t H = c.hidden, I = c.inter, E = c.num_experts, K = c.top_k, MM = c.max_tokens;
+  const size_t H = c.hidden, I = c.inter, E = c.num_experts, MM = c.max_tokens;
   const size_t G = sm_count;
-  const size_t NP = MM * K, UMAX = (E < NP ? E : NP);
+  size_t NP, UMAX;
+  union_bounds(c, &NP, &UMAX);
+  const bool shared = (c.flags & MOE_FLAG_SHARED_EXPERT) != 0;
+  const size_t n_cnt = shared ? E + 1 : E;
   const size_t nr_max = (I + G - 1) / G, nrd_max = (H + G - 1) / G;
   *pl = moe::FusedPlan{};
   pl->G = (int)G;
@@ -69,7 +82,7 @@ bool make_plan(const moe_config& c, int sm_count, size_t smem_limit, moe::FusedP
   pl->o_ppos = (int)take(NP * 4, 16);
   pl->o_union = (int)take(UMAX * 4, 16);
   pl->o_poff = (int)take((UMAX + 1) * 4, 16);
-  pl->o_cnt = (int)take(E * 4, 16);
+  pl->o_cnt = (int)take(n_cnt * 4, 16);
   pl->o_act = (int)take(MM * H, 16);
   pl->o_dsm = (int)take(NP * nrd_max * 4, 16);
   off = align_up(off, 128);
@@ -96,16 +109,18 @@ bool make_plan(const moe_config& c, int sm_count, size_t smem_limit, moe::FusedP
   pl->o_part = (int)off;
   off = align_up(off + ns_gu * (size_t)pl->part_slot, 128);
   // ring_gu also holds the router rows of the CTA and then the gathered
-  // logits [M][E] fp32 between routing and the first weight chunk
+  // logits [M][E] fp32 between routing and the first weight chunk; with a
+  // shared expert they start one slot in (slot 0 fills during routing)
   pl->wr_bytes_max = (int)(((E + G - 1) / G) * H * 4);
   if ((E + G - 1) / G > (size_t)moe::kMaxRowsPerCta) return false;  // router rows per CTA
-  const size_t staged = std::max((size_t)pl->wr_bytes_max, MM * E * 4);
+  const size_t staged = std::max((size_t)pl->wr_bytes_max, MM * E * 4) + (shared ? pl->slot_gu : 0);
   const size_t ring_gu_bytes = align_up(std::max(ns_gu * (size_t)pl->slot_gu, staged), 128);
   pl->o_ring_gu = (int)off;
   pl->o_ring_d = (int)(off + ring_gu_bytes);
   pl->smem_bytes = (int)(pl->o_ring_d + ns_d * pl->slot_d);
-  // ring_d holds the bf16 activations during routing when they fit
-  pl->x_staged = (MM * H * 2 <= ns_d * (size_t)pl->slot_d) ? 1 : 0;
+  // ring_d holds the bf16 activations during routing when they fit (after
+  // slot 0 with a shared expert)
+  pl->x_staged = (MM * H * 2 + (shared ? pl->slot_d : 0) <= ns_d * (size_t)pl->slot_d) ? 1 : 0;
   return (size_t)pl->smem_bytes <= smem_limit;
 }
 
@@ -130,6 +145,7 @@ struct moe_ctx {
   size_t smem_gateup = 0, smem_fused = 0;
   long long spin_limit = 0;
   int force_stall = 0;
+  void (*fused)(moe::Params, moe::FusedWs, moe::FusedPlan) = nullptr;  // k_fused instantiation
   moe::FusedPlan plan{};
   moe::FusedWs fws{};
 };
@@ -171,10 +187,13 @@ moe_status moe_create(const moe_config* cfg, moe_ctx** out) {
   ctx->sm_count = prop.multiProcessorCount;
   ctx->variant = (c.flags & MOE_FLAG_SPLIT_KERNELS) ? kSplit : kFused;
   ctx->spin_limit = kDefaultSpinLimit;
+  ctx->fused = (c.flags & MOE_FLAG_SHARED_EXPERT) ? moe::k_fused<true> : moe::k_fused<false>;
 
   // workspace layout
   const size_t H = c.hidden, I = c.inter, E = c.num_experts, K = c.top_k, MM = c.max_tokens;
   const size_t NP = MM * K, UMAX = (E < NP ? E : NP);
+  size_t NPF, UMAXF;  // pairs and entries of the persistent kernel
+  union_bounds(c, &NPF, &UMAXF);
   size_t off = 0;
   auto take = [&](size_t bytes) { size_t o = off; off = align_up(off + bytes, 256); return o; };
   const size_t o_ctrl = take(64 * sizeof(unsigned));
@@ -189,10 +208,10 @@ moe_status moe_create(const moe_config* cfg, moe_ctx** out) {
   const size_t o_ptok = take(NP * sizeof(int));
   const size_t o_pslot = take(NP * sizeof(int));
   const size_t o_pw = take(NP * sizeof(float));
-  const size_t o_h = take(NP * I * sizeof(float));
+  const size_t o_h = take(NPF * I * sizeof(float));
   const size_t o_flog = take(MM * E * sizeof(float));
   const size_t o_rcnt = take(sizeof(unsigned long long));
-  const size_t o_gcnt = take(UMAX * moe::kCounterStride * sizeof(unsigned long long));
+  const size_t o_gcnt = take(UMAXF * moe::kCounterStride * sizeof(unsigned long long));
   ctx->ws_bytes = off;
   if (cudaMalloc(&ctx->ws_base, ctx->ws_bytes) != cudaSuccess) {
     cudaGetLastError();
@@ -236,10 +255,10 @@ moe_status moe_create(const moe_config* cfg, moe_ctx** out) {
     err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_d, moe::k_down, moe::kThreads, 0);
   const bool plan_ok = make_plan(c, ctx->sm_count, (size_t)prop.sharedMemPerBlockOptin, &ctx->plan);
   if (err == cudaSuccess && plan_ok)
-    err = cudaFuncSetAttribute(moe::k_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, ctx->plan.smem_bytes);
+    err = cudaFuncSetAttribute(ctx->fused, cudaFuncAttributeMaxDynamicSharedMemorySize, ctx->plan.smem_bytes);
   int occ_f = 0;
   if (err == cudaSuccess && plan_ok)
-    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_f, moe::k_fused, moe::kFusedThreads,
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_f, ctx->fused, moe::kFusedThreads,
                                                         ctx->plan.smem_bytes);
   if (err != cudaSuccess || occ_g < 1 || occ_d < 1 || !plan_ok || occ_f < 1) {
     cudaGetLastError();
@@ -274,7 +293,7 @@ moe_status moe_load_experts(moe_ctx* ctx, const float* router_w, const uint8_t* 
   if (!guard.ok) return MOE_ERR_CUDA;
   const moe_config& c = ctx->cfg;
   if (!(load_flags & MOE_LOAD_SKIP_VALIDATE)) {
-    const size_t E = c.num_experts, H = c.hidden, I = c.inter;
+    const size_t E = c.num_experts + ((c.flags & MOE_FLAG_SHARED_EXPERT) ? 1 : 0), H = c.hidden, I = c.inter;
     unsigned* bad = ctx->ws.ctrl + 4;
     if (cudaMemset(bad, 0, sizeof(unsigned)) != cudaSuccess) return MOE_ERR_CUDA;
     moe::k_scan_scales<<<ctx->sm_count * 4, 256>>>(w13_scales, E * 2 * I * (H / 32), bad);
@@ -353,7 +372,7 @@ moe_status moe_decode(moe_ctx* ctx, const void* x_bf16, int32_t M, void* y_bf16,
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, moe::k_fused, p, ctx->fws, ctx->plan) != cudaSuccess) {
+    if (cudaLaunchKernelEx(&cfg, ctx->fused, p, ctx->fws, ctx->plan) != cudaSuccess) {
       cudaGetLastError();
       return MOE_ERR_CUDA;
     }
@@ -421,9 +440,11 @@ moe_status moe_query(const moe_ctx* ctx, char* buf, size_t len) {
                  "{\"lib\": \"libmoe\", \"arch\": \"sm_100a\", \"device\": %d, \"sm_count\": %d, "
                  "\"variant\": \"fused\", \"kernels\": [\"k_fused\"], \"grid\": [%d], \"threads\": %d, "
                  "\"smem\": %d, \"ring_gu\": [%d, %d], \"ring_d\": [%d, %d], \"pdl\": true, \"pre_rmsnorm\": %s, "
+                 "\"shared_expert\": %s, "
                  "\"hidden\": %d, \"inter\": %d, \"num_experts\": %d, \"top_k\": %d, \"max_tokens\": %d}",
                  ctx->dev, ctx->sm_count, pl.G, moe::kFusedThreads, pl.smem_bytes, pl.ns_gu, pl.slot_gu, pl.ns_d,
-                 pl.slot_d, (c.flags & MOE_FLAG_PRE_RMSNORM) ? "true" : "false", c.hidden, c.inter, c.num_experts,
+                 pl.slot_d, (c.flags & MOE_FLAG_PRE_RMSNORM) ? "true" : "false",
+                 (c.flags & MOE_FLAG_SHARED_EXPERT) ? "true" : "false", c.hidden, c.inter, c.num_experts,
                  c.top_k, c.max_tokens);
   }
   if (n < 0 || (size_t)n >= len) return MOE_ERR_INVALID_ARG;

@@ -668,9 +668,10 @@ __device__ __forceinline__ void topk_warp(const float* l, int E, int K, int* ids
 
 // One warp, M*K <= 32 pairs: the expert union (ascending ids) and the pairs
 // grouped by expert in (token, slot) order, from ranks computed with
-// shuffles (no shared-memory scratch). Pair i = (i / K, i % K).
+// shuffles (no shared-memory scratch). Pair i = (i / K, i % K); pair
+// positions start at pbase.
 __device__ __forceinline__ int union_small(const int* s_ids, int np, int K, int* s_union, int* s_poff, int* s_pm,
-                                           int* s_ppos) {
+                                           int* s_ppos, int pbase) {
   const int lane = threadIdx.x & 31;
   const int id = (lane < np) ? s_ids[lane] : 0x7fffffff;
   int rank = 0, urank = 0;
@@ -684,18 +685,26 @@ __device__ __forceinline__ int union_small(const int* s_ids, int np, int K, int*
   }
   const int U = __popc(__ballot_sync(0xffffffffu, leader));
   if (lane < np) {
-    s_pm[rank] = lane / K;
-    s_ppos[lane] = rank;
+    s_pm[pbase + rank] = lane / K;
+    s_ppos[lane] = pbase + rank;
     if (leader) {
       s_union[urank] = id;
-      s_poff[urank] = rank;
+      s_poff[urank] = pbase + rank;
     }
   }
-  if (lane == 0) s_poff[U] = np;
+  if (lane == 0) s_poff[U] = pbase + np;
   return U;
 }
 
 // ---------------------------------------------------------------- the kernel
+// kShared: the weight arrays hold E + 1 experts and expert E is a shared
+// expert that every token passes with weight 1 ("NVIDIA Shows 3 Ways to Speed
+// Up MoE Inference on DGX Spark", Ling 3.0: 8 routed experts plus 1 shared).
+// It is union entry 0, with pairs 0 .. M-1 (token order); the routed entries
+// follow. It needs no routing, so its chunks are requested at kernel start and
+// its gate/up items run while the router logits of the other CTAs arrive;
+// the routing scratch then sits one slot into each ring, clear of slot 0.
+template <bool kShared>
 __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw, FusedPlan pl) {
   extern __shared__ __align__(128) unsigned char smem[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -729,9 +738,10 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
   uint8_t* hstage = smem + pl.o_h;
   uint8_t* ring_gu = smem + pl.o_ring_gu;
   uint8_t* ring_d = smem + pl.o_ring_d;
-  float* wr_s = reinterpret_cast<float*>(ring_gu);       // router rows (routing phase only)
-  float* s_logit = reinterpret_cast<float*>(ring_gu);    // gathered logits (after the router rows)
-  uint4* x_s = reinterpret_cast<uint4*>(ring_d);         // staged bf16 x (routing phase only)
+  float* wr_s = reinterpret_cast<float*>(ring_gu + (kShared ? pl.slot_gu : 0));  // router rows (routing phase only)
+  float* s_logit = wr_s;                                                          // gathered logits (after them)
+  uint4* x_s = reinterpret_cast<uint4*>(ring_d + (kShared ? pl.slot_d : 0));      // staged bf16 x (routing only)
+  const int ub = kShared ? 1 : 0;  // first routed union entry
 
   const int e0 = (int)((long long)E * b / G), e1 = (int)((long long)E * (b + 1) / G), ne = e1 - e0;
   // this CTA's share of every union expert (independent of the routing)
@@ -740,6 +750,120 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
   const int gu_items = (nr > 0) ? (nr + kGuRowsPerItem - 1) / kGuRowsPerItem : 0;  // per expert
   const int d_items = (nrd > 0) ? (nrd + kDownRowsPerItem - 1) / kDownRowsPerItem : 0;
 
+  // ---------------- weight stream. Each bulk copy costs its issuing thread
+  //   about a hundred nanoseconds, so the first use of every ring slot is
+  //   issued by all warps in parallel (lane 0 of warp w takes entries w, w+16,
+  //   ...; gate/up chunks first, then down chunks); later uses wait for their
+  //   slot to drain and are issued by lane 0 of warp 0.
+  auto issue_gu = [&](int u) {
+    const int e = s_union[u];
+    const int slot = u % pl.ns_gu;
+    uint8_t* sp = ring_gu + (size_t)slot * pl.slot_gu;
+    GuChunk ch;
+    size_t ga0, ua0;
+    unsigned gn, un;
+    const unsigned bytes = gu_layout(p, e, n0, nr, sp, &ch, &ga0, &gn, &ua0, &un);
+    mbar_expect_tx(full_gu + slot, bytes);
+    const size_t grow = (size_t)e * 2 * I + n0, urow = grow + I;
+    const unsigned codes = (unsigned)(nr * H / 2);
+    tma_load_1d(sp, p.w13c + grow * (H / 2), codes, full_gu + slot);
+    tma_load_1d(sp + codes, p.w13c + urow * (H / 2), codes, full_gu + slot);
+    tma_load_1d(sp + 2 * codes, p.w13s + ga0, gn, full_gu + slot);
+    tma_load_1d(sp + 2 * codes + gn, p.w13s + ua0, un, full_gu + slot);
+  };
+  auto issue_d = [&](int u) {
+    const int e = s_union[u];
+    const int slot = u % pl.ns_d;
+    uint8_t* sp = ring_d + (size_t)slot * pl.slot_d;
+    DChunk ch;
+    size_t sa0;
+    unsigned sn;
+    const unsigned bytes = d_layout(p, e, r0, nrd, sp, &ch, &sa0, &sn);
+    mbar_expect_tx(full_d + slot, bytes);
+    const unsigned codes = (unsigned)(nrd * I / 2);
+    tma_load_1d(sp, p.w2c + ((size_t)e * H + r0) * (I / 2), codes, full_d + slot);
+    tma_load_1d(sp + codes, p.w2s + sa0, sn, full_d + slot);
+  };
+  // one gate/up item: rows of item g of this CTA's chunk of entry u, every
+  // pair of the entry; the last item of the entry publishes it GPU-wide
+  auto gu_work = [&](int u, int g) {
+    const int slot = u % pl.ns_gu, use = u / pl.ns_gu;
+    if (use > 0 && lane == 0) smem_count_wait(done_gu + slot, (unsigned)(use * gu_items), p);
+    __syncwarp();
+    mbar_wait(full_gu + slot, use & 1, p);
+    GuChunk ch;
+    size_t ga0, ua0;
+    unsigned gn, un;
+    gu_layout(p, s_union[u], n0, nr, ring_gu + (size_t)slot * pl.slot_gu, &ch, &ga0, &gn, &ua0, &un);
+    const int pb = s_poff[u], pe = s_poff[u + 1];
+    if (pe - pb >= kMmaMinPairs && pl.part_slot > 0) {
+      // several pairs: the entry's items split K; each runs warp MMAs over
+      // all rows and pairs, and the last one to finish sums the partials
+      // in chunk order (deterministic), applies SwiGLU and writes h
+      const int nkb = H / 32, nrg = (nr + 7) >> 3, nct = min(pl.part_ct, (pe - pb + 7) >> 3);
+      const int kb0 = g * nkb / gu_items, kb1 = (g + 1) * nkb / gu_items;
+      float4* part = reinterpret_cast<float4*>(smem + pl.o_part + (size_t)slot * pl.part_slot);
+      for (int rg = 0; rg < nrg; ++rg) {
+        float acc[4 * kMaxPairTiles];
+        gu_mma_slice(p, ch, 8 * rg, min(8, nr - 8 * rg), kb0, kb1, pb, pe, s_pm, act, acc);
+#pragma unroll
+        for (int ct = 0; ct < kMaxPairTiles; ++ct)
+          if (ct < nct)
+            part[((g * nrg + rg) * pl.part_ct + ct) * 32 + lane] =
+                make_float4(acc[4 * ct], acc[4 * ct + 1], acc[4 * ct + 2], acc[4 * ct + 3]);
+      }
+      __syncwarp();
+      unsigned done = 0;
+      if (lane == 0) done = atom_add_acqrel_cta_smem(reinterpret_cast<unsigned*>(s_cnt + u), 1u) + 1u;
+      done = __shfl_sync(0xffffffffu, done, 0);
+      if ((int)done == gu_items) {
+        const int gq = lane >> 2, tq = lane & 3;
+        for (int rg = 0; rg < nrg; ++rg) {
+          const int row = 8 * rg + gq;
+          for (int ct = 0; ct < nct; ++ct) {
+            float4 v = part[(rg * pl.part_ct + ct) * 32 + lane];
+            for (int c = 1; c < gu_items; ++c) {
+              const float4 w = part[((c * nrg + rg) * pl.part_ct + ct) * 32 + lane];
+              v.x += w.x; v.y += w.y; v.z += w.z; v.w += w.w;
+            }
+            const float gg[2] = {v.x, v.y}, uu[2] = {v.z, v.w};
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+              const int q = 8 * ct + 2 * tq + i;
+              if (q < pe - pb && row < nr) {
+                const float sx = s_xs[s_pm[pb + q]];
+                const float gv = gg[i] * sx, uv = uu[i] * sx;
+                p.ws.h[(size_t)(pb + q) * I + n0 + row] = gv / (1.f + expf(-gv)) * uv;
+              }
+            }
+          }
+        }
+        __syncwarp();
+        // orders the warp's h stores (through the warp barrier) before the
+        // GPU-wide arrival for the entry
+        if (lane == 0) grid_arrive(gu_counter(fw, u));
+      }
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(empty_gu + slot);
+        atomicAdd(done_gu + slot, 1u);
+      }
+      __syncwarp();
+      return;
+    }
+    const int a = g * kGuRowsPerItem, cnt = min(kGuRowsPerItem, nr - a);
+    gu_item(p, ch, a, cnt, n0, pb, pe, s_pm, act, s_xs);
+    __syncwarp();
+    if (lane == 0) {
+      mbar_arrive(empty_gu + slot);
+      atomicAdd(done_gu + slot, 1u);
+      // acq_rel at CTA scope: the warp completing the entry sees every
+      // other warp's h stores, then releases them GPU-wide
+      const unsigned done = atom_add_acqrel_cta_smem(reinterpret_cast<unsigned*>(s_cnt + u), 1u) + 1u;
+      if ((int)done == gu_items) grid_arrive(gu_counter(fw, u));
+    }
+    __syncwarp();
+  };
   if (tid < kMaxSlots) {
     if (tid < pl.ns_gu) { mbar_init(full_gu + tid, 1); mbar_init(empty_gu + tid, max(1, gu_items)); }
     if (tid < pl.ns_d) {
@@ -758,12 +882,28 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
       tma_load_1d(wr_s, p.wr + (size_t)e0 * H, (unsigned)(ne * H * 4), wr_bar);
     }
   }
+  if constexpr (kShared) {
+    // the shared entry's chunks (thread 0 initialised slot 0 of both rings)
+    if (tid == 0) {
+      s_union[0] = E;
+      if (nr > 0) issue_gu(0);
+      if (nrd > 0) issue_d(0);
+    }
+  }
   // Everything above is independent of the previous kernel on the stream.
   pdl_wait();
   if (tid == 0) {
     s_int[1] = (int)(ld_relaxed_u32(fw.epoch) + 1u);
-    s_int[2] = 0;  // gate/up queue head
-    s_int[3] = 0;  // down queue head
+    s_int[2] = kShared ? gu_items : 0;  // queue head (the shared entry's gate/up items run early)
+    s_int[3] = 0;
+    if constexpr (kShared) {
+      s_poff[0] = 0;
+      s_poff[1] = M;
+      s_cnt[0] = 0;
+    }
+  }
+  if constexpr (kShared) {
+    if (tid < M) s_pm[tid] = tid;
   }
   unsigned* s_amax_u = reinterpret_cast<unsigned*>(s_amax);
   if (tid < M) s_amax_u[tid] = 0u;
@@ -931,6 +1071,12 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
     if (b == 0 && p.out_xq) *reinterpret_cast<uint2*>(p.out_xq + (size_t)i * 8) = out;
   }
   if (b == 0 && p.out_xscale && tid < M) p.out_xscale[tid] = s_xs[tid];
+  if constexpr (kShared) {
+    // the shared entry's gate/up items, while thread 0 waits for the router
+    __syncthreads();
+    if (warp >= 1)
+      for (int g = warp - 1; g < gu_items; g += kFusedWarps - 1) gu_work(0, g);
+  }
 
   if (tid == 0)
     grid_wait(fw.route_cnt, (unsigned long long)(p.force_stall ? epoch + 0x40000000u : epoch) * G, p);
@@ -961,20 +1107,22 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
 
   // ---- A4: expert union (ascending ids) and the (token, slot) pairs of each
   //          entry in (token, slot) order; one warp, no block barriers
-  const int np = M * K;
+  // (with a shared expert, routed entries start at 1 and their pairs at M)
+  const int np = M * K, pbase = kShared ? M : 0;
   if (warp == 0 && np <= 32) {
-    const int Us = union_small(s_ids, np, K, s_union, s_poff, s_pm, s_ppos);
-    if (lane == 0) s_int[0] = Us;
-    for (int u = lane; u < Us; u += 32) s_cnt[u] = 0;  // per-entry gate/up item counters
+    const int Us = union_small(s_ids, np, K, s_union + ub, s_poff + ub, s_pm, s_ppos, pbase);
+    if (lane == 0) s_int[0] = ub + Us;
+    for (int u = lane; u < Us; u += 32) s_cnt[ub + u] = 0;  // per-entry gate/up item counters
   } else if (warp == 0) {
-    for (int e = lane; e < E; e += 32) s_cnt[e] = 0;
+    int* s_ec = s_cnt + ub;  // [E] per-expert scratch, clear of the shared entry's counter
+    for (int e = lane; e < E; e += 32) s_ec[e] = 0;
     __syncwarp();
-    for (int i = lane; i < np; i += 32) atomicAdd(&s_cnt[s_ids[i]], 1);
+    for (int i = lane; i < np; i += 32) atomicAdd(&s_ec[s_ids[i]], 1);
     __syncwarp();
     const int per = (E + 31) / 32;
     const int ea = min(E, lane * per), eb = min(E, ea + per);
     int nz = 0, cs = 0;
-    for (int e = ea; e < eb; ++e) { nz += s_cnt[e] > 0; cs += s_cnt[e]; }
+    for (int e = ea; e < eb; ++e) { nz += s_ec[e] > 0; cs += s_ec[e]; }
     int nz_ex = nz, cs_ex = cs;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -986,18 +1134,18 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
     cs_ex -= cs;
     __syncwarp();
     for (int e = ea; e < eb; ++e) {
-      const int c = s_cnt[e];
+      const int c = s_ec[e];
       if (c > 0) {
-        s_union[nz_ex] = e;
-        s_poff[nz_ex] = cs_ex;
+        s_union[ub + nz_ex] = e;
+        s_poff[ub + nz_ex] = pbase + cs_ex;
         ++nz_ex;
         cs_ex += c;
       }
-      s_cnt[e] = cs_ex - c;  // first pair position of expert e
+      s_ec[e] = pbase + cs_ex - c;  // first pair position of expert e
     }
     if (lane == 31) {
-      s_poff[nz_ex] = cs_ex;
-      s_int[0] = nz_ex;
+      s_poff[ub + nz_ex] = pbase + cs_ex;
+      s_int[0] = ub + nz_ex;
     }
     __syncwarp();
     // stable placement: rank within each 32-pair batch by matching experts
@@ -1008,63 +1156,29 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
       const int rank = __popc(same & ((1u << lane) - 1u));
       int pos = 0;
       if (i < np) {
-        pos = s_cnt[e] + rank;
+        pos = s_ec[e] + rank;
         s_pm[pos] = i / K;
         s_ppos[i] = pos;
       }
       __syncwarp();
-      if (i < np && rank == 0) s_cnt[e] += __popc(same);
+      if (i < np && rank == 0) s_ec[e] += __popc(same);
       __syncwarp();
     }
     const int U = s_int[0];
     __syncwarp();
-    for (int u = lane; u < U; u += 32) s_cnt[u] = 0;  // per-entry gate/up item counters
+    for (int u = ub + lane; u < U; u += 32) s_cnt[u] = 0;  // per-entry gate/up item counters
   }
   __syncthreads();
   const int U = s_int[0];
 
-  // ---------------- weight stream. Each bulk copy costs its issuing thread
-  //   about a hundred nanoseconds, so the first use of every ring slot is
-  //   issued by all warps in parallel (lane 0 of warp w takes entries w, w+16,
-  //   ...; gate/up chunks first, then down chunks); later uses wait for their
-  //   slot to drain and are issued by lane 0 of warp 0.
-  auto issue_gu = [&](int u) {
-    const int e = s_union[u];
-    const int slot = u % pl.ns_gu;
-    uint8_t* sp = ring_gu + (size_t)slot * pl.slot_gu;
-    GuChunk ch;
-    size_t ga0, ua0;
-    unsigned gn, un;
-    const unsigned bytes = gu_layout(p, e, n0, nr, sp, &ch, &ga0, &gn, &ua0, &un);
-    mbar_expect_tx(full_gu + slot, bytes);
-    const size_t grow = (size_t)e * 2 * I + n0, urow = grow + I;
-    const unsigned codes = (unsigned)(nr * H / 2);
-    tma_load_1d(sp, p.w13c + grow * (H / 2), codes, full_gu + slot);
-    tma_load_1d(sp + codes, p.w13c + urow * (H / 2), codes, full_gu + slot);
-    tma_load_1d(sp + 2 * codes, p.w13s + ga0, gn, full_gu + slot);
-    tma_load_1d(sp + 2 * codes + gn, p.w13s + ua0, un, full_gu + slot);
-  };
-  auto issue_d = [&](int u) {
-    const int e = s_union[u];
-    const int slot = u % pl.ns_d;
-    uint8_t* sp = ring_d + (size_t)slot * pl.slot_d;
-    DChunk ch;
-    size_t sa0;
-    unsigned sn;
-    const unsigned bytes = d_layout(p, e, r0, nrd, sp, &ch, &sa0, &sn);
-    mbar_expect_tx(full_d + slot, bytes);
-    const unsigned codes = (unsigned)(nrd * I / 2);
-    tma_load_1d(sp, p.w2c + ((size_t)e * H + r0) * (I / 2), codes, full_d + slot);
-    tma_load_1d(sp + codes, p.w2s + sa0, sn, full_d + slot);
-  };
   const int n_gu0 = (nr > 0) ? min(U, pl.ns_gu) : 0;
   const int n_d0 = (nrd > 0) ? min(U, pl.ns_d) : 0;
-  if (lane == 0 && (warp < n_gu0 || warp < n_d0)) {
+  if (lane == 0 && (ub + warp < n_gu0 || ub + warp < n_d0)) {
     // ring_gu and ring_d were read and written through the generic proxy
     // during routing; order that before the async-proxy (TMA) writes
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    for (int u = warp; u < n_gu0; u += kFusedWarps) issue_gu(u);
-    for (int u = warp; u < n_d0; u += kFusedWarps) issue_d(u);
+    for (int u = ub + warp; u < n_gu0; u += kFusedWarps) issue_gu(u);
+    for (int u = ub + warp; u < n_d0; u += kFusedWarps) issue_d(u);
   }
   if (warp == 0) {
     // refills of drained slots (more union entries than slots): one thread
@@ -1142,83 +1256,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
       sub = q % d_items;
     }
     if (!is_down) {
-      const int g = sub;
-      const int slot = u % pl.ns_gu, use = u / pl.ns_gu;
-      if (use > 0 && lane == 0) smem_count_wait(done_gu + slot, (unsigned)(use * gu_items), p);
-      __syncwarp();
-      mbar_wait(full_gu + slot, use & 1, p);
-      GuChunk ch;
-      size_t ga0, ua0;
-      unsigned gn, un;
-      gu_layout(p, s_union[u], n0, nr, ring_gu + (size_t)slot * pl.slot_gu, &ch, &ga0, &gn, &ua0, &un);
-      const int pb = s_poff[u], pe = s_poff[u + 1];
-      if (pe - pb >= kMmaMinPairs && pl.part_slot > 0) {
-        // several pairs: the entry's items split K; each runs warp MMAs over
-        // all rows and pairs, and the last one to finish sums the partials
-        // in chunk order (deterministic), applies SwiGLU and writes h
-        const int nkb = H / 32, nrg = (nr + 7) >> 3, nct = min(pl.part_ct, (pe - pb + 7) >> 3);
-        const int kb0 = g * nkb / gu_items, kb1 = (g + 1) * nkb / gu_items;
-        float4* part = reinterpret_cast<float4*>(smem + pl.o_part + (size_t)slot * pl.part_slot);
-        for (int rg = 0; rg < nrg; ++rg) {
-          float acc[4 * kMaxPairTiles];
-          gu_mma_slice(p, ch, 8 * rg, min(8, nr - 8 * rg), kb0, kb1, pb, pe, s_pm, act, acc);
-#pragma unroll
-          for (int ct = 0; ct < kMaxPairTiles; ++ct)
-            if (ct < nct)
-              part[((g * nrg + rg) * pl.part_ct + ct) * 32 + lane] =
-                  make_float4(acc[4 * ct], acc[4 * ct + 1], acc[4 * ct + 2], acc[4 * ct + 3]);
-        }
-        __syncwarp();
-        unsigned done = 0;
-        if (lane == 0) done = atom_add_acqrel_cta_smem(reinterpret_cast<unsigned*>(s_cnt + u), 1u) + 1u;
-        done = __shfl_sync(0xffffffffu, done, 0);
-        if ((int)done == gu_items) {
-          const int gq = lane >> 2, tq = lane & 3;
-          for (int rg = 0; rg < nrg; ++rg) {
-            const int row = 8 * rg + gq;
-            for (int ct = 0; ct < nct; ++ct) {
-              float4 v = part[(rg * pl.part_ct + ct) * 32 + lane];
-              for (int c = 1; c < gu_items; ++c) {
-                const float4 w = part[((c * nrg + rg) * pl.part_ct + ct) * 32 + lane];
-                v.x += w.x; v.y += w.y; v.z += w.z; v.w += w.w;
-              }
-              const float gg[2] = {v.x, v.y}, uu[2] = {v.z, v.w};
-#pragma unroll
-              for (int i = 0; i < 2; ++i) {
-                const int q = 8 * ct + 2 * tq + i;
-                if (q < pe - pb && row < nr) {
-                  const float sx = s_xs[s_pm[pb + q]];
-                  const float gv = gg[i] * sx, uv = uu[i] * sx;
-                  p.ws.h[(size_t)(pb + q) * I + n0 + row] = gv / (1.f + expf(-gv)) * uv;
-                }
-              }
-            }
-          }
-          __syncwarp();
-          // orders the warp's h stores (through the warp barrier) before the
-          // GPU-wide arrival for the entry
-          if (lane == 0) grid_arrive(gu_counter(fw, u));
-        }
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(empty_gu + slot);
-          atomicAdd(done_gu + slot, 1u);
-        }
-        __syncwarp();
-        continue;
-      }
-      const int a = g * kGuRowsPerItem, cnt = min(kGuRowsPerItem, nr - a);
-      gu_item(p, ch, a, cnt, n0, pb, pe, s_pm, act, s_xs);
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(empty_gu + slot);
-        atomicAdd(done_gu + slot, 1u);
-        // acq_rel at CTA scope: the warp completing the entry sees every
-        // other warp's h stores, then releases them GPU-wide
-        const unsigned done = atom_add_acqrel_cta_smem(reinterpret_cast<unsigned*>(s_cnt + u), 1u) + 1u;
-        if ((int)done == gu_items) grid_arrive(gu_counter(fw, u));
-      }
-      __syncwarp();
+      gu_work(u, sub);
     } else {
       const int gd = sub;
       const int slot = u % pl.ns_d, use = u / pl.ns_d;
@@ -1261,6 +1299,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
     const int m = i / nrd, rl = i % nrd;
     float acc = 0.f;
     for (int s = 0; s < K; ++s) acc = fmaf(s_w[m * K + s], dsm[(size_t)s_ppos[m * K + s] * pl.rpc_max + rl], acc);
+    if constexpr (kShared) acc += dsm[(size_t)m * pl.rpc_max + rl];  // shared expert, weight 1
     p.y[(size_t)m * H + r0 + rl] = __float2bfloat16_rn(acc);
   }
   if (b == 0 && ct == 0) {

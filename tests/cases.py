@@ -28,14 +28,15 @@ def bits(t: torch.Tensor) -> np.ndarray:
 class Layer:
     """Seeded inputs of one MoE layer, on the device and (lazily) on the CPU."""
 
-    def __init__(self, H, I, E, K, M, seed=0, layer=0, mode="gap", device="cuda:0"):
+    def __init__(self, H, I, E, K, M, seed=0, layer=0, mode="gap", device="cuda:0", shared=False):
         self.H, self.I, self.E, self.K, self.M = H, I, E, K, M
         self.seed, self.layer = seed, layer
+        self.shared = shared  # expert E (the last of E + 1) is a shared expert
         self.x = synth.gen_x(seed, M, H, layer=layer)
         self.wr = synth.force_router(self.x, synth.gen_router(seed, layer, E, H), K, mode, seed=seed,
                                      layer=layer) if M > 0 else synth.gen_router(seed, layer, E, H)
         self.dev = torch.device(device)
-        self.experts = synth.layer_experts_torch(seed, layer, E, H, I, self.dev)
+        self.experts = synth.layer_experts_torch(seed, layer, E + int(shared), H, I, self.dev)
         self.wr_d = torch.from_numpy(self.wr).to(self.dev)
         self.x_d = self.x.to(self.dev)
 
@@ -55,9 +56,14 @@ class Layer:
         logits = oracle.router_logits(xb, self.wr)
         ids, _ = oracle.topk(logits, self.K)
         per = self.expert_slices(ids)
+        if self.shared:
+            sh = synth.expert_np(self.seed, self.layer, self.E, self.H, self.I)
+            return oracle.moe_decode_shared(xb, self.wr, *per, sh, self.H, self.I, self.E, self.K)
         return oracle.moe_decode(xb, self.wr, *per, self.H, self.I, self.E, self.K)
 
     def make_ctx(self, flags=0, max_tokens=None):
+        if self.shared:
+            flags |= moe.MOE_FLAG_SHARED_EXPERT
         ctx = moe.MoELayer(self.H, self.I, self.E, self.K, max_tokens or max(1, self.M), flags=flags,
                            device=self.dev.index or 0)
         ctx.load_experts(self.wr_d, *self.experts)

@@ -90,6 +90,32 @@ def test_persistent_kernel_plan_fits(L, shape):
     assert pl["o_act"] % 16 == 0 and pl["o_ring_gu"] % 128 == 0 and pl["o_ring_d"] % 128 == 0
 
 
+def test_shared_expert_flag_without_gpu(L):
+    """The shared-expert flag is a persistent-kernel option: with the split
+    path it is refused before any CUDA call. Its plan has one more union
+    entry and one more pair per token, and still fits."""
+    out = ctypes.c_void_p()
+    c = moe.moe_config(256, 64, 16, 2, 1, moe.MOE_FLAG_SHARED_EXPERT | moe.MOE_FLAG_SPLIT_KERNELS, 0)
+    assert L.moe_create(ctypes.byref(c), ctypes.byref(out)) == 2 and not out.value
+    c = moe.moe_config(256, 64, 16, 2, 1, moe.MOE_FLAG_SHARED_EXPERT | moe.MOE_FLAG_PRE_RMSNORM | 0x8, 0)
+    assert L.moe_create(ctypes.byref(c), ctypes.byref(out)) == 1 and not out.value
+    for shape in [(2560, 768, 256, 8, 1), (2560, 768, 256, 8, 32), (128, 64, 8, 8, 3), (256, 64, 16, 2, 1)]:
+        st0, base = moe.plan_query(*shape)
+        st, pl = moe.plan_query(*shape, flags=moe.MOE_FLAG_SHARED_EXPERT)
+        assert st == 0 and pl["ok"], pl
+        H, I, E, K, MM = shape
+        assert pl["ns_gu"] >= min(2, min(E, MM * K) + 1) and pl["ns_d"] >= min(2, min(E, MM * K) + 1)
+        # dsm grows by one row block per token
+        assert pl["o_dsm"] >= base["o_dsm"]
+        assert pl["smem"] <= 232448
+        # slot 0 of each ring fills during routing: the router rows, the
+        # gathered logits and the staged x start one slot in and still fit
+        staged = max(pl["router_bytes_per_cta"], MM * E * 4)
+        assert pl["o_ring_d"] - pl["o_ring_gu"] >= pl["slot_gu"] + staged
+        if pl["x_staged"]:
+            assert MM * H * 2 + pl["slot_d"] <= pl["ns_d"] * pl["slot_d"]
+
+
 def test_plan_rejects_what_does_not_fit(L):
     st, pl = moe.plan_query(8192, 4096, 1024, 32, 32)
     assert st == 2 and not pl["ok"]

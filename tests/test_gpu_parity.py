@@ -89,6 +89,36 @@ def test_shared_experts_many_pairs(M):
     compare(L, got, L.oracle(tokens=sample), tokens=sample)
 
 
+@pytest.mark.parametrize("shape,M,mode", [((256, 64, 16, 2), 1, "natural"), ((160, 96, 12, 4), 7, "gap"),
+                                          ((2560, 768, 256, 8), 1, "gap"), ((2560, 768, 256, 8), 4, "natural"),
+                                          ((2560, 768, 256, 8), 5, "shared"), ((128, 64, 8, 8), 3, "natural")])
+def test_shared_expert(shape, M, mode):
+    """One always-active shared expert besides the routed ones: every token
+    checked in full. Covers the tiny and ragged layers, the Ling-shaped layer
+    at M=1 and M=4, five tokens on the same 8 routed experts (the shared
+    entry then has as many pairs as each routed one, so both take the
+    tensor-core gate/up path), and a layer whose union holds every routed
+    expert (the shared entry is then the (E+1)-th)."""
+    H, I, E, K = shape
+    L = Layer(H, I, E, K, M, seed=21, mode=mode, shared=True)
+    ctx = L.make_ctx(0)
+    assert ctx.query()["shared_expert"] is True
+    got = L.run(ctx)
+    compare(L, got, L.oracle())
+    again = L.run(ctx)
+    assert torch.equal(got["y"], again["y"])
+
+
+def test_shared_expert_ring_reuse_sampled():
+    """Shared expert in a context sized for 32 tokens (few ring slots, so the
+    shared entry reuses a slot), M=32 under Zipf routing, sampled tokens."""
+    M = 32
+    L = Layer(2560, 768, 256, 8, M, seed=22, mode="zipf", shared=True)
+    got = L.run(L.make_ctx(0, max_tokens=32))
+    sample = [0, 13, 31]
+    compare(L, got, L.oracle(tokens=sample), tokens=sample)
+
+
 @pytest.mark.parametrize("M,mode", [(1, "gap"), (2, "zipf"), (4, "gap"), (3, "shared")])
 def test_deep_ring_reuse(M, mode):
     """A context sized for 32 tokens leaves 4 ring slots, so every slot is
