@@ -701,9 +701,12 @@ __device__ __forceinline__ int union_small(const int* s_ids, int np, int K, int*
 // expert that every token passes with weight 1 ("NVIDIA Shows 3 Ways to Speed
 // Up MoE Inference on DGX Spark", Ling 3.0: 8 routed experts plus 1 shared).
 // It is union entry 0, with pairs 0 .. M-1 (token order); the routed entries
-// follow. It needs no routing, so its chunks are requested at kernel start and
-// its gate/up items run while the router logits of the other CTAs arrive;
-// the routing scratch then sits one slot into each ring, clear of slot 0.
+// follow. It needs no routing, so its chunks are requested before routing
+// starts (by two warps that have no activation rows to scan at M=1), and the
+// routing scratch sits one slot into each ring, clear of slot 0. Its gate/up
+// items are the head of the work queue. (Running them while the router
+// logits arrive measured slower: the wait for the router is shorter than an
+// item, so they lengthened routing.)
 template <bool kShared>
 __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw, FusedPlan pl) {
   extern __shared__ __align__(128) unsigned char smem[];
@@ -882,21 +885,14 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
       tma_load_1d(wr_s, p.wr + (size_t)e0 * H, (unsigned)(ne * H * 4), wr_bar);
     }
   }
-  if constexpr (kShared) {
-    // the shared entry's chunks (thread 0 initialised slot 0 of both rings)
-    if (tid == 0) {
-      s_union[0] = E;
-      if (nr > 0) issue_gu(0);
-      if (nrd > 0) issue_d(0);
-    }
-  }
   // Everything above is independent of the previous kernel on the stream.
   pdl_wait();
   if (tid == 0) {
     s_int[1] = (int)(ld_relaxed_u32(fw.epoch) + 1u);
-    s_int[2] = kShared ? gu_items : 0;  // queue head (the shared entry's gate/up items run early)
-    s_int[3] = 0;
+    s_int[2] = 0;  // gate/up queue head
+    s_int[3] = 0;  // down queue head
     if constexpr (kShared) {
+      s_union[0] = E;
       s_poff[0] = 0;
       s_poff[1] = M;
       s_cnt[0] = 0;
@@ -909,6 +905,12 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
   if (tid < M) s_amax_u[tid] = 0u;
   __syncthreads();
   const unsigned epoch = (unsigned)s_int[1];
+  if constexpr (kShared) {
+    // the shared entry's chunks, into slot 0 of each ring (its barriers were
+    // initialised before the block barrier above)
+    if (lane == 0 && warp == kFusedWarps - 1 && nr > 0) issue_gu(0);
+    if (lane == 0 && warp == kFusedWarps - 2 && nrd > 0) issue_d(0);
+  }
 
   // ---- A1: per-token amax (unsigned max of |x| bit patterns) and, when it
   //          fits, a shared-memory copy of x for the router
@@ -1071,12 +1073,6 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
     if (b == 0 && p.out_xq) *reinterpret_cast<uint2*>(p.out_xq + (size_t)i * 8) = out;
   }
   if (b == 0 && p.out_xscale && tid < M) p.out_xscale[tid] = s_xs[tid];
-  if constexpr (kShared) {
-    // the shared entry's gate/up items, while thread 0 waits for the router
-    __syncthreads();
-    if (warp >= 1)
-      for (int g = warp - 1; g < gu_items; g += kFusedWarps - 1) gu_work(0, g);
-  }
 
   if (tid == 0)
     grid_wait(fw.route_cnt, (unsigned long long)(p.force_stall ? epoch + 0x40000000u : epoch) * G, p);
