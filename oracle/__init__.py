@@ -59,6 +59,11 @@ def lib():
         L.oracle_rmsnorm.argtypes = [ctypes.c_int, ctypes.c_int, _u16p, ctypes.c_double, _u16p]
         L.oracle_moe_decode_shared.argtypes = ([ctypes.c_int] * 5 + [_u16p, _f32p] + [_u8pp] * 4 + [_u8p] * 4 +
                                                [_u8p, _f32p, _f64p, _i32p, _f64p, _f64p])
+        L.oracle_quantize_f32.argtypes = [ctypes.c_int, _f32p, _u8p, _f32p]
+        L.oracle_expert_a8.argtypes = [ctypes.c_int, ctypes.c_int, _u8p, ctypes.c_float] + [_u8p] * 4 + [
+            _u8p, _f32p, _f64p]
+        L.oracle_moe_decode_a8.argtypes = ([ctypes.c_int] * 5 + [_u16p, _f32p] + [_u8pp] * 4 + [_u8p] * 4 +
+                                           [_u8p, _f32p, _f64p, _i32p, _f64p, _f64p])
         L.oracle_lm_quantize.argtypes = [ctypes.c_int, ctypes.c_int, _u16p, _u8p, _f32p]
         L.oracle_lm_head.argtypes = [ctypes.c_int] * 3 + [_u8p, _f32p, _u16p, _f64p]
         _lib = L
@@ -205,6 +210,47 @@ def moe_decode_shared(x_bits, router_w, w13c, w13s, w2c, w2s, shared, H, I, E, k
     _check(lib().oracle_moe_decode_shared(
         H, I, E, k, M, _p(x, _u16p), _p(wr, _f32p), *[p[0] for p in ptrs], *[_p(a, _u8p) for a in sh],
         _p(out["q"], _u8p), _p(out["s"], _f32p), _p(out["logits"], _f64p), _p(out["ids"], _i32p), _p(out["weights"], _f64p), _p(out["y64"], _f64p)), "moe_decode_shared")
+    return out
+
+
+def quantize_f32(v):
+    """A1 rule on one fp32 vector: (codes uint8 [n], scale float)."""
+    a = np.ascontiguousarray(v, dtype=np.float32)
+    q = np.zeros(a.shape[0], np.uint8)
+    s = np.zeros(1, np.float32)
+    _check(lib().oracle_quantize_f32(a.shape[0], _p(a, _f32p), _p(q, _u8p), _p(s, _f32p)), "quantize_f32")
+    return q, float(s[0])
+
+
+def expert_a8(q_m, s_m, w13c, w13s, w2c, w2s, H, I):
+    """A5-A7 with the FP8 intermediate: returns (hq [I] uint8, hs, d [H])."""
+    q = np.ascontiguousarray(q_m, dtype=np.uint8)
+    arrs = [np.ascontiguousarray(a, dtype=np.uint8) for a in (w13c, w13s, w2c, w2s)]
+    hq = np.zeros(I, np.uint8)
+    hs = np.zeros(1, np.float32)
+    d = np.zeros(H, np.float64)
+    _check(lib().oracle_expert_a8(H, I, _p(q, _u8p), float(s_m), *[_p(a, _u8p) for a in arrs],
+                                  _p(hq, _u8p), _p(hs, _f32p), _p(d, _f64p)), "expert_a8")
+    return hq, float(hs[0]), d
+
+
+def moe_decode_a8(x_bits, router_w, w13c, w13s, w2c, w2s, H, I, E, k, shared=None):
+    """A1-A8 with the FP8 intermediate for every expert; shared = (w13c,
+    w13s, w2c, w2s) of one shared expert or None. Returns dict with q, s,
+    logits, ids, weights, y64."""
+    x = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    wr = np.ascontiguousarray(router_w, dtype=np.float32)
+    M = x.shape[0]
+    ptrs = [_expert_ptrs(t, E) for t in (w13c, w13s, w2c, w2s)]
+    sh = [np.ascontiguousarray(a, dtype=np.uint8) for a in shared] if shared is not None else None
+    shp = [_p(a, _u8p) for a in sh] if sh is not None else [_u8p()] * 4
+    out = dict(q=np.zeros((M, H), np.uint8), s=np.zeros(M, np.float32),
+               logits=np.zeros((M, E), np.float64), ids=np.zeros((M, k), np.int32),
+               weights=np.zeros((M, k), np.float64), y64=np.zeros((M, H), np.float64))
+    _check(lib().oracle_moe_decode_a8(
+        H, I, E, k, M, _p(x, _u16p), _p(wr, _f32p), *[p[0] for p in ptrs], *shp,
+        _p(out["q"], _u8p), _p(out["s"], _f32p), _p(out["logits"], _f64p), _p(out["ids"], _i32p),
+        _p(out["weights"], _f64p), _p(out["y64"], _f64p)), "moe_decode_a8")
     return out
 
 

@@ -322,6 +322,105 @@ int oracle_moe_decode_shared(int H, int I, int E, int k, int M,
   return 0;
 }
 
+// The A1 steps of oracle_quantize, on fp32 input.
+int oracle_quantize_f32(int n, const float* v, uint8_t* q, float* s) {
+  if (n <= 0 || !v || !q || !s) return -1;
+  float amax = 0.0f;
+  for (int i = 0; i < n; ++i) amax = std::max(amax, std::fabs(v[i]));
+  if (amax == 0.0f) {
+    for (int i = 0; i < n; ++i) q[i] = 0;
+    *s = 1.0f;
+    return 0;
+  }
+  volatile float inv = 448.0f / amax;  // fp32 division, round to nearest even
+  for (int i = 0; i < n; ++i) {
+    volatile float t = v[i] * inv;  // fp32 multiply
+    q[i] = (uint8_t)oracle_e4m3_encode(t);
+  }
+  volatile float sm = amax / 448.0f;
+  *s = sm;
+  return 0;
+}
+
+// h in fp64 from oracle_expert, rounded to fp32, quantised; then the down
+// projection of the dequantised codes in fp64.
+int oracle_expert_a8(int H, int I, const uint8_t* q_m, float s_m,
+                     const uint8_t* w13_codes, const uint8_t* w13_scales,
+                     const uint8_t* w2_codes, const uint8_t* w2_scales,
+                     uint8_t* hq_out, float* hs_out, double* d_out) {
+  if (!d_out || H <= 0 || I <= 0) return -1;
+  std::vector<double> h(I), dtmp(H);
+  int rc = oracle_expert(H, I, q_m, s_m, w13_codes, w13_scales, w2_codes, w2_scales, h.data(), dtmp.data());
+  if (rc) return rc;
+  std::vector<float> hf(I);
+  for (int n = 0; n < I; ++n) hf[n] = (float)h[n];
+  std::vector<uint8_t> hq(I);
+  float hs = 1.0f;
+  rc = oracle_quantize_f32(I, hf.data(), hq.data(), &hs);
+  if (rc) return rc;
+  std::vector<double> hd(I);
+  for (int n = 0; n < I; ++n) hd[n] = oracle_e4m3_value(hq[n]);
+  for (int r = 0; r < H; ++r) {
+    const uint8_t* dc = w2_codes + (size_t)r * (I / 2);
+    const uint8_t* ds = w2_scales + (size_t)r * (I / 32);
+    double acc = 0.0;
+    for (int n = 0; n < I; ++n) acc += mx_element(dc, ds, n) * hd[n];
+    d_out[r] = (double)hs * acc;
+  }
+  if (hq_out) std::copy(hq.begin(), hq.end(), hq_out);
+  if (hs_out) *hs_out = hs;
+  return 0;
+}
+
+// A1-A4 as in oracle_moe_decode, then every expert through oracle_expert_a8;
+// y = sum_slot w * d (+ the shared expert's d with weight 1).
+int oracle_moe_decode_a8(int H, int I, int E, int k, int M,
+                         const uint16_t* x, const float* router_w,
+                         const uint8_t* const* w13_codes, const uint8_t* const* w13_scales,
+                         const uint8_t* const* w2_codes, const uint8_t* const* w2_scales,
+                         const uint8_t* sh_w13_codes, const uint8_t* sh_w13_scales,
+                         const uint8_t* sh_w2_codes, const uint8_t* sh_w2_scales,
+                         uint8_t* q, float* s, double* logits, int32_t* ids, double* weights,
+                         double* y64) {
+  if (H <= 0 || I <= 0 || E <= 0 || k <= 0 || k > E || M < 0 || !y64) return -1;
+  const bool shared = sh_w13_codes || sh_w13_scales || sh_w2_codes || sh_w2_scales;
+  if (shared && !(sh_w13_codes && sh_w13_scales && sh_w2_codes && sh_w2_scales)) return -1;
+  std::vector<uint8_t> qv((size_t)M * H);
+  std::vector<float> sv(M);
+  std::vector<double> lv((size_t)M * E), wv((size_t)M * k), d(H);
+  std::vector<int32_t> iv((size_t)M * k);
+  int rc = oracle_quantize(M, H, x, qv.data(), sv.data());
+  if (rc) return rc;
+  rc = oracle_router_logits(M, H, E, x, router_w, lv.data());
+  if (rc) return rc;
+  rc = oracle_topk(M, E, k, lv.data(), iv.data(), wv.data());
+  if (rc) return rc;
+  for (int m = 0; m < M; ++m) {
+    const uint8_t* qm = qv.data() + (size_t)m * H;
+    for (int r = 0; r < H; ++r) y64[(size_t)m * H + r] = 0.0;
+    for (int j = 0; j < k; ++j) {
+      const int e = iv[(size_t)m * k + j];
+      rc = oracle_expert_a8(H, I, qm, sv[m], w13_codes[e], w13_scales[e], w2_codes[e], w2_scales[e], nullptr,
+                            nullptr, d.data());
+      if (rc) return rc;
+      const double w = wv[(size_t)m * k + j];
+      for (int r = 0; r < H; ++r) y64[(size_t)m * H + r] += w * d[r];
+    }
+    if (shared) {
+      rc = oracle_expert_a8(H, I, qm, sv[m], sh_w13_codes, sh_w13_scales, sh_w2_codes, sh_w2_scales, nullptr,
+                            nullptr, d.data());
+      if (rc) return rc;
+      for (int r = 0; r < H; ++r) y64[(size_t)m * H + r] += d[r];
+    }
+  }
+  if (q) std::copy(qv.begin(), qv.end(), q);
+  if (s) std::copy(sv.begin(), sv.end(), s);
+  if (logits) std::copy(lv.begin(), lv.end(), logits);
+  if (ids) std::copy(iv.begin(), iv.end(), ids);
+  if (weights) std::copy(wv.begin(), wv.end(), weights);
+  return 0;
+}
+
 // Brute force over all E experts: expert e is kept for token m when fewer
 // than k experts rank above it (higher logit, or equal logit and lower index);
 // the kept experts' weights are exp(l_e - max) renormalised over the kept set.

@@ -104,6 +104,33 @@ int oracle_moe_decode_shared(int H, int I, int E, int k, int M,
                              const uint8_t* sh_w2_codes, const uint8_t* sh_w2_scales,
                              uint8_t* q, float* s, double* logits, int32_t* ids, double* weights,
                              double* y64);
+/* The A1 rule on fp32 values (the FP8 intermediate below): amax = max|v|,
+ * inv = fl32(448/amax), code = E4M3_RNE_sat(fl32(v*inv)), s = fl32(amax/448);
+ * amax == 0 gives zero codes and s = 1. One vector of n values. */
+int oracle_quantize_f32(int n, const float* v, uint8_t* q, float* s);
+
+/* A5-A7 with an FP8 intermediate (a true A8 down projection: "W4A8",
+ * section "Why is MoE decoding on DGX Spark memory-bound?" of the DGX Spark
+ * MoE page). Reading: the SwiGLU output h of the pair, computed as in
+ * oracle_expert and rounded to fp32, is quantised by oracle_quantize_f32
+ * over its I elements; d = s_h * W2 . E4M3(hq) in fp64. hq_out [I] and
+ * hs_out may be NULL. */
+int oracle_expert_a8(int H, int I, const uint8_t* q_m, float s_m,
+                     const uint8_t* w13_codes, const uint8_t* w13_scales,
+                     const uint8_t* w2_codes, const uint8_t* w2_scales,
+                     uint8_t* hq_out, float* hs_out, double* d_out);
+
+/* A1-A8 with the FP8 intermediate for every expert, and optionally one
+ * shared expert (sh_* all NULL for none; otherwise as in
+ * oracle_moe_decode_shared). Outputs as oracle_moe_decode_shared. */
+int oracle_moe_decode_a8(int H, int I, int E, int k, int M,
+                         const uint16_t* x, const float* router_w,
+                         const uint8_t* const* w13_codes, const uint8_t* const* w13_scales,
+                         const uint8_t* const* w2_codes, const uint8_t* const* w2_scales,
+                         const uint8_t* sh_w13_codes, const uint8_t* sh_w13_scales,
+                         const uint8_t* sh_w2_codes, const uint8_t* sh_w2_scales,
+                         uint8_t* q, float* s, double* logits, int32_t* ids, double* weights,
+                         double* y64);
 /* Brute force: every expert for every token, masked by a rank-count top-k
  * and weighted by a softmax renormalised over the kept experts. */
 int oracle_moe_dense(int H, int I, int E, int k, int M,

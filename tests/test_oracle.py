@@ -471,3 +471,88 @@ def test_lm_head_linear_and_homogeneous(oracle_mod):
     assert np.allclose(la + lb, lx, rtol=1e-12, atol=1e-9)
     l2 = oracle_mod.lm_head(codes, scales, bf16_bits(x * 2))
     assert np.array_equal(l2, 2 * lx)
+
+
+# ------------------------------------------------- FP8 intermediate (A8 down)
+def _mx_decode_np(codes: np.ndarray, scales: np.ndarray, K: int) -> np.ndarray:
+    """Dequantise packed MXFP4 rows [R][K/2] + [R][K/32] with numpy and the
+    OCP E2M1 table fixture (low nibble = even element)."""
+    table = np.zeros(16, np.float64)
+    for code, val in read_golden("e2m1_values.txt"):
+        table[int(code)] = float(val)
+    c = np.asarray(codes, np.uint8).reshape(-1, K // 2)
+    el = np.empty((c.shape[0], K), np.float64)
+    el[:, 0::2] = table[c & 0xF]
+    el[:, 1::2] = table[c >> 4]
+    sc = 2.0 ** (np.asarray(scales, np.float64).reshape(-1, K // 32) - 127.0)
+    return el * np.repeat(sc, 32, axis=1)
+
+
+def test_quantize_f32_hand_and_torch(oracle_mod):
+    q, s = oracle_mod.quantize_f32(np.array([1.0, 2.0, 3.0, 4.0], np.float32))
+    assert q.tolist() == [0x6E, 0x76, 0x7A, 0x7E] and s == np.float32(4.0) / np.float32(448.0)
+    q, s = oracle_mod.quantize_f32(np.zeros(5, np.float32))
+    assert not q.any() and s == 1.0
+    g = torch.Generator().manual_seed(11)
+    for scale in (1e-6, 0.03, 1.0, 700.0):
+        v = (torch.randn(300, generator=g) * scale).float()
+        v[7] = 0.0
+        v[9] = v[10] * 1e-4  # deep in the subnormal range after scaling
+        q, s = oracle_mod.quantize_f32(v.numpy())
+        amax = v.abs().max()
+        inv = torch.tensor(448.0, dtype=torch.float32) / amax
+        ref = torch.clamp(v * inv, -448.0, 448.0).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+        assert np.array_equal(q, ref), scale
+        assert s == (amax / torch.tensor(448.0)).item()
+
+
+def test_expert_a8_is_the_dequantised_down_projection(oracle_mod):
+    # The A8 expert = SwiGLU output h (fp64 from the plain expert, rounded to
+    # fp32), quantised by torch's float8 conversion, then W2 (dequantised by
+    # numpy from the MX table) times the dequantised h in fp64.
+    H, I = 256, 64
+    x = synth.gen_x(12, 2, H)
+    q, s = oracle_mod.quantize(bf16_bits(x))
+    ex = synth.expert_np(12, 0, 3, H, I)
+    w2 = _mx_decode_np(ex[2], ex[3], I)  # [H][I]
+    for m in range(2):
+        h, _ = oracle_mod.expert(q[m], s[m], *ex, H, I)
+        hq, hs, d = oracle_mod.expert_a8(q[m], s[m], *ex, H, I)
+        h32 = torch.from_numpy(h.astype(np.float32))
+        amax = h32.abs().max()
+        inv = torch.tensor(448.0, dtype=torch.float32) / amax
+        ref = torch.clamp(h32 * inv, -448.0, 448.0).to(torch.float8_e4m3fn)
+        assert np.array_equal(hq, ref.view(torch.uint8).numpy())
+        assert hs == (amax / torch.tensor(448.0)).item()
+        hd = ref.to(torch.float64).numpy() * hs
+        want = w2 @ hd
+        assert np.all(np.abs(d - want) <= 1e-12 * np.abs(w2) @ np.abs(hd))
+        # E4M3 rounding bound on every element, and the largest maps to 448
+        err = np.abs(hd - h.astype(np.float32).astype(np.float64))
+        assert np.all(err <= 2.0 ** -4 * np.abs(h) * (1 + 1e-6) + hs * 2.0 ** -10)
+        assert hq[int(np.argmax(np.abs(h)))] & 0x7F == 0x7E
+
+
+def test_moe_decode_a8_invariants(oracle_mod):
+    H, I, E, k, M = 256, 64, 16, 4, 3
+    x, wr, per = _tiny_layer(M=M, k=k, mode="gap")
+    plain = oracle_mod.moe_decode(x, wr, *per, H, I, E, k)
+    a8 = oracle_mod.moe_decode_a8(x, wr, *per, H, I, E, k)
+    for key in ("q", "s", "logits", "ids", "weights"):
+        assert np.array_equal(a8[key], plain[key])
+    # quantising h moves y by a few percent of its norm: visible, not larger
+    rel = np.linalg.norm(a8["y64"] - plain["y64"]) / np.linalg.norm(plain["y64"])
+    assert 2e-3 < rel < 0.1, rel
+    # zero down codes give zero; +1 on every down scale doubles y exactly
+    z2 = [np.zeros_like(a) for a in per[2]]
+    assert not oracle_mod.moe_decode_a8(x, wr, per[0], per[1], z2, per[3], H, I, E, k)["y64"].any()
+    s2 = [a + 1 for a in per[3]]
+    dbl = oracle_mod.moe_decode_a8(x, wr, per[0], per[1], per[2], s2, H, I, E, k)["y64"]
+    assert np.array_equal(dbl, 2 * a8["y64"])
+    # the shared expert adds its own A8 output with weight 1
+    sh = _shared_expert()
+    withsh = oracle_mod.moe_decode_a8(x, wr, *per, H, I, E, k, shared=sh)["y64"]
+    qv, sv = oracle_mod.quantize(x)
+    for m in range(M):
+        _, _, d = oracle_mod.expert_a8(qv[m], sv[m], *sh, H, I)
+        assert np.all(np.abs(withsh[m] - a8["y64"][m] - d) <= 1e-13 * (np.abs(a8["y64"][m]) + np.abs(d)))
