@@ -215,6 +215,7 @@ def run_ours(args):
     M = args.tokens
     L = args.layers
     flags = moe.MOE_FLAG_SPLIT_KERNELS if args.variant == "split" else 0
+    flags |= moe.MOE_FLAG_FP8_INTERMEDIATE if args.fp8_intermediate else 0
     x, ctxs, _weights = build_pool(device, M, args.routing, layers=L, flags=flags, stack=args.stack,
                                    shared=args.shared_expert)
     n_shared = int(args.shared_expert)
@@ -286,13 +287,15 @@ def run_ours(args):
     achieved = alg / (us_per_layer * 1e-6) / 1e9
     workload = (f"ling_stack{L}_rmsnorm_M{M}" if args.stack else f"ling_layer_M{M}_{args.routing}")
     workload += "_shared1" if n_shared else ""
+    workload += "_a8" if args.fp8_intermediate else ""
     traffic = recorded_traffic("k_fused", workload)
 
     # ---- end to end through the public API with host buffers
     e2e = run_e2e(args, ctxs, x, device, M, L, stack=args.stack)
 
     # ---- CPU oracle baseline (rank 0 only)
-    cpu = run_cpu_baseline(args, M, shared=args.shared_expert) if rank == 0 and not args.no_cpu else None
+    cpu = (run_cpu_baseline(args, M, shared=args.shared_expert, a8=args.fp8_intermediate)
+           if rank == 0 and not args.no_cpu else None)
 
     launches = layer_steps * (3 if info["variant"] == "split" else 1)
     line = {
@@ -301,7 +304,8 @@ def run_ours(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp8e4m3 x mxfp4 (f16/fp32 accumulate)",
         "data": "synthetic (seeded SplitMix64; random MXFP4 weights, N(0,1) bf16 activations)",
         "config": {"workload": workload, "hidden": H, "inter": I, "num_experts": E, "top_k": K, "tokens": M,
-                   "routing": args.routing, "shared_experts": n_shared, "layers_in_pool": L,
+                   "routing": args.routing, "shared_experts": n_shared,
+                   "fp8_intermediate": bool(args.fp8_intermediate), "layers_in_pool": L,
                    "pool_weight_bytes": L * (E + n_shared) * expert_bytes(),
                    "l2": "inputs larger than L2: each layer-step reads a different layer of the pool",
                    "step": (f"{L}-layer stack (RMSNorm between layers) in one CUDA graph" if args.stack
@@ -389,20 +393,22 @@ def cpu_sample_steps(M, n_layers, seed=SEED, shared=False):
     return xb, steps
 
 
-def oracle_step(xb, step):
+def oracle_step(xb, step, a8=False):
     import oracle
     wr, per, sh = step
+    if a8:
+        return oracle.moe_decode_a8(xb, wr, *per, H, I, E, K, shared=sh)
     if sh is None:
         return oracle.moe_decode(xb, wr, *per, H, I, E, K)
     return oracle.moe_decode_shared(xb, wr, *per, sh, H, I, E, K)
 
 
-def run_cpu_baseline(args, M, n_layers=None, shared=False):
+def run_cpu_baseline(args, M, n_layers=None, shared=False, a8=False):
     n_layers = n_layers or args.cpu_layers
     xb, steps = cpu_sample_steps(M, n_layers, shared=shared)
     t0 = time.perf_counter()
     for st in steps:
-        oracle_step(xb, st)
+        oracle_step(xb, st, a8)
     dt = time.perf_counter() - t0
     return {"value": round(M * n_layers / dt, 3), "unit": "tokens/s", "cores": 1, "kind": "oracle",
             "sample": f"{n_layers} layer-steps of the same workload (M={M}, distinct pool layers), "
@@ -417,17 +423,18 @@ def run_reference(args):
     n = max(1, args.ref_layers)
     xb, steps = cpu_sample_steps(M, n, shared=args.shared_expert)
     for _ in range(min(args.warmup, 1)):
-        oracle_step(xb, steps[0])
+        oracle_step(xb, steps[0], args.fp8_intermediate)
     t0 = time.perf_counter()
     for s in range(args.steps):
-        oracle_step(xb, steps[s % n])
+        oracle_step(xb, steps[s % n], args.fp8_intermediate)
     dt = time.perf_counter() - t0
     value = M * args.steps / dt
     line = {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s",
             "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(dt * 1e3 / args.steps, 3), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": f"ling_layer_M{M}_{args.routing}" + ("_shared1" if args.shared_expert else ""),
+            "config": {"workload": f"ling_layer_M{M}_{args.routing}" + ("_shared1" if args.shared_expert else "")
+                       + ("_a8" if args.fp8_intermediate else ""),
                        "hidden": H, "inter": I, "num_experts": E, "top_k": K, "tokens": M,
                        "shared_experts": int(args.shared_expert),
                        "step": "one layer-step of the CPU oracle on host cores"},
@@ -559,6 +566,8 @@ def main():
     ap.add_argument("--variant", choices=["fused", "split"], default="fused")
     ap.add_argument("--shared-expert", action="store_true",
                     help="one always-active shared expert per layer besides the top-8 routed ones")
+    ap.add_argument("--fp8-intermediate", action="store_true",
+                    help="quantise the SwiGLU output to E4M3 per (token, expert) before the down projection")
     ap.add_argument("--stack", action="store_true",
                     help="chain the pool as a stack: layer l+1 takes RMSNorm(y_l)")
     ap.add_argument("--op", choices=["moe", "lm_head"], default="moe",

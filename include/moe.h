@@ -86,6 +86,24 @@ typedef enum {
                                        Persistent kernel only: with
                                        MOE_FLAG_SPLIT_KERNELS, moe_create
                                        returns MOE_ERR_UNSUPPORTED */
+#define MOE_FLAG_FP8_INTERMEDIATE 0x8u /* FP8 input to the down projection too
+                                       (W4A8 on the same page, section "Why
+                                       is MoE decoding on DGX Spark
+                                       memory-bound?", read as 8-bit inputs
+                                       for both projections): the SwiGLU
+                                       output h of each (token, expert) pair
+                                       is quantised like the activations,
+                                       over its I elements: amax = max|h|,
+                                       inv = fl32(448/amax), code =
+                                       E4M3_RNE_sat(fl32(h*inv)), scale
+                                       fl32(amax/448) (amax == 0: zero codes,
+                                       scale 1); the down projection uses
+                                       scale * E4M3(code). h itself is fp32
+                                       SwiGLU of fp32 sums, so a code can
+                                       differ from one computed from exact h
+                                       where h*inv lies at a rounding
+                                       boundary. Persistent kernel only, as
+                                       MOE_FLAG_SHARED_EXPERT */
 
 typedef struct {
   int32_t hidden;      /* H: multiple of 32, 32..8192                        */
@@ -179,7 +197,8 @@ moe_status moe_debug_set_wait(moe_ctx* ctx, long long budget_cycles, int force_s
  * It computes what moe_decode computes, with the three-kernel form of the
  * step (the MOE_FLAG_SPLIT_KERNELS path). There is no context. The layer's
  * shapes come from cfg (max_tokens and device are ignored; of the flags,
- * MOE_FLAG_SHARED_EXPERT and MOE_FLAG_PRE_RMSNORM return MOE_ERR_UNSUPPORTED
+ * MOE_FLAG_SHARED_EXPERT, MOE_FLAG_PRE_RMSNORM and MOE_FLAG_FP8_INTERMEDIATE
+ * return MOE_ERR_UNSUPPORTED
  * and MOE_FLAG_SPLIT_KERNELS is ignored), and the
  * weights, x and y are passed in directly with the layouts, alignment and
  * optional outputs of moe_load_experts and moe_decode. The scale bytes are not

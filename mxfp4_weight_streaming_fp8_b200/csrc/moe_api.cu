@@ -32,9 +32,9 @@ moe_status validate_config(const moe_config& c) {
   if (c.num_experts < 1 || c.num_experts > moe::kMaxExperts) return MOE_ERR_INVALID_ARG;
   if (c.top_k < 1 || c.top_k > c.num_experts || c.top_k > moe::kMaxTopK) return MOE_ERR_INVALID_ARG;
   if (c.max_tokens < 1 || c.max_tokens > moe::kMaxTokens) return MOE_ERR_INVALID_ARG;
-  if (c.flags & ~(MOE_FLAG_SPLIT_KERNELS | MOE_FLAG_PRE_RMSNORM | MOE_FLAG_SHARED_EXPERT)) return MOE_ERR_INVALID_ARG;
-  if ((c.flags & (MOE_FLAG_PRE_RMSNORM | MOE_FLAG_SHARED_EXPERT)) && (c.flags & MOE_FLAG_SPLIT_KERNELS))
-    return MOE_ERR_UNSUPPORTED;
+  const uint32_t fused_only = MOE_FLAG_PRE_RMSNORM | MOE_FLAG_SHARED_EXPERT | MOE_FLAG_FP8_INTERMEDIATE;
+  if (c.flags & ~(MOE_FLAG_SPLIT_KERNELS | fused_only)) return MOE_ERR_INVALID_ARG;
+  if ((c.flags & fused_only) && (c.flags & MOE_FLAG_SPLIT_KERNELS)) return MOE_ERR_UNSUPPORTED;
   return MOE_OK;
 }
 
@@ -187,7 +187,11 @@ moe_status moe_create(const moe_config* cfg, moe_ctx** out) {
   ctx->sm_count = prop.multiProcessorCount;
   ctx->variant = (c.flags & MOE_FLAG_SPLIT_KERNELS) ? kSplit : kFused;
   ctx->spin_limit = kDefaultSpinLimit;
-  ctx->fused = (c.flags & MOE_FLAG_SHARED_EXPERT) ? moe::k_fused<true> : moe::k_fused<false>;
+  {
+    const bool sh = (c.flags & MOE_FLAG_SHARED_EXPERT) != 0, f8 = (c.flags & MOE_FLAG_FP8_INTERMEDIATE) != 0;
+    ctx->fused = sh ? (f8 ? moe::k_fused<true, true> : moe::k_fused<true, false>)
+                    : (f8 ? moe::k_fused<false, true> : moe::k_fused<false, false>);
+  }
 
   // workspace layout
   const size_t H = c.hidden, I = c.inter, E = c.num_experts, K = c.top_k, MM = c.max_tokens;
@@ -440,11 +444,12 @@ moe_status moe_query(const moe_ctx* ctx, char* buf, size_t len) {
                  "{\"lib\": \"libmoe\", \"arch\": \"sm_100a\", \"device\": %d, \"sm_count\": %d, "
                  "\"variant\": \"fused\", \"kernels\": [\"k_fused\"], \"grid\": [%d], \"threads\": %d, "
                  "\"smem\": %d, \"ring_gu\": [%d, %d], \"ring_d\": [%d, %d], \"pdl\": true, \"pre_rmsnorm\": %s, "
-                 "\"shared_expert\": %s, "
+                 "\"shared_expert\": %s, \"fp8_intermediate\": %s, "
                  "\"hidden\": %d, \"inter\": %d, \"num_experts\": %d, \"top_k\": %d, \"max_tokens\": %d}",
                  ctx->dev, ctx->sm_count, pl.G, moe::kFusedThreads, pl.smem_bytes, pl.ns_gu, pl.slot_gu, pl.ns_d,
                  pl.slot_d, (c.flags & MOE_FLAG_PRE_RMSNORM) ? "true" : "false",
-                 (c.flags & MOE_FLAG_SHARED_EXPERT) ? "true" : "false", c.hidden, c.inter, c.num_experts,
+                 (c.flags & MOE_FLAG_SHARED_EXPERT) ? "true" : "false",
+                 (c.flags & MOE_FLAG_FP8_INTERMEDIATE) ? "true" : "false", c.hidden, c.inter, c.num_experts,
                  c.top_k, c.max_tokens);
   }
   if (n < 0 || (size_t)n >= len) return MOE_ERR_INVALID_ARG;

@@ -457,9 +457,25 @@ __device__ __forceinline__ int h_rescale_exp(float mx) {
   return min(126, 9 - ex);
 }
 
+// FP8 intermediate (kFp8H): h of a pair is quantised like the activations
+// before the down projection (the W4A8 recipe on "NVIDIA Shows 3 Ways to
+// Speed Up MoE Inference on DGX Spark", section "Why is MoE decoding on DGX
+// Spark memory-bound?", read as 8-bit inputs for both projections): over the
+// pair's I elements, amax = max|h|, inv = fl32(448/amax), code =
+// E4M3_RNE_sat(fl32(h*inv)), scale fl32(amax/448) (amax == 0: zero codes,
+// scale 1). The codes' values are exact in f16, so the down path's f16
+// products stay exact.
+__device__ __forceinline__ uint32_t h_fp8x2(float a, float b, float inv) {
+  return e4m3x2_to_f16x2(f32x2_to_e4m3x2(__fmul_rn(a, inv), __fmul_rn(b, inv)));
+}
+__device__ __forceinline__ float h_fp8_inv(float amax) { return amax > 0.f ? __fdiv_rn(448.f, amax) : 0.f; }
+__device__ __forceinline__ float h_fp8_scale(float amax) { return amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f; }
+
 // Stage h of the pairs [pb, pe) of one expert (pe - pb <= kHPairs) into
 // shared memory as f16, each pair vector rescaled by 2^t, with 2^-t kept in
-// hscale. One warp; h is read from L2 (written by other CTAs).
+// hscale (kFp8H: as E4M3 values, with the pair's FP8 scale in hscale). One
+// warp; h is read from L2 (written by other CTAs).
+template <bool kFp8H>
 __device__ __forceinline__ void stage_h(const Params& p, int pb, int pe, __half2* hbuf, float* hscale) {
   const int lane = threadIdx.x & 31;
   const int I = p.I;
@@ -480,17 +496,31 @@ __device__ __forceinline__ void stage_h(const Params& p, int pb, int pe, __half2
       for (int k = 0; k < kQ; ++k)
         mx = fmaxf(mx, fmaxf(fmaxf(fabsf(__uint_as_float(v[k].x)), fabsf(__uint_as_float(v[k].y))),
                              fmaxf(fabsf(__uint_as_float(v[k].z)), fabsf(__uint_as_float(v[k].w)))));
-      const int t = h_rescale_exp(warp_max(mx));
-      const float up = ldexpf(1.f, t);
+      if constexpr (kFp8H) {
+        const float amax = warp_max(mx), inv = h_fp8_inv(amax);
 #pragma unroll
-      for (int k = 0; k < kQ; ++k) {
-        const int q = lane + 32 * k;
-        if (q < I / 4) {
-          dst[2 * q] = __floats2half2_rn(__uint_as_float(v[k].x) * up, __uint_as_float(v[k].y) * up);
-          dst[2 * q + 1] = __floats2half2_rn(__uint_as_float(v[k].z) * up, __uint_as_float(v[k].w) * up);
+        for (int k = 0; k < kQ; ++k) {
+          const int q = lane + 32 * k;
+          if (q < I / 4) {
+            uint32_t* d32 = reinterpret_cast<uint32_t*>(dst + 2 * q);
+            d32[0] = h_fp8x2(__uint_as_float(v[k].x), __uint_as_float(v[k].y), inv);
+            d32[1] = h_fp8x2(__uint_as_float(v[k].z), __uint_as_float(v[k].w), inv);
+          }
         }
+        if (lane == 0) hscale[j] = h_fp8_scale(amax);
+      } else {
+        const int t = h_rescale_exp(warp_max(mx));
+        const float up = ldexpf(1.f, t);
+#pragma unroll
+        for (int k = 0; k < kQ; ++k) {
+          const int q = lane + 32 * k;
+          if (q < I / 4) {
+            dst[2 * q] = __floats2half2_rn(__uint_as_float(v[k].x) * up, __uint_as_float(v[k].y) * up);
+            dst[2 * q + 1] = __floats2half2_rn(__uint_as_float(v[k].z) * up, __uint_as_float(v[k].w) * up);
+          }
+        }
+        if (lane == 0) hscale[j] = ldexpf(1.f, -t);
       }
-      if (lane == 0) hscale[j] = ldexpf(1.f, -t);
     } else {
       // wide intermediate: one pass for the max, one to convert
       float mx = 0.f;
@@ -499,14 +529,25 @@ __device__ __forceinline__ void stage_h(const Params& p, int pb, int pe, __half2
         mx = fmaxf(mx, fmaxf(fmaxf(fabsf(__uint_as_float(v.x)), fabsf(__uint_as_float(v.y))),
                              fmaxf(fabsf(__uint_as_float(v.z)), fabsf(__uint_as_float(v.w)))));
       }
-      const int t = h_rescale_exp(warp_max(mx));
-      const float up = ldexpf(1.f, t);
-      for (int q = lane; q < I / 4; q += 32) {
-        const uint4 v = ld_cg_u4(hp + q);
-        dst[2 * q] = __floats2half2_rn(__uint_as_float(v.x) * up, __uint_as_float(v.y) * up);
-        dst[2 * q + 1] = __floats2half2_rn(__uint_as_float(v.z) * up, __uint_as_float(v.w) * up);
+      if constexpr (kFp8H) {
+        const float amax = warp_max(mx), inv = h_fp8_inv(amax);
+        for (int q = lane; q < I / 4; q += 32) {
+          const uint4 v = ld_cg_u4(hp + q);
+          uint32_t* d32 = reinterpret_cast<uint32_t*>(dst + 2 * q);
+          d32[0] = h_fp8x2(__uint_as_float(v.x), __uint_as_float(v.y), inv);
+          d32[1] = h_fp8x2(__uint_as_float(v.z), __uint_as_float(v.w), inv);
+        }
+        if (lane == 0) hscale[j] = h_fp8_scale(amax);
+      } else {
+        const int t = h_rescale_exp(warp_max(mx));
+        const float up = ldexpf(1.f, t);
+        for (int q = lane; q < I / 4; q += 32) {
+          const uint4 v = ld_cg_u4(hp + q);
+          dst[2 * q] = __floats2half2_rn(__uint_as_float(v.x) * up, __uint_as_float(v.y) * up);
+          dst[2 * q + 1] = __floats2half2_rn(__uint_as_float(v.z) * up, __uint_as_float(v.w) * up);
+        }
+        if (lane == 0) hscale[j] = ldexpf(1.f, -t);
       }
-      if (lane == 0) hscale[j] = ldexpf(1.f, -t);
     }
   }
 }
@@ -558,7 +599,8 @@ __device__ __forceinline__ void d_rows(const Params& p, const DChunk& ch, int a,
 
 // Down item: rows [a, a+cnt) for every pair of the expert; h from the staged
 // shared-memory copy when the expert has at most `hpairs` pairs, else read
-// and rescaled here from L2.
+// and rescaled (kFp8H: quantised) here from L2.
+template <bool kFp8H>
 __device__ __forceinline__ void d_item(const Params& p, const DChunk& ch, int a, int cnt, int pb, int pe,
                                        const __half2* hbuf, const float* hscale, int hpairs, float* dsm, int rpc) {
   const int lane = threadIdx.x & 31;
@@ -598,13 +640,20 @@ __device__ __forceinline__ void d_item(const Params& p, const DChunk& ch, int a,
               for (int t = 0; t < 32; ++t) mx = fmaxf(mx, fabsf(__ldcg(hp + bk * 32 + t)));
           }
         }
-        const int t = h_rescale_exp(warp_max(mx));
-        const float up = ldexpf(1.f, t);
-        down = ldexpf(1.f, -t);
+        if constexpr (kFp8H) {
+          const float amax = warp_max(mx), inv = h_fp8_inv(amax);
+          down = h_fp8_scale(amax);
 #pragma unroll
-        for (int q = 0; q < 16; ++q) {
-          __half2 v = __floats2half2_rn(hv[2 * q] * up, hv[2 * q + 1] * up);
-          h2[q] = *reinterpret_cast<uint32_t*>(&v);
+          for (int q = 0; q < 16; ++q) h2[q] = h_fp8x2(hv[2 * q], hv[2 * q + 1], inv);
+        } else {
+          const int t = h_rescale_exp(warp_max(mx));
+          const float up = ldexpf(1.f, t);
+          down = ldexpf(1.f, -t);
+#pragma unroll
+          for (int q = 0; q < 16; ++q) {
+            __half2 v = __floats2half2_rn(hv[2 * q] * up, hv[2 * q + 1] * up);
+            h2[q] = *reinterpret_cast<uint32_t*>(&v);
+          }
         }
       }
       d_rows(p, ch, a, cnt, blk, h2, down, dsm + (size_t)pp * rpc, b0 == 0);
@@ -707,7 +756,8 @@ __device__ __forceinline__ int union_small(const int* s_ids, int np, int K, int*
 // items are the head of the work queue. (Running them while the router
 // logits arrive measured slower: the wait for the router is shorter than an
 // item, so they lengthened routing.)
-template <bool kShared>
+// kFp8H: the FP8 intermediate (see h_fp8x2) for every expert.
+template <bool kShared, bool kFp8H>
 __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw, FusedPlan pl) {
   extern __shared__ __align__(128) unsigned char smem[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -1268,7 +1318,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
         // CTAs, then stage h once for the CTA
         if (lane == 0) grid_wait(gu_counter(fw, u), tgt, p);
         __syncwarp();
-        if (pe - pb <= pl.hpairs) stage_h(p, pb, pe, hbuf, hscale);
+        if (pe - pb <= pl.hpairs) stage_h<kFp8H>(p, pb, pe, hbuf, hscale);
         __syncwarp();
         if (lane == 0) mbar_arrive(h_bar + slot);
       } else {
@@ -1280,7 +1330,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
       unsigned sn;
       d_layout(p, s_union[u], r0, nrd, ring_d + (size_t)slot * pl.slot_d, &ch, &sa0, &sn);
       const int a = gd * kDownRowsPerItem, cnt = min(kDownRowsPerItem, nrd - a);
-      d_item(p, ch, a, cnt, pb, pe, hbuf, hscale, pl.hpairs, dsm, pl.rpc_max);
+      d_item<kFp8H>(p, ch, a, cnt, pb, pe, hbuf, hscale, pl.hpairs, dsm, pl.rpc_max);
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(empty_d + slot);

@@ -21,6 +21,7 @@ STATUS_NAMES = {
 MOE_FLAG_SPLIT_KERNELS = 0x1
 MOE_FLAG_PRE_RMSNORM = 0x2
 MOE_FLAG_SHARED_EXPERT = 0x4
+MOE_FLAG_FP8_INTERMEDIATE = 0x8
 MOE_LOAD_BORROW = 0x0
 MOE_LOAD_SKIP_VALIDATE = 0x1
 

@@ -28,10 +28,11 @@ def bits(t: torch.Tensor) -> np.ndarray:
 class Layer:
     """Seeded inputs of one MoE layer, on the device and (lazily) on the CPU."""
 
-    def __init__(self, H, I, E, K, M, seed=0, layer=0, mode="gap", device="cuda:0", shared=False):
+    def __init__(self, H, I, E, K, M, seed=0, layer=0, mode="gap", device="cuda:0", shared=False, a8=False):
         self.H, self.I, self.E, self.K, self.M = H, I, E, K, M
         self.seed, self.layer = seed, layer
         self.shared = shared  # expert E (the last of E + 1) is a shared expert
+        self.a8 = a8          # FP8 intermediate (MOE_FLAG_FP8_INTERMEDIATE)
         self.x = synth.gen_x(seed, M, H, layer=layer)
         self.wr = synth.force_router(self.x, synth.gen_router(seed, layer, E, H), K, mode, seed=seed,
                                      layer=layer) if M > 0 else synth.gen_router(seed, layer, E, H)
@@ -48,14 +49,19 @@ class Layer:
                 per[t][e] = parts[t]
         return per
 
-    def oracle(self, tokens=None):
-        """Oracle outputs for the given token subset (default all)."""
+    def oracle(self, tokens=None, a8=None):
+        """Oracle outputs for the given token subset (default all); a8
+        overrides the layer's FP8-intermediate setting."""
+        a8 = self.a8 if a8 is None else a8
         xb = bits(self.x)
         if tokens is not None:
             xb = xb[list(tokens)]
         logits = oracle.router_logits(xb, self.wr)
         ids, _ = oracle.topk(logits, self.K)
         per = self.expert_slices(ids)
+        if a8:
+            sh = synth.expert_np(self.seed, self.layer, self.E, self.H, self.I) if self.shared else None
+            return oracle.moe_decode_a8(xb, self.wr, *per, self.H, self.I, self.E, self.K, shared=sh)
         if self.shared:
             sh = synth.expert_np(self.seed, self.layer, self.E, self.H, self.I)
             return oracle.moe_decode_shared(xb, self.wr, *per, sh, self.H, self.I, self.E, self.K)
@@ -64,6 +70,8 @@ class Layer:
     def make_ctx(self, flags=0, max_tokens=None):
         if self.shared:
             flags |= moe.MOE_FLAG_SHARED_EXPERT
+        if self.a8:
+            flags |= moe.MOE_FLAG_FP8_INTERMEDIATE
         ctx = moe.MoELayer(self.H, self.I, self.E, self.K, max_tokens or max(1, self.M), flags=flags,
                            device=self.dev.index or 0)
         ctx.load_experts(self.wr_d, *self.experts)

@@ -119,6 +119,76 @@ def test_shared_expert_ring_reuse_sampled():
     compare(L, got, L.oracle(tokens=sample), tokens=sample)
 
 
+def _check_a8(L, got, tokens=None, discriminate=True):
+    """The step with the FP8 intermediate against its oracle: the element
+    bound used everywhere, and (discriminate) per token much closer to it
+    than to the step without: ||y - y_a8|| <= 0.5 ||y - y_plain||.
+
+    The kernel's fp32 h differs from the oracle's exact h by its f16/fp32
+    accumulation, so an element of h that lies at an E4M3 rounding boundary
+    can take the neighbouring code; both codes are correct roundings. Each
+    such flip moves y by about one E4M3 step of one h element; with I = 768
+    that is well inside both checks (a CPU emulation of the kernel's
+    accumulation gave ||y - y_a8|| = 0.0037 ||y|| against
+    ||y_a8 - y_plain|| = 0.026 ||y|| at the Ling shape). Small-I layers are
+    run only on inputs whose h keeps at least 1e-3 (relative) from every
+    boundary, where one flip of a large element could exceed the bound."""
+    t = list(range(L.M)) if tokens is None else list(tokens)
+    ref = L.oracle(tokens=tokens)
+    worst = compare(L, got, ref, tokens=tokens)
+    if discriminate:
+        plain = L.oracle(tokens=tokens, a8=False)
+        y = got["y"].float().cpu().numpy().astype(np.float64)[t]
+        for i in range(len(t)):
+            e8 = np.linalg.norm(y[i] - ref["y64"][i])
+            ep = np.linalg.norm(y[i] - plain["y64"][i])
+            assert e8 <= 0.5 * ep, (t[i], e8, ep)
+    return worst
+
+
+@pytest.mark.parametrize("shape,M,mode,shared", [((2560, 768, 256, 8), 1, "gap", False),
+                                                 ((2560, 768, 256, 8), 4, "natural", False),
+                                                 ((2560, 768, 256, 8), 6, "shared", False),
+                                                 ((2560, 768, 256, 8), 4, "natural", True)])
+def test_fp8_intermediate(shape, M, mode, shared):
+    """FP8-quantised h before the down projection, every token checked: the
+    staged-h path (entries with at most 4 pairs), the path that reads h from
+    L2 (six tokens on the same 8 experts give 6 pairs per entry), and with a
+    shared expert."""
+    H, I, E, K = shape
+    L = Layer(H, I, E, K, M, seed=31, mode=mode, shared=shared, a8=True)
+    ctx = L.make_ctx(0)
+    assert ctx.query()["fp8_intermediate"] is True
+    got = L.run(ctx)
+    worst = _check_a8(L, got)
+    print(f"A8 {shape} M={M} {mode} shared={shared}: worst y error = {worst:.3f} of the bound")
+    assert torch.equal(got["y"], L.run(ctx)["y"])
+
+
+@pytest.mark.parametrize("M,mode", [(3, "shared"), (5, "shared")])
+def test_fp8_intermediate_wide_h(M, mode):
+    """I = 1056 > 1024: h is staged (3 pairs per entry) or read from L2 (5
+    pairs) in the passes used for wide intermediates."""
+    L = Layer(512, 1056, 16, 2, M, seed=33, mode=mode, a8=True)
+    got = L.run(L.make_ctx(0))
+    _check_a8(L, got)
+
+
+def test_fp8_intermediate_tiny():
+    # seed 57: every h element keeps >= 1.19e-3 (relative) from an E4M3
+    # rounding boundary, so the codes cannot flip
+    L = Layer(256, 64, 16, 2, 1, seed=57, mode="natural", a8=True)
+    got = L.run(L.make_ctx(0))
+    _check_a8(L, got)
+
+
+def test_fp8_intermediate_m32_sampled():
+    M = 32
+    L = Layer(2560, 768, 256, 8, M, seed=32, mode="zipf", a8=True)
+    got = L.run(L.make_ctx(0, max_tokens=32))
+    _check_a8(L, got, tokens=[0, 17, 31])
+
+
 @pytest.mark.parametrize("M,mode", [(1, "gap"), (2, "zipf"), (4, "gap"), (3, "shared")])
 def test_deep_ring_reuse(M, mode):
     """A context sized for 32 tokens leaves 4 ring slots, so every slot is
