@@ -551,6 +551,46 @@ def run_lm_head(args):
     lm.close()
 
 
+def run_reference_lm_head(args):
+    """Reference arm of --op lm_head: the CPU oracle's FP8 LM head on a
+    bounded sample of rows, each step one call for M tokens, scaled to the
+    full vocabulary. The FP8 copy is made once, outside the timed steps, as
+    the library does at load."""
+    import numpy as np
+    import torch
+    import oracle
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return
+    M = args.tokens
+    rows = max(1, min(LM_V, args.ref_rows))
+    g = torch.Generator().manual_seed(SEED)
+    w = (torch.randn(rows, LM_H, generator=g) * 0.02).to(torch.bfloat16)
+    x = torch.randn(M, LM_H, generator=g).to(torch.bfloat16)
+    codes, scales = oracle.lm_quantize(w.view(torch.int16).numpy().view(np.uint16))
+    xb = x.view(torch.int16).numpy().view(np.uint16)
+    for _ in range(min(args.warmup, 1)):
+        oracle.lm_head(codes, scales, xb)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.lm_head(codes, scales, xb)
+    dt = time.perf_counter() - t0
+    per_call = dt / args.steps * LM_V / rows
+    value = M / per_call
+    line = {"impl": "reference", "metric": LM_METRIC, "value": round(value, 4), "unit": "tokens/s",
+            "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(per_call * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"lm_head_fp8_V{LM_V}_H{LM_H}_M{M}", "vocab": LM_V, "hidden": LM_H,
+                       "tokens": M, "step": "one LM head call of the CPU oracle on host cores"},
+            "cpu_baseline": {"value": round(value, 4), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                             "sample": f"{rows} of {LM_V} rows per call ({args.steps} calls, {dt:.2f} s), "
+                                       "scaled to the full matrix"},
+            "e2e": {"value": round(value, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -562,6 +602,8 @@ def main():
     ap.add_argument("--layers", type=int, default=POOL_LAYERS)
     ap.add_argument("--cpu-layers", type=int, default=16)
     ap.add_argument("--ref-layers", type=int, default=4)
+    ap.add_argument("--ref-rows", type=int, default=32768,
+                    help="LM head rows per reference (CPU oracle) call, scaled to the vocabulary")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--variant", choices=["fused", "split"], default="fused")
     ap.add_argument("--shared-expert", action="store_true",
@@ -575,7 +617,9 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
-    if args.impl == "reference":
+    if args.impl == "reference" and args.op == "lm_head":
+        run_reference_lm_head(args)
+    elif args.impl == "reference":
         run_reference(args)
     elif args.op == "lm_head":
         run_lm_head(args)
