@@ -118,6 +118,20 @@ def test_shared_expert_flag_without_gpu(L):
             assert MM * H * 2 + pl["slot_d"] <= pl["ns_d"] * pl["slot_d"]
 
 
+def test_fp8_intermediate_flag_without_gpu(L):
+    """The FP8-intermediate option changes no buffer: its plan equals the
+    plain one, alone and with a shared expert; the split path refuses it."""
+    F8, SH = moe.MOE_FLAG_FP8_INTERMEDIATE, moe.MOE_FLAG_SHARED_EXPERT
+    for shape in [(2560, 768, 256, 8, 1), (2560, 768, 256, 8, 32), (512, 1056, 16, 2, 5), (256, 64, 16, 2, 1)]:
+        for base_flags in (0, SH):
+            st0, base = moe.plan_query(*shape, flags=base_flags)
+            st, pl = moe.plan_query(*shape, flags=base_flags | F8)
+            assert st == st0 == 0 and pl == base
+    out = ctypes.c_void_p()
+    c = moe.moe_config(256, 64, 16, 2, 1, F8 | moe.MOE_FLAG_SPLIT_KERNELS, 0)
+    assert L.moe_create(ctypes.byref(c), ctypes.byref(out)) == 2 and not out.value
+
+
 def test_plan_rejects_what_does_not_fit(L):
     st, pl = moe.plan_query(8192, 4096, 1024, 32, 32)
     assert st == 2 and not pl["ok"]
