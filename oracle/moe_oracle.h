@@ -20,11 +20,16 @@
  *         Spark" (aitujian.cn copy): sections "Why is MoE decoding on DGX Spark
  *         memory-bound?" (weight streaming, W4A8 recipe), "What are the 3
  *         optimizations?" (MXFP4 MoE kernels; up to 32 experts for a 4-token
- *         verify), "What is Ling 3.0 ..." (top-8 routed experts per token).
+ *         verify; the online FP8 LM head), "What is Ling 3.0 ..." (top-8
+ *         routed experts plus one shared expert per token).
  *
  * Parity status: every function here is pinned by a CPU test (format tables,
  * a hand-derived 2-expert example, one-hot probes, brute-force dense
- * evaluation, invariants). None is "parity unpinned".
+ * evaluation, invariants; the shared-expert step by reduction to the routed
+ * step and to a single expert; the FP8-intermediate step by torch's float8
+ * conversion, numpy's dequantised down projection and the E4M3 rounding
+ * bound; the LM head by a hand row, torch's float8 conversion and one-hot
+ * columns). None is "parity unpinned".
  *
  * Layouts (row-major, K contiguous):
  *   x        bf16 bit patterns [M][H]
