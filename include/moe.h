@@ -73,8 +73,10 @@ typedef enum {
                                        moe_create returns MOE_ERR_UNSUPPORTED */
 #define MOE_FLAG_SHARED_EXPERT 0x4u /* one shared expert besides the routed ones
                                        ("NVIDIA Shows 3 Ways to Speed Up MoE
-                                       Inference on DGX Spark", Ling 3.0: 8 of
-                                       512 routed experts plus 1 shared). The
+                                       Inference on DGX Spark", section on
+                                       Ling 3.0: each token goes to its 8
+                                       routed experts and to one shared
+                                       expert). The
                                        four expert arrays hold E + 1 experts;
                                        expert E (the last) is the shared one,
                                        same shape and format, never routed

@@ -250,8 +250,12 @@ moe_status moe_create(const moe_config* cfg, moe_ctx** out) {
   // launch shapes
   ctx->grid_route = (int)(E < (size_t)ctx->sm_count ? E : (size_t)ctx->sm_count);
   ctx->smem_gateup = MM * H * 2;
-  cudaError_t err = cudaFuncSetAttribute(moe::k_gateup, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)ctx->smem_gateup);
+  // The dynamic shared-memory limit of a kernel is per device and process,
+  // not per context: every context raises it to the device's opt-in maximum
+  // (the same value each time), so creating a context with a smaller plan
+  // never lowers the limit another context's launches rely on.
+  const int smem_optin = (int)prop.sharedMemPerBlockOptin;
+  cudaError_t err = cudaFuncSetAttribute(moe::k_gateup, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_optin);
   int occ_g = 0, occ_d = 0;
   if (err == cudaSuccess)
     err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_g, moe::k_gateup, moe::kThreads, ctx->smem_gateup);
@@ -259,7 +263,7 @@ moe_status moe_create(const moe_config* cfg, moe_ctx** out) {
     err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_d, moe::k_down, moe::kThreads, 0);
   const bool plan_ok = make_plan(c, ctx->sm_count, (size_t)prop.sharedMemPerBlockOptin, &ctx->plan);
   if (err == cudaSuccess && plan_ok)
-    err = cudaFuncSetAttribute(ctx->fused, cudaFuncAttributeMaxDynamicSharedMemorySize, ctx->plan.smem_bytes);
+    err = cudaFuncSetAttribute(ctx->fused, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_optin);
   int occ_f = 0;
   if (err == cudaSuccess && plan_ok)
     err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_f, ctx->fused, moe::kFusedThreads,
@@ -395,9 +399,11 @@ moe_status moe_sync_status(moe_ctx* ctx, void* stream) {
     return MOE_ERR_CUDA;
   if (status == 0) return MOE_OK;
   // a wait gave up: clear the whole workspace (status, barrier state, epoch
-  // and every epoch-tagged word) so the next call starts clean
-  if (cudaMemset(ctx->ws_base, 0, ctx->ws_bytes) != cudaSuccess) return MOE_ERR_CUDA;
-  if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
+  // and every epoch-tagged word) on the context's stream, so the next call
+  // starts clean; only that stream is waited for
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(ctx->ws_base, 0, ctx->ws_bytes, st) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MOE_ERR_CUDA;
   return MOE_ERR_TIMEOUT;
 }
 

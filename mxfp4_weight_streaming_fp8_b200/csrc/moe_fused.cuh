@@ -1,10 +1,10 @@
 // moe_fused.cuh -- the whole decode step as one persistent kernel per layer.
 //
 // One CTA per SM (grid = SM count, 512 threads). A step is a chain of
-// dependent phases (routing -> expert gate/up -> expert down). At batch 1,
-// reading the weights sets its time ("reading model weights drove execution
-// time": MarkTechPost, "NVIDIA Shows 3 Ways to Speed Up MoE Inference on DGX
-// Spark", section "Why is MoE decoding on DGX Spark memory-bound?"). So the
+// dependent phases (routing -> expert gate/up -> expert down). At batch 1 the
+// time goes into streaming the weights from memory (MarkTechPost, "NVIDIA
+// Shows 3 Ways to Speed Up MoE Inference on DGX Spark", section "Why is MoE
+// decoding on DGX Spark memory-bound?"). So the
 // kernel is built to start the weight stream as early as possible, and to
 // leave only a short tail once the last byte arrives.
 //
@@ -748,7 +748,8 @@ __device__ __forceinline__ int union_small(const int* s_ids, int np, int K, int*
 // ---------------------------------------------------------------- the kernel
 // kShared: the weight arrays hold E + 1 experts and expert E is a shared
 // expert that every token passes with weight 1 ("NVIDIA Shows 3 Ways to Speed
-// Up MoE Inference on DGX Spark", Ling 3.0: 8 routed experts plus 1 shared).
+// Up MoE Inference on DGX Spark", section on Ling 3.0: one shared expert
+// beside the 8 routed ones).
 // It is union entry 0, with pairs 0 .. M-1 (token order); the routed entries
 // follow. It needs no routing, so its chunks are requested before routing
 // starts (by two warps that have no activation rows to scan at M=1), and the

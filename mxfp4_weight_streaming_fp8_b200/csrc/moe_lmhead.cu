@@ -417,8 +417,10 @@ moe_status moe_lm_create(int32_t vocab, int32_t hidden, int32_t max_tokens, int3
   lm->sm_count = prop.multiProcessorCount;
   if (!lm_plan(hidden, max_tokens, prop.sharedMemPerBlockOptin, &lm->ns, &lm->smem, &lm->o_bar, &lm->o_misc,
                &lm->o_x, &lm->o_part, &lm->o_ring) ||
-      cudaFuncSetAttribute(moe::k_lm_head, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lm->smem) !=
-          cudaSuccess) {
+      // the limit is per device and process: raise it to the opt-in maximum,
+      // never to this context's (possibly smaller) plan
+      cudaFuncSetAttribute(moe::k_lm_head, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)prop.sharedMemPerBlockOptin) != cudaSuccess) {
     cudaGetLastError();
     delete lm;
     return MOE_ERR_UNSUPPORTED;

@@ -91,19 +91,19 @@ static __global__ void __launch_bounds__(kThreads) k_gateup(Params p) {
   }
 }
 
-// Down + combine: one warp per output row r; for each union expert (ascending
-// id) and each of its (token, slot) pairs, d = <W2[e][r], h_pair>, and
-// y[m][r] accumulates w_pair * d in that order (deterministic, no atomics).
+// Down + combine: one warp per output row r. For each union expert and each
+// of its (token, slot) pairs, d = <W2[e][r], h_pair> is kept per (token,
+// slot); then y[m][r] sums w * d over the token's slots in slot order (the
+// order of the top-k, highest logit first), deterministic and without
+// atomics, the same order the persistent kernel uses.
 static __global__ void __launch_bounds__(kThreads) k_down(Params p) {
-  __shared__ float yacc[kWarps][kMaxTokens];
+  __shared__ float dslot[kWarps][kMaxTokens * kMaxTopK];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int H = p.H, I = p.I, nblk = I / 32;
+  const int H = p.H, I = p.I, K = p.K, nblk = I / 32;
   const int U = __ldcg(p.ws.meta);
   const int gw = blockIdx.x * kWarps + warp, GW = gridDim.x * kWarps;
   const int r0 = (int)((long long)H * gw / GW), r1 = (int)((long long)H * (gw + 1) / GW);
   for (int r = r0; r < r1; ++r) {
-    if (lane < kMaxTokens) yacc[warp][lane] = 0.f;
-    __syncwarp();
     for (int u = 0; u < U; ++u) {
       const int e = __ldcg(p.ws.union_ids + u);
       const size_t row = (size_t)e * H + r;
@@ -122,14 +122,15 @@ static __global__ void __launch_bounds__(kThreads) k_down(Params p) {
           acc = fmaf(sc, mxfp4_dot32_f32(c, hv), acc);
         }
         acc = warp_sum(acc);
-        if (lane == 0) {
-          const int m = __ldcg(p.ws.pair_tok + pp);
-          yacc[warp][m] += __ldcg(p.ws.pair_w + pp) * acc;
-        }
-        __syncwarp();
+        if (lane == 0) dslot[warp][__ldcg(p.ws.pair_tok + pp) * K + __ldcg(p.ws.pair_slot + pp)] = acc;
       }
     }
-    if (lane < p.M) p.y[(size_t)lane * H + r] = __float2bfloat16_rn(yacc[warp][lane]);
+    __syncwarp();
+    if (lane < p.M) {
+      float y = 0.f;
+      for (int s = 0; s < K; ++s) y = fmaf(__ldcg(p.ws.wts + lane * K + s), dslot[warp][lane * K + s], y);
+      p.y[(size_t)lane * H + r] = __float2bfloat16_rn(y);
+    }
     __syncwarp();
   }
 }

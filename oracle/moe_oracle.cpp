@@ -184,8 +184,9 @@ int oracle_topk(int M, int E, int k, const double* logits, int32_t* ids, double*
   return 0;
 }
 
-// A4 -- the expert union over M tokens (a 4-token verify "can activate up to
-// 32 experts instead of 8" [MTP "What are the 3 optimizations?"]).
+// A4 -- the expert union over M tokens. A 4-token verify step can touch as
+// many as 32 distinct experts where a single token touches 8 [MTP "What are
+// the 3 optimizations?"].
 int oracle_union(int M, int E, int k, const int32_t* ids, int32_t* union_ids,
                  int32_t* pair_off, int32_t* pair_tok, int32_t* pair_slot) {
   if (M < 0 || E <= 0 || k <= 0) return -1;

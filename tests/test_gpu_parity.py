@@ -331,3 +331,16 @@ def test_device_generator_matches_cpu_slices():
         part = synth.expert_np(11, 3, e, H, I)
         for a, b in zip(full, part):
             assert np.array_equal(a[e].cpu().numpy(), b)
+
+
+def test_smaller_context_keeps_larger_context_working():
+    """The dynamic shared-memory limit of a kernel is per device, not per
+    context: creating a context with a smaller plan after a larger one must
+    not break the larger one's launches (persistent and three-kernel paths)."""
+    L = Layer(2560, 768, 256, 8, 4, seed=14, mode="natural")
+    for flags in (0, moe.MOE_FLAG_SPLIT_KERNELS):
+        big = L.make_ctx(flags, max_tokens=32)
+        small = L.make_ctx(flags, max_tokens=1)
+        got = L.run(big)
+        compare(L, got, L.oracle())
+        small.close()
