@@ -106,6 +106,25 @@ typedef enum {
                                        where h*inv lies at a rounding
                                        boundary. Persistent kernel only, as
                                        MOE_FLAG_SHARED_EXPERT */
+#define MOE_FLAG_CUDA_CORES 0x10u    /* run the persistent CUDA-core kernel
+                                       (E2M1 decoded in registers for both
+                                       projections) */
+#define MOE_FLAG_TENSOR_CORES 0x20u  /* run the persistent tensor-core kernel
+                                       (gate/up on tcgen05 block-scaled MMAs,
+                                       down on CUDA cores); needs H and I to
+                                       be multiples of 128 and its
+                                       shared-memory plan to fit, else
+                                       moe_create returns MOE_ERR_UNSUPPORTED.
+                                       With neither flag (and without
+                                       MOE_FLAG_SPLIT_KERNELS) moe_create
+                                       picks the tensor-core kernel when the
+                                       shape allows it and max_tokens is at
+                                       least MOE_TC_MIN_TOKENS, else the
+                                       CUDA-core kernel. Both compute the same
+                                       step; moe_query names the one a context
+                                       runs. Setting both flags is
+                                       MOE_ERR_INVALID_ARG */
+#define MOE_TC_MIN_TOKENS 2
 
 typedef struct {
   int32_t hidden;      /* H: multiple of 32, 32..8192                        */
@@ -187,6 +206,17 @@ moe_status moe_plan_query(const moe_config* cfg, int32_t sm_count, size_t smem_l
  * word, finishes with garbage output and returns, and moe_sync_status then
  * reports MOE_ERR_TIMEOUT. Returns INVALID_ARG for a NULL ctx. */
 moe_status moe_debug_set_wait(moe_ctx* ctx, long long budget_cycles, int force_stall);
+
+/* Test hook for measurements of the tensor-core kernel: with a non-NULL
+ * device pointer to grid x 16 uint64 words (8-byte aligned), every later
+ * moe_decode of this context writes %globaltimer stamps of its phases per CTA
+ * there (slot 0 kernel start, 1 after the programmatic-launch wait, 2 logits
+ * published, 3 all logits gathered, 4 routing done, 5 first gate/up stage
+ * landed, 6 last MMA issued, 7 gate/up epilogue done, 9 last entry's h
+ * ready, 10/11 down work done, 12 kernel end); slots not reached keep their
+ * value. NULL turns it off. Ignored by the other kernels. Returns
+ * INVALID_ARG for a NULL ctx or a misaligned pointer. */
+moe_status moe_debug_set_trace(moe_ctx* ctx, unsigned long long* trace);
 
 /* Size of the fixed device scratch array behind moe_decode_static. */
 #define MOE_STATIC_SCRATCH_BYTES ((size_t)4 << 20)

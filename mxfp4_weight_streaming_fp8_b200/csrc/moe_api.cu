@@ -2,11 +2,13 @@
 // validation, the per-context workspace, and kernel launches on the caller's
 // stream. No allocation happens after moe_create; nothing falls back to the
 // CPU.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstdio>
 #include <algorithm>
 #include <cstring>
+#include <mutex>
 #include <new>
 
 #include "../../include/moe.h"
@@ -14,6 +16,7 @@
 #include "moe_host.h"
 #include "moe_fused.cuh"
 #include "moe_split.cuh"
+#include "moe_tc.cuh"
 
 using moe_host::aligned16;
 using moe_host::align_up;
@@ -22,7 +25,7 @@ using moe_host::kDefaultSpinLimit;
 
 namespace {
 
-enum Variant { kFused = 0, kSplit = 1 };
+enum Variant { kFused = 0, kSplit = 1, kTc = 2 };
 
 
 
@@ -33,7 +36,10 @@ moe_status validate_config(const moe_config& c) {
   if (c.top_k < 1 || c.top_k > c.num_experts || c.top_k > moe::kMaxTopK) return MOE_ERR_INVALID_ARG;
   if (c.max_tokens < 1 || c.max_tokens > moe::kMaxTokens) return MOE_ERR_INVALID_ARG;
   const uint32_t fused_only = MOE_FLAG_PRE_RMSNORM | MOE_FLAG_SHARED_EXPERT | MOE_FLAG_FP8_INTERMEDIATE;
-  if (c.flags & ~(MOE_FLAG_SPLIT_KERNELS | fused_only)) return MOE_ERR_INVALID_ARG;
+  if (c.flags & ~(MOE_FLAG_SPLIT_KERNELS | MOE_FLAG_CUDA_CORES | MOE_FLAG_TENSOR_CORES | fused_only))
+    return MOE_ERR_INVALID_ARG;
+  if ((c.flags & MOE_FLAG_CUDA_CORES) && (c.flags & MOE_FLAG_TENSOR_CORES)) return MOE_ERR_INVALID_ARG;
+  if ((c.flags & MOE_FLAG_TENSOR_CORES) && (c.flags & MOE_FLAG_SPLIT_KERNELS)) return MOE_ERR_INVALID_ARG;
   if ((c.flags & fused_only) && (c.flags & MOE_FLAG_SPLIT_KERNELS)) return MOE_ERR_UNSUPPORTED;
   return MOE_OK;
 }
@@ -124,6 +130,141 @@ bool make_plan(const moe_config& c, int sm_count, size_t smem_limit, moe::FusedP
   return (size_t)pl->smem_bytes <= smem_limit;
 }
 
+// Shared-memory plan of the tensor-core kernel (mirrors k_tc's carving).
+// Returns false when the shape is outside what k_tc covers or does not fit.
+bool make_tc_plan(const moe_config& c, int sm_count, size_t smem_limit, moe::TcPlan* pl) {
+  const size_t H = c.hidden, I = c.inter, E = c.num_experts, MM = c.max_tokens;
+  const size_t G = sm_count;
+  if (H % 128 || I % 128) return false;  // K-chunks of 128 elements
+  size_t NP, UMAX;
+  union_bounds(c, &NP, &UMAX);
+  const size_t KCH = H / 128;
+  *pl = moe::TcPlan{};
+  pl->G = (int)G;
+  pl->max_pairs = (int)NP;
+  pl->max_union = (int)UMAX;
+  const size_t units_max = UMAX * (I / 4);
+  const size_t tu_max = std::min<size_t>(moe::kTcMaxUnits, (units_max + G - 1) / G);
+  pl->tu_max = (int)tu_max;
+  pl->ks = (tu_max <= 12 && KCH % 2 == 0) ? 2 : 1;
+  const size_t ks = pl->ks, nstage = KCH / ks;
+  pl->nb_max = (int)std::max<size_t>(8, (MM + 7) / 8 * 8);
+  pl->slot_gu = (int)(tu_max * ks * 1024);
+  pl->bx_bytes = (int)(KCH * (pl->nb_max / 8) * 1024);
+  const size_t overread = (moe::kTcMaxUnits - tu_max) * ks * 1024;  // junk MMA rows past the last slot
+  pl->sc_bytes = (int)align_up(8 * tu_max * (H / 32), 128);
+  const size_t nrd_max = (H + G - 1) / G;
+  pl->rpc_max = (int)nrd_max;
+  pl->slot_d = (int)align_up(nrd_max * (I / 2) + nrd_max * (I / 32) + 32, 128);
+  pl->hpairs = 0;  // h is read from L2 by each down item (no staged copy)
+  pl->hslot = 0;
+  if ((E + G - 1) / G > (size_t)moe::kMaxRowsPerCta) return false;
+  pl->wr_bytes_max = (int)align_up(((E + G - 1) / G) * H * 4, 128);
+  const size_t lg_bytes = align_up(MM * E * 4 + E * 4, 128);  // gathered logits + union scratch
+  // fixed regions
+  size_t fixed = align_up(std::max<size_t>(pl->bx_bytes, overread), 1024) + 2 * pl->sc_bytes;
+  const size_t bar_bytes = (2 * moe::kTcMaxSlots + 4 + 3 * moe::kMaxSlots + 1 + 6) * 8 + moe::kMaxSlots * 4;
+  // tensor memory: 2 accumulators of 32 columns, 2 tiles' scale factors (4
+  // columns per K-chunk), 4 columns of token scale factors
+  const size_t cols = 64 + 8 * KCH + 4;
+  if (cols > 512) return false;
+  pl->tmem_cols = 32;
+  while ((size_t)pl->tmem_cols < cols) pl->tmem_cols *= 2;
+  const size_t misc_bytes = (3 * moe::kMaxTokens + moe::kTcWarps * moe::kMaxRowsPerCta * 4 + 8) * 4;
+  const size_t small = align_up(bar_bytes, 16) + align_up(misc_bytes, 16) + 4 * align_up(NP * 4, 16) +
+                       align_up(UMAX * 4, 16) + align_up((UMAX + 1) * 4, 16) + align_up(NP * nrd_max * 4, 16);
+  fixed += small + 1024 /* alignment slack */ + 4 * 128;
+  if (fixed >= smem_limit) return false;
+  size_t room = smem_limit - fixed;
+  // down ring: up to 8 entries in flight, at least 2
+  size_t ns_d = std::min<size_t>(UMAX, 8), per_d = pl->slot_d + pl->hslot;
+  while (ns_d > 2 && room < ns_d * per_d + 2 * (size_t)pl->slot_gu) --ns_d;
+  if (room < ns_d * per_d) return false;
+  room -= ns_d * per_d;
+  size_t ns_gu = std::min<size_t>({(size_t)moe::kTcMaxSlots, nstage, room / pl->slot_gu});
+  if (ns_gu < 1) return false;
+  if (ns_gu < 2 && nstage >= 2) return false;
+  pl->ns_gu = (int)ns_gu;
+  pl->ns_d = (int)ns_d;
+  // layout
+  // routing scratch: the router rows at the start of the gate/up ring; the
+  // gathered logits after them when they fit there, else in the down ring
+  // after the staged x (both rings are idle until routing ends)
+  const size_t ring_gu_bytes = ns_gu * (size_t)pl->slot_gu;
+  const size_t ring_d_bytes = ns_d * (size_t)pl->slot_d + ns_d * (size_t)pl->hslot;
+  const bool x_fits = MM * H * 2 <= ring_d_bytes;
+  const bool lg_in_gu = pl->wr_bytes_max + lg_bytes <= ring_gu_bytes;
+  const bool lg_in_d = !lg_in_gu && (x_fits ? align_up(MM * H * 2, 128) : 0) + lg_bytes <= ring_d_bytes;
+  size_t off = 0;
+  auto take = [&](size_t bytes, size_t a) { off = align_up(off, a); size_t o = off; off += bytes; return o; };
+  pl->o_ring_gu =
+      (int)take(std::max(ring_gu_bytes, (size_t)pl->wr_bytes_max + ((lg_in_gu || lg_in_d) ? 0 : lg_bytes)), 1024);
+  pl->o_bx = (int)take(std::max<size_t>(pl->bx_bytes, overread), 1024);
+  pl->o_sf = (int)off;  // (no shared-memory scale-factor staging)
+  pl->o_sc = (int)take(2 * (size_t)pl->sc_bytes, 128);
+  pl->o_sfb = (int)off;
+  pl->o_ring_d = (int)take(ns_d * (size_t)pl->slot_d, 128);
+  pl->o_h = (int)take(ns_d * (size_t)pl->hslot, 16);
+  pl->x_staged = x_fits ? 1 : 0;
+  pl->o_lg = lg_in_d ? pl->o_ring_d + (int)(x_fits ? align_up(MM * H * 2, 128) : 0)
+                     : pl->o_ring_gu + pl->wr_bytes_max;
+  pl->o_bar = (int)take(bar_bytes, 16);
+  pl->o_misc = (int)take(misc_bytes, 16);
+  pl->o_ids = (int)take(NP * 4, 16);
+  pl->o_w = (int)take(NP * 4, 16);
+  pl->o_pm = (int)take(NP * 4, 16);
+  pl->o_ppos = (int)take(NP * 4, 16);
+  pl->o_union = (int)take(UMAX * 4, 16);
+  pl->o_poff = (int)take((UMAX + 1) * 4, 16);
+  pl->o_dsm = (int)take(NP * nrd_max * 4, 16);
+  pl->smem_bytes = (int)(off + 1024);
+  return (size_t)pl->smem_bytes <= smem_limit;
+}
+
+// cuTensorMapEncodeTiled from the driver, looked up once through the runtime
+// (no link against libcuda).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_tiled() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+    else
+      cudaGetLastError();
+  });
+  return fn;
+}
+
+// The gate/up code maps of k_tc over the caller's w13_codes [Eall][2I][H/2]
+// (4-bit elements): dimensions (128 elements of a K-chunk | 4 rows, H/2 bytes
+// apart | gate/up, I rows apart | K-chunk, 64 bytes apart | 4-row quad,
+// 4 rows apart), unpacked to 16 bytes per 16 codes with a 128-byte swizzle.
+// Map n-1 copies n units (quads, coordinate e*I/2 + j for gate rows 4j..4j+3
+// of expert e) x ks K-chunks. The coordinates k_tc issues keep j < I/4, so a
+// copy never reaches past expert e's up rows.
+bool encode_w13_maps(const void* w13c, size_t Eall, size_t H, size_t I, int ks, CUtensorMap* maps) {
+  EncodeTiledFn enc = encode_tiled();
+  if (!enc) return false;
+  if (reinterpret_cast<uintptr_t>(w13c) & 31) return false;  // 16U4_ALIGN16B wants 32-byte alignment
+  const cuuint64_t dims[5] = {128, 4, 2, (cuuint64_t)(H / 128), (cuuint64_t)(Eall * (I / 2))};
+  const cuuint64_t strides[4] = {(cuuint64_t)(H / 2), (cuuint64_t)(I * (H / 2)), 64, (cuuint64_t)(4 * (H / 2))};
+  const cuuint32_t es[5] = {1, 1, 1, 1, 1};
+  for (int n = 1; n <= moe::kTcMaxUnits; ++n) {
+    const cuuint32_t box[5] = {128, 4, 2, (cuuint32_t)ks, (cuuint32_t)n};
+    if (enc(maps + n - 1, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 5, const_cast<void*>(w13c), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return false;
+  }
+  return true;
+}
+
 }  // namespace
 
 struct moe_ctx {
@@ -145,9 +286,14 @@ struct moe_ctx {
   size_t smem_gateup = 0, smem_fused = 0;
   long long spin_limit = 0;
   int force_stall = 0;
+  unsigned long long* trace = nullptr;
   void (*fused)(moe::Params, moe::FusedWs, moe::FusedPlan) = nullptr;  // k_fused instantiation
   moe::FusedPlan plan{};
   moe::FusedWs fws{};
+  void (*tc)(moe::Params, moe::TcWs, moe::TcPlan, const moe::TcMaps) = nullptr;  // k_tc instantiation
+  moe::TcPlan tplan{};
+  moe::TcWs tws{};
+  moe::TcMaps maps{};  // encoded at load, passed by value at every launch
 };
 
 extern "C" {
@@ -191,6 +337,21 @@ moe_status moe_create(const moe_config* cfg, moe_ctx** out) {
     const bool sh = (c.flags & MOE_FLAG_SHARED_EXPERT) != 0, f8 = (c.flags & MOE_FLAG_FP8_INTERMEDIATE) != 0;
     ctx->fused = sh ? (f8 ? moe::k_fused<true, true> : moe::k_fused<true, false>)
                     : (f8 ? moe::k_fused<false, true> : moe::k_fused<false, false>);
+    ctx->tc = sh ? (f8 ? moe::k_tc<true, true> : moe::k_tc<true, false>)
+                 : (f8 ? moe::k_tc<false, true> : moe::k_tc<false, false>);
+  }
+  // the tensor-core kernel when asked for, or by default from
+  // MOE_TC_MIN_TOKENS tokens on, wherever its shape rules hold
+  {
+    const bool want_tc = (c.flags & MOE_FLAG_TENSOR_CORES) ||
+                         (!(c.flags & MOE_FLAG_CUDA_CORES) && c.max_tokens >= MOE_TC_MIN_TOKENS);
+    const bool tc_ok = make_tc_plan(c, prop.multiProcessorCount, (size_t)prop.sharedMemPerBlockOptin, &ctx->tplan) &&
+                       encode_tiled() != nullptr;
+    if ((c.flags & MOE_FLAG_TENSOR_CORES) && !tc_ok) {
+      delete ctx;
+      return MOE_ERR_UNSUPPORTED;
+    }
+    if (ctx->variant == kFused && want_tc && tc_ok) ctx->variant = kTc;
   }
 
   // workspace layout
@@ -216,6 +377,9 @@ moe_status moe_create(const moe_config* cfg, moe_ctx** out) {
   const size_t o_flog = take(MM * E * sizeof(float));
   const size_t o_rcnt = take(sizeof(unsigned long long));
   const size_t o_gcnt = take(UMAXF * moe::kCounterStride * sizeof(unsigned long long));
+  const size_t o_tlog = take(MM * E * sizeof(unsigned long long));
+  const size_t o_th = take(NPF * I * sizeof(float));
+  const size_t o_tcnt = take(2 * UMAXF * moe::kTcCntStride * sizeof(unsigned));
   ctx->ws_bytes = off;
   if (cudaMalloc(&ctx->ws_base, ctx->ws_bytes) != cudaSuccess) {
     cudaGetLastError();
@@ -246,6 +410,10 @@ moe_status moe_create(const moe_config* cfg, moe_ctx** out) {
   ctx->fws.route_cnt = reinterpret_cast<unsigned long long*>(b + o_rcnt);
   ctx->fws.gu_cnt = reinterpret_cast<unsigned long long*>(b + o_gcnt);
   ctx->fws.epoch = w.ctrl + 5;
+  ctx->tws.logits = reinterpret_cast<unsigned long long*>(b + o_tlog);
+  ctx->tws.h = reinterpret_cast<float*>(b + o_th);
+  ctx->tws.hcnt = reinterpret_cast<unsigned*>(b + o_tcnt);
+  ctx->tws.epoch = w.ctrl + 6;
 
   // launch shapes
   ctx->grid_route = (int)(E < (size_t)ctx->sm_count ? E : (size_t)ctx->sm_count);
@@ -268,6 +436,13 @@ moe_status moe_create(const moe_config* cfg, moe_ctx** out) {
   if (err == cudaSuccess && plan_ok)
     err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_f, ctx->fused, moe::kFusedThreads,
                                                         ctx->plan.smem_bytes);
+  if (err == cudaSuccess && ctx->variant == kTc) {
+    err = cudaFuncSetAttribute(ctx->tc, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_optin);
+    int occ_t = 0;
+    if (err == cudaSuccess)
+      err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_t, ctx->tc, moe::kTcThreads, ctx->tplan.smem_bytes);
+    if (err == cudaSuccess && occ_t < 1) ctx->variant = kFused;
+  }
   if (err != cudaSuccess || occ_g < 1 || occ_d < 1 || !plan_ok || occ_f < 1) {
     cudaGetLastError();
     cudaFree(ctx->ws_base);
@@ -313,6 +488,10 @@ moe_status moe_load_experts(moe_ctx* ctx, const float* router_w, const uint8_t* 
       ctx->loaded = false;
       return MOE_ERR_BAD_WEIGHTS;
     }
+  }
+  if (ctx->variant == kTc) {
+    const size_t Eall = c.num_experts + ((c.flags & MOE_FLAG_SHARED_EXPERT) ? 1 : 0);
+    if (!encode_w13_maps(w13_codes, Eall, c.hidden, c.inter, ctx->tplan.ks, ctx->maps.m)) return MOE_ERR_INVALID_ARG;
   }
   ctx->wr = router_w;
   ctx->w13c = w13_codes;
@@ -362,6 +541,7 @@ moe_status moe_decode(moe_ctx* ctx, const void* x_bf16, int32_t M, void* y_bf16,
   p.out_xscale = xscale;
   p.spin_limit = ctx->spin_limit;
   p.force_stall = ctx->force_stall;
+  p.trace = ctx->variant == kTc ? ctx->trace : nullptr;
   p.pre_rmsnorm = (c.flags & MOE_FLAG_PRE_RMSNORM) ? 1 : 0;
   p.out_xn = static_cast<__nv_bfloat16*>(xnorm_bf16);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -371,16 +551,18 @@ moe_status moe_decode(moe_ctx* ctx, const void* x_bf16, int32_t M, void* y_bf16,
     moe::k_down<<<ctx->grid_down, moe::kThreads, 0, st>>>(p);
   } else {
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(ctx->grid_fused);
-    cfg.blockDim = dim3(moe::kFusedThreads);
-    cfg.dynamicSmemBytes = ctx->smem_fused;
+    cfg.gridDim = dim3(ctx->variant == kTc ? ctx->tplan.G : ctx->grid_fused);
+    cfg.blockDim = dim3(ctx->variant == kTc ? moe::kTcThreads : moe::kFusedThreads);
+    cfg.dynamicSmemBytes = ctx->variant == kTc ? ctx->tplan.smem_bytes : ctx->smem_fused;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, ctx->fused, p, ctx->fws, ctx->plan) != cudaSuccess) {
+    const cudaError_t le = ctx->variant == kTc ? cudaLaunchKernelEx(&cfg, ctx->tc, p, ctx->tws, ctx->tplan, ctx->maps)
+                                               : cudaLaunchKernelEx(&cfg, ctx->fused, p, ctx->fws, ctx->plan);
+    if (le != cudaSuccess) {
       cudaGetLastError();
       return MOE_ERR_CUDA;
     }
@@ -413,22 +595,47 @@ moe_status moe_plan_query(const moe_config* cfg, int32_t sm_count, size_t smem_l
   if (v != MOE_OK) return v;
   moe::FusedPlan pl{};
   const bool ok = make_plan(*cfg, sm_count, smem_limit, &pl);
+  moe::TcPlan tp{};
+  const bool tok = make_tc_plan(*cfg, sm_count, smem_limit, &tp);
+  const bool tc = tok && !(cfg->flags & (MOE_FLAG_SPLIT_KERNELS | MOE_FLAG_CUDA_CORES)) &&
+                  ((cfg->flags & MOE_FLAG_TENSOR_CORES) || cfg->max_tokens >= MOE_TC_MIN_TOKENS);
   const int n = snprintf(buf, len,
-                         "{\"ok\": %s, \"grid\": %d, \"threads\": %d, \"smem\": %d, \"slot_gu\": %d, "
+                         "{\"ok\": %s, \"variant\": \"%s\", \"grid\": %d, \"threads\": %d, \"smem\": %d, "
+                         "\"slot_gu\": %d, "
                          "\"ns_gu\": %d, \"slot_d\": %d, \"ns_d\": %d, \"rows_per_cta_down\": %d, "
                          "\"router_bytes_per_cta\": %d, \"o_act\": %d, \"o_dsm\": %d, \"o_ring_gu\": %d, "
-                         "\"o_ring_d\": %d, \"o_h\": %d, \"hslot\": %d, \"hpairs\": %d, \"x_staged\": %d}",
-                         ok ? "true" : "false", pl.G, moe::kFusedThreads, pl.smem_bytes, pl.slot_gu, pl.ns_gu,
-                         pl.slot_d, pl.ns_d, pl.rpc_max, pl.wr_bytes_max, pl.o_act, pl.o_dsm, pl.o_ring_gu,
-                         pl.o_ring_d, pl.o_h, pl.hslot, pl.hpairs, pl.x_staged);
+                         "\"o_ring_d\": %d, \"o_h\": %d, \"hslot\": %d, \"hpairs\": %d, \"x_staged\": %d, "
+                         "\"tc\": {\"ok\": %s, \"grid\": %d, \"threads\": %d, \"smem\": %d, \"ks\": %d, "
+                         "\"tu_max\": %d, \"nb_max\": %d, \"ns_gu\": %d, \"slot_gu\": %d, \"ns_d\": %d, "
+                         "\"slot_d\": %d, \"rpc_max\": %d, \"hslot\": %d, \"hpairs\": %d, \"wr_bytes_max\": %d, "
+                         "\"x_staged\": %d, \"o_ring_gu\": %d, \"o_bx\": %d, \"o_sf\": %d, \"o_sc\": %d, "
+                         "\"o_sfb\": %d, \"o_ring_d\": %d, \"o_h\": %d, \"o_bar\": %d, \"o_misc\": %d, "
+                         "\"o_ids\": %d, \"o_w\": %d, \"o_pm\": %d, \"o_ppos\": %d, \"o_union\": %d, "
+                         "\"o_poff\": %d, \"o_dsm\": %d, \"sc_bytes\": %d, \"bx_bytes\": %d, "
+                         "\"max_pairs\": %d, \"max_union\": %d, \"o_lg\": %d, \"tmem_cols\": %d}}",
+                         (tc || ok) ? "true" : "false", tc ? "tc" : "fused", pl.G, moe::kFusedThreads, pl.smem_bytes,
+                         pl.slot_gu, pl.ns_gu, pl.slot_d, pl.ns_d, pl.rpc_max, pl.wr_bytes_max, pl.o_act, pl.o_dsm,
+                         pl.o_ring_gu, pl.o_ring_d, pl.o_h, pl.hslot, pl.hpairs, pl.x_staged, tok ? "true" : "false",
+                         tp.G, moe::kTcThreads, tp.smem_bytes, tp.ks, tp.tu_max, tp.nb_max, tp.ns_gu, tp.slot_gu,
+                         tp.ns_d, tp.slot_d, tp.rpc_max, tp.hslot, tp.hpairs, tp.wr_bytes_max, tp.x_staged,
+                         tp.o_ring_gu, tp.o_bx, tp.o_sf, tp.o_sc, tp.o_sfb, tp.o_ring_d, tp.o_h, tp.o_bar, tp.o_misc,
+                         tp.o_ids, tp.o_w, tp.o_pm, tp.o_ppos, tp.o_union, tp.o_poff, tp.o_dsm, tp.sc_bytes,
+                         tp.bx_bytes, tp.max_pairs, tp.max_union, tp.o_lg, tp.tmem_cols);
   if (n < 0 || (size_t)n >= len) return MOE_ERR_INVALID_ARG;
-  return ok ? MOE_OK : MOE_ERR_UNSUPPORTED;
+  return (tc || ok) ? MOE_OK : MOE_ERR_UNSUPPORTED;
 }
 
 moe_status moe_debug_set_wait(moe_ctx* ctx, long long budget_cycles, int force_stall) {
   if (!ctx) return MOE_ERR_INVALID_ARG;
   ctx->spin_limit = budget_cycles > 0 ? budget_cycles : kDefaultSpinLimit;
   ctx->force_stall = force_stall ? 1 : 0;
+  return MOE_OK;
+}
+
+moe_status moe_debug_set_trace(moe_ctx* ctx, unsigned long long* trace) {
+  if (!ctx) return MOE_ERR_INVALID_ARG;
+  if (trace && (reinterpret_cast<uintptr_t>(trace) & 7)) return MOE_ERR_INVALID_ARG;
+  ctx->trace = trace;
   return MOE_OK;
 }
 
@@ -445,6 +652,21 @@ moe_status moe_query(const moe_ctx* ctx, char* buf, size_t len) {
                  "\"hidden\": %d, \"inter\": %d, \"num_experts\": %d, \"top_k\": %d, \"max_tokens\": %d}",
                  ctx->dev, ctx->sm_count, ctx->grid_route, ctx->grid_gateup, ctx->grid_down, moe::kThreads,
                  ctx->smem_gateup, c.hidden, c.inter, c.num_experts, c.top_k, c.max_tokens);
+  } else if (ctx->variant == kTc) {
+    const moe::TcPlan& tp = ctx->tplan;
+    n = snprintf(buf, len,
+                 "{\"lib\": \"libmoe\", \"arch\": \"sm_100a\", \"device\": %d, \"sm_count\": %d, "
+                 "\"variant\": \"tc\", \"kernels\": [\"k_tc\"], \"grid\": [%d], \"threads\": %d, "
+                 "\"smem\": %d, \"gate_up\": \"tcgen05.mma kind::mxf8f6f4 block_scale M=128 N=%d\", "
+                 "\"units_per_tile\": %d, \"kchunks_per_stage\": %d, \"ring_gu\": [%d, %d], \"ring_d\": [%d, %d], "
+                 "\"x_staged\": %d, \"pdl\": true, \"pre_rmsnorm\": %s, \"shared_expert\": %s, "
+                 "\"fp8_intermediate\": %s, \"hidden\": %d, \"inter\": %d, \"num_experts\": %d, \"top_k\": %d, "
+                 "\"max_tokens\": %d}",
+                 ctx->dev, ctx->sm_count, tp.G, moe::kTcThreads, tp.smem_bytes, tp.nb_max, tp.tu_max, tp.ks, tp.ns_gu,
+                 tp.slot_gu, tp.ns_d, tp.slot_d, tp.x_staged, (c.flags & MOE_FLAG_PRE_RMSNORM) ? "true" : "false",
+                 (c.flags & MOE_FLAG_SHARED_EXPERT) ? "true" : "false",
+                 (c.flags & MOE_FLAG_FP8_INTERMEDIATE) ? "true" : "false", c.hidden, c.inter, c.num_experts, c.top_k,
+                 c.max_tokens);
   } else {
     n = snprintf(buf, len,
                  "{\"lib\": \"libmoe\", \"arch\": \"sm_100a\", \"device\": %d, \"sm_count\": %d, "

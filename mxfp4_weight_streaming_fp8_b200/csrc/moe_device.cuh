@@ -58,6 +58,7 @@ struct Params {
   long long spin_limit;  // device-side wait budget in clock64 cycles
   int force_stall;       // test hook: the logits wait targets a tag nobody writes
   int pre_rmsnorm;       // x <- bf16(x * rsqrt(mean(x^2) + eps)) before A1/A2
+  unsigned long long* trace;  // test hook: per-CTA phase timestamps (globaltimer), or null
   __nv_bfloat16* out_xn; // optional [M][H] normalised input
 };
 

@@ -22,6 +22,9 @@ MOE_FLAG_SPLIT_KERNELS = 0x1
 MOE_FLAG_PRE_RMSNORM = 0x2
 MOE_FLAG_SHARED_EXPERT = 0x4
 MOE_FLAG_FP8_INTERMEDIATE = 0x8
+MOE_FLAG_CUDA_CORES = 0x10
+MOE_FLAG_TENSOR_CORES = 0x20
+MOE_TC_MIN_TOKENS = 2
 MOE_LOAD_BORROW = 0x0
 MOE_LOAD_SKIP_VALIDATE = 0x1
 
@@ -71,6 +74,8 @@ def lib() -> ctypes.CDLL:
         L.moe_decode_static.restype = ctypes.c_int
         L.moe_debug_set_wait.argtypes = [_vp, ctypes.c_longlong, ctypes.c_int]
         L.moe_debug_set_wait.restype = ctypes.c_int
+        L.moe_debug_set_trace.argtypes = [_vp, _vp]
+        L.moe_debug_set_trace.restype = ctypes.c_int
         L.moe_lm_create.argtypes = [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                     ctypes.POINTER(_vp)]
         L.moe_lm_create.restype = ctypes.c_int
@@ -104,7 +109,7 @@ def _stream_handle(stream):
 def plan_query(hidden, inter, num_experts, top_k, max_tokens, flags=0, sm_count=148, smem_limit=232448):
     """(status, plan dict) of the persistent kernel for a shape; host only."""
     cfg = moe_config(hidden, inter, num_experts, top_k, max_tokens, flags, 0)
-    buf = ctypes.create_string_buffer(1024)
+    buf = ctypes.create_string_buffer(4096)
     st = lib().moe_plan_query(ctypes.byref(cfg), sm_count, smem_limit, buf, len(buf))
     return st, (json.loads(buf.value.decode()) if buf.value else None)
 
@@ -179,6 +184,11 @@ class MoELayer:
 
     def set_wait(self, budget_cycles: int, force_stall: bool = False) -> int:
         return lib().moe_debug_set_wait(self._ctx, int(budget_cycles), int(bool(force_stall)))
+
+    def set_trace(self, trace) -> int:
+        """Per-CTA phase timestamps of the tensor-core kernel into a device
+        uint64 tensor of grid x 48 words (None turns it off)."""
+        return lib().moe_debug_set_trace(self._ctx, _ptr(trace))
 
     def query(self) -> dict:
         buf = ctypes.create_string_buffer(1024)

@@ -99,7 +99,8 @@ def test_shared_expert_flag_without_gpu(L):
     assert L.moe_create(ctypes.byref(c), ctypes.byref(out)) == 2 and not out.value
     c = moe.moe_config(256, 64, 16, 2, 1, moe.MOE_FLAG_FP8_INTERMEDIATE | moe.MOE_FLAG_SPLIT_KERNELS, 0)
     assert L.moe_create(ctypes.byref(c), ctypes.byref(out)) == 2 and not out.value
-    c = moe.moe_config(256, 64, 16, 2, 1, moe.MOE_FLAG_SHARED_EXPERT | moe.MOE_FLAG_PRE_RMSNORM | 0x10, 0)
+    # an unknown flag bit is refused as an invalid argument (0x10 is MOE_FLAG_CUDA_CORES)
+    c = moe.moe_config(256, 64, 16, 2, 1, moe.MOE_FLAG_SHARED_EXPERT | moe.MOE_FLAG_PRE_RMSNORM | 0x40, 0)
     assert L.moe_create(ctypes.byref(c), ctypes.byref(out)) == 1 and not out.value
     for shape in [(2560, 768, 256, 8, 1), (2560, 768, 256, 8, 32), (128, 64, 8, 8, 3), (256, 64, 16, 2, 1)]:
         st0, base = moe.plan_query(*shape)
