@@ -63,6 +63,7 @@ def load_peaks():
 KERNEL_SOURCES = {
     # the device code each kernel is compiled from
     "k_fused": ("moe_fused.cuh", "moe_device.cuh"),
+    "k_tc": ("moe_tc.cuh", "moe_fused.cuh", "moe_device.cuh"),
     "k_lm_head": ("moe_lmhead.cu", "moe_device.cuh"),
 }
 
@@ -176,7 +177,7 @@ def sum_over_ranks(value: float, ws: int, device=None) -> float:
 
 
 # ------------------------------------------------------------------ workload
-def build_pool(device, M, mode, layers=POOL_LAYERS, seed=SEED, flags=0, stack=False, shared=False):
+def build_pool(device, M, mode, layers=POOL_LAYERS, seed=SEED, flags=0, stack=False, shared=False, repack=False):
     """One context per layer of the pool. With stack=True, layers after the
     first normalise their input (RMSNorm) and take the previous output. With
     shared=True every layer has one more expert (index E), the shared one."""
@@ -195,7 +196,7 @@ def build_pool(device, M, mode, layers=POOL_LAYERS, seed=SEED, flags=0, stack=Fa
         lflags = flags | (moe.MOE_FLAG_PRE_RMSNORM if (stack and l > 0) else 0)
         lflags |= moe.MOE_FLAG_SHARED_EXPERT if shared else 0
         ctx = moe.MoELayer(H, I, E, K, M, flags=lflags, device=device.index)
-        ctx.load_experts(wr_d, *ex, validate=False)
+        ctx.load_experts(wr_d, *ex, validate=False, repack=repack)
         ctxs.append(ctx)
         weights.append((wr_d, ex))
     return x, ctxs, weights
@@ -214,10 +215,11 @@ def run_ours(args):
     from mxfp4_weight_streaming_fp8_b200 import moe
     M = args.tokens
     L = args.layers
-    flags = moe.MOE_FLAG_SPLIT_KERNELS if args.variant == "split" else 0
+    flags = {"split": moe.MOE_FLAG_SPLIT_KERNELS, "cuda": moe.MOE_FLAG_CUDA_CORES,
+             "tc": moe.MOE_FLAG_TENSOR_CORES}.get(args.variant, 0)
     flags |= moe.MOE_FLAG_FP8_INTERMEDIATE if args.fp8_intermediate else 0
     x, ctxs, _weights = build_pool(device, M, args.routing, layers=L, flags=flags, stack=args.stack,
-                                   shared=args.shared_expert)
+                                   shared=args.shared_expert, repack=args.repack)
     n_shared = int(args.shared_expert)
     info = ctxs[0].query()
     x_d = x.to(device)
@@ -252,7 +254,8 @@ def run_ours(args):
 
     # the same pool as a dependent chain: layer l+1 takes RMSNorm(y_l), so no
     # layer-step can overlap the previous one (timed after the headline graph)
-    chain = None if args.stack else build_chain(device, ctxs, _weights, x_d, M, flags, args.shared_expert)
+    chain = None if args.stack else build_chain(device, ctxs, _weights, x_d, M, flags, args.shared_expert,
+                                                args.repack)
 
     cur = torch.cuda.current_stream()
     for _ in range(args.warmup):
@@ -301,7 +304,7 @@ def run_ours(args):
     workload = (f"ling_stack{L}_rmsnorm_M{M}" if args.stack else f"ling_layer_M{M}_{args.routing}")
     workload += "_shared1" if n_shared else ""
     workload += "_a8" if args.fp8_intermediate else ""
-    traffic = recorded_traffic("k_fused", workload)
+    traffic = recorded_traffic({"fused": "k_fused", "tc": "k_tc"}.get(info["variant"], "split"), workload)
 
     # ---- end to end through the public API with host buffers
     e2e = run_e2e(args, ctxs, x, device, M, L, stack=args.stack)
@@ -330,7 +333,8 @@ def run_ours(args):
         "expert_frac_of_8tbs": round(exp_b / (us_per_layer * 1e-6) / 8e12, 4),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
-                     "traffic": traffic, "kernel": "k_fused" if info["variant"] == "fused" else "k_gateup+k_down",
+                     "traffic": traffic,
+                     "kernel": {"fused": "k_fused", "tc": "k_tc"}.get(info["variant"], "k_gateup+k_down"),
                      "algorithmic_bytes_per_launch": alg},
         "gpu_launches": launches,
         "clocks": clk.summary(),
@@ -366,7 +370,7 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
-def build_chain(device, ctxs, weights, x_d, M, flags, shared):
+def build_chain(device, ctxs, weights, x_d, M, flags, shared, repack=False):
     """Contexts over the pool's own weights chained as a stack (layers after
     the first normalise their input), captured in one CUDA graph."""
     import torch
@@ -377,7 +381,7 @@ def build_chain(device, ctxs, weights, x_d, M, flags, shared):
         lflags = flags | (moe.MOE_FLAG_PRE_RMSNORM if l > 0 else 0)
         lflags |= moe.MOE_FLAG_SHARED_EXPERT if shared else 0
         c = moe.MoELayer(H, I, E, K, M, flags=lflags, device=device.index)
-        c.load_experts(wr_d, *ex, validate=False)
+        c.load_experts(wr_d, *ex, validate=False, repack=repack)
         chain.append(c)
     ys = [torch.empty_like(x_d) for _ in range(L)]
     stream = torch.cuda.Stream(device)
@@ -704,7 +708,11 @@ def main():
     ap.add_argument("--ref-rows", type=int, default=32768,
                     help="LM head rows per reference (CPU oracle) call, scaled to the vocabulary")
     ap.add_argument("--no-cpu", action="store_true")
-    ap.add_argument("--variant", choices=["fused", "split"], default="fused")
+    ap.add_argument("--variant", choices=["auto", "cuda", "tc", "split"], default="auto",
+                    help="auto: the library's choice for the shape; cuda: the CUDA-core persistent kernel; "
+                         "tc: the tensor-core persistent kernel; split: the three-kernel path")
+    ap.add_argument("--repack", action="store_true",
+                    help="load the layers with MOE_LOAD_COPY_REPACK (context-owned, kernel-private weight layout)")
     ap.add_argument("--shared-expert", action="store_true",
                     help="one always-active shared expert per layer besides the top-8 routed ones")
     ap.add_argument("--fp8-intermediate", action="store_true",

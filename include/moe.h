@@ -146,13 +146,28 @@ moe_status moe_create(const moe_config* cfg, moe_ctx** out);
 /* moe_load_experts load_flags */
 #define MOE_LOAD_BORROW 0x0u        /* keep the caller's pointers (they must outlive the ctx) */
 #define MOE_LOAD_SKIP_VALIDATE 0x1u /* do not scan scale bytes for 0xFF */
+#define MOE_LOAD_COPY_REPACK 0x2u   /* copy the five arrays into memory the context
+                                       owns, re-tiling the gate/up codes into the
+                                       running kernel's private layout; the
+                                       caller may free its arrays after the call */
 
 /* Attach one layer's weights (device pointers, layouts above, each 16-byte
- * aligned). The context borrows them: nothing is copied, and the caller keeps
- * ownership. Unless MOE_LOAD_SKIP_VALIDATE is set, the scale bytes are scanned
- * on the device for the NaN encoding 0xFF, synchronously on the legacy
- * default stream; MOE_ERR_BAD_WEIGHTS if any is found. May be called again to
- * re-point the context at other weights. */
+ * aligned).
+ * Without MOE_LOAD_COPY_REPACK the context borrows them: nothing is copied,
+ * and the caller keeps ownership; the arrays must outlive their use.
+ * With MOE_LOAD_COPY_REPACK the context allocates one device buffer for a
+ * copy of all five arrays (about the size of the inputs) and copies them,
+ * synchronously. For the tensor-core kernel the gate/up codes are re-tiled
+ * so that each 8-row unit (4 gate rows and the 4 up rows of the same
+ * intermediate indices) and 128-element K-chunk is one contiguous 512-byte
+ * block, [E][I/4][H/128][8][64 B]: each stage of the weight stream then reads
+ * whole blocks instead of 64-byte pieces of 8 rows. The CUDA-core and split
+ * kernels get a plain copy in the layout above. The buffer is freed by the
+ * next moe_load_experts or by moe_destroy. OOM if the allocation fails.
+ * Unless MOE_LOAD_SKIP_VALIDATE is set, the scale bytes are scanned on the
+ * device for the NaN encoding 0xFF, synchronously on the legacy default
+ * stream; MOE_ERR_BAD_WEIGHTS if any is found. May be called again to point
+ * the context at other weights. */
 moe_status moe_load_experts(moe_ctx* ctx, const float* router_w,
                             const uint8_t* w13_codes, const uint8_t* w13_scales,
                             const uint8_t* w2_codes, const uint8_t* w2_scales,

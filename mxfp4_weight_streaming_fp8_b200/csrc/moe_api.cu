@@ -170,8 +170,10 @@ bool make_tc_plan(const moe_config& c, int sm_count, size_t smem_limit, moe::TcP
   if (cols > 512) return false;
   pl->tmem_cols = 32;
   while ((size_t)pl->tmem_cols < cols) pl->tmem_cols *= 2;
-  const size_t misc_bytes = (3 * moe::kMaxTokens + moe::kTcWarps * moe::kMaxRowsPerCta * 4 + 8) * 4;
-  const size_t small = align_up(bar_bytes, 16) + align_up(misc_bytes, 16) + 4 * align_up(NP * 4, 16) +
+  const size_t misc_bytes = (3 * moe::kMaxTokens + moe::kTcWarps * moe::kMaxRowsPerCta * 4 + 8 + moe::kTcMaxTiles) * 4;
+  // tiles a CTA may get: at most one more than the rounds of tu_max-unit tiles
+  if ((units_max + G * tu_max - 1) / (G * tu_max) + 1 > (size_t)moe::kTcMaxTiles) return false;
+  const size_t small = align_up(bar_bytes, 16) + align_up(misc_bytes, 16) + align_up(UMAX * 4, 16) + 4 * align_up(NP * 4, 16) +
                        align_up(UMAX * 4, 16) + align_up((UMAX + 1) * 4, 16) + align_up(NP * nrd_max * 4, 16);
   fixed += small + 1024 /* alignment slack */ + 4 * 128;
   if (fixed >= smem_limit) return false;
@@ -193,12 +195,15 @@ bool make_tc_plan(const moe_config& c, int sm_count, size_t smem_limit, moe::TcP
   const size_t ring_gu_bytes = ns_gu * (size_t)pl->slot_gu;
   const size_t ring_d_bytes = ns_d * (size_t)pl->slot_d + ns_d * (size_t)pl->hslot;
   const bool x_fits = MM * H * 2 <= ring_d_bytes;
-  const bool lg_in_gu = pl->wr_bytes_max + lg_bytes <= ring_gu_bytes;
-  const bool lg_in_d = !lg_in_gu && (x_fits ? align_up(MM * H * 2, 128) : 0) + lg_bytes <= ring_d_bytes;
+  // a region of its own when there is room (then no second proxy fence)
+  const bool lg_own = fixed + ns_gu * (size_t)pl->slot_gu + ns_d * per_d + lg_bytes + 128 <= smem_limit &&
+                      lg_bytes <= 16384;
+  const bool lg_in_gu = !lg_own && pl->wr_bytes_max + lg_bytes <= ring_gu_bytes;
+  const bool lg_in_d = !lg_own && !lg_in_gu && (x_fits ? align_up(MM * H * 2, 128) : 0) + lg_bytes <= ring_d_bytes;
   size_t off = 0;
   auto take = [&](size_t bytes, size_t a) { off = align_up(off, a); size_t o = off; off += bytes; return o; };
-  pl->o_ring_gu =
-      (int)take(std::max(ring_gu_bytes, (size_t)pl->wr_bytes_max + ((lg_in_gu || lg_in_d) ? 0 : lg_bytes)), 1024);
+  pl->o_ring_gu = (int)take(
+      std::max(ring_gu_bytes, (size_t)pl->wr_bytes_max + ((lg_own || lg_in_gu || lg_in_d) ? 0 : lg_bytes)), 1024);
   pl->o_bx = (int)take(std::max<size_t>(pl->bx_bytes, overread), 1024);
   pl->o_sf = (int)off;  // (no shared-memory scale-factor staging)
   pl->o_sc = (int)take(2 * (size_t)pl->sc_bytes, 128);
@@ -206,10 +211,13 @@ bool make_tc_plan(const moe_config& c, int sm_count, size_t smem_limit, moe::TcP
   pl->o_ring_d = (int)take(ns_d * (size_t)pl->slot_d, 128);
   pl->o_h = (int)take(ns_d * (size_t)pl->hslot, 16);
   pl->x_staged = x_fits ? 1 : 0;
-  pl->o_lg = lg_in_d ? pl->o_ring_d + (int)(x_fits ? align_up(MM * H * 2, 128) : 0)
-                     : pl->o_ring_gu + pl->wr_bytes_max;
+  pl->lg_own = lg_own ? 1 : 0;
+  pl->o_lg = lg_own ? (int)take(lg_bytes, 128)
+             : lg_in_d ? pl->o_ring_d + (int)(x_fits ? align_up(MM * H * 2, 128) : 0)
+                       : pl->o_ring_gu + pl->wr_bytes_max;
   pl->o_bar = (int)take(bar_bytes, 16);
   pl->o_misc = (int)take(misc_bytes, 16);
+  pl->o_hready = (int)take(UMAX * 4, 16);
   pl->o_ids = (int)take(NP * 4, 16);
   pl->o_w = (int)take(NP * 4, 16);
   pl->o_pm = (int)take(NP * 4, 16);
@@ -265,6 +273,26 @@ bool encode_w13_maps(const void* w13c, size_t Eall, size_t H, size_t I, int ks, 
   return true;
 }
 
+// The same maps over the re-tiled copy [Eall][I/4][H/128][8][64 B]:
+// dimensions (128 elements | 8 rows, 64 bytes apart | K-chunk, 512 bytes
+// apart | unit e*I/4 + j, H/128 * 512 bytes apart).
+bool encode_w13_maps_repacked(const void* w13r, size_t Eall, size_t H, size_t I, int ks, CUtensorMap* maps) {
+  EncodeTiledFn enc = encode_tiled();
+  if (!enc) return false;
+  if (reinterpret_cast<uintptr_t>(w13r) & 31) return false;
+  const cuuint64_t dims[4] = {128, 8, (cuuint64_t)(H / 128), (cuuint64_t)(Eall * (I / 4))};
+  const cuuint64_t strides[3] = {64, 512, (cuuint64_t)((H / 128) * 512)};
+  const cuuint32_t es[4] = {1, 1, 1, 1};
+  for (int n = 1; n <= moe::kTcMaxUnits; ++n) {
+    const cuuint32_t box[4] = {128, 8, (cuuint32_t)ks, (cuuint32_t)n};
+    if (enc(maps + n - 1, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 4, const_cast<void*>(w13r), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return false;
+  }
+  return true;
+}
+
 }  // namespace
 
 struct moe_ctx {
@@ -294,6 +322,7 @@ struct moe_ctx {
   moe::TcPlan tplan{};
   moe::TcWs tws{};
   moe::TcMaps maps{};  // encoded at load, passed by value at every launch
+  void* owned = nullptr;  // MOE_LOAD_COPY_REPACK: the context's copy of the weights
 };
 
 extern "C" {
@@ -461,6 +490,7 @@ void moe_destroy(moe_ctx* ctx) {
   if (!ctx) return;
   DeviceGuard guard(ctx->dev);
   if (ctx->ws_base) cudaFree(ctx->ws_base);
+  if (ctx->owned) cudaFree(ctx->owned);
   delete ctx;
 }
 
@@ -468,7 +498,7 @@ moe_status moe_load_experts(moe_ctx* ctx, const float* router_w, const uint8_t* 
                             const uint8_t* w13_scales, const uint8_t* w2_codes, const uint8_t* w2_scales,
                             uint32_t load_flags) {
   if (!ctx || !router_w || !w13_codes || !w13_scales || !w2_codes || !w2_scales) return MOE_ERR_INVALID_ARG;
-  if (load_flags & ~MOE_LOAD_SKIP_VALIDATE) return MOE_ERR_INVALID_ARG;
+  if (load_flags & ~(MOE_LOAD_SKIP_VALIDATE | MOE_LOAD_COPY_REPACK)) return MOE_ERR_INVALID_ARG;
   if (!aligned16(router_w) || !aligned16(w13_codes) || !aligned16(w13_scales) || !aligned16(w2_codes) ||
       !aligned16(w2_scales))
     return MOE_ERR_INVALID_ARG;
@@ -489,9 +519,59 @@ moe_status moe_load_experts(moe_ctx* ctx, const float* router_w, const uint8_t* 
       return MOE_ERR_BAD_WEIGHTS;
     }
   }
+  const size_t Eall = c.num_experts + ((c.flags & MOE_FLAG_SHARED_EXPERT) ? 1 : 0);
+  const size_t H = c.hidden, I = c.inter;
+  if (ctx->owned) {  // a previous copy
+    cudaFree(ctx->owned);
+    ctx->owned = nullptr;
+  }
+  ctx->loaded = false;
+  ctx->tws.repacked = 0;
+  if (load_flags & MOE_LOAD_COPY_REPACK) {
+    const size_t b_wr = align_up((size_t)c.num_experts * H * 4, 256), b_13 = align_up(Eall * 2 * I * (H / 2), 256),
+                 b_13s = align_up(Eall * 2 * I * (H / 32), 256), b_2 = align_up(Eall * H * (I / 2), 256),
+                 b_2s = align_up(Eall * H * (I / 32), 256);
+    if (cudaMalloc(&ctx->owned, b_wr + b_13 + b_13s + b_2 + b_2s) != cudaSuccess) {
+      cudaGetLastError();
+      ctx->owned = nullptr;
+      return MOE_ERR_OOM;
+    }
+    char* o = static_cast<char*>(ctx->owned);
+    float* wr = reinterpret_cast<float*>(o);
+    uint8_t* w13 = reinterpret_cast<uint8_t*>(o + b_wr);
+    uint8_t* w13s = w13 + b_13;
+    uint8_t* w2 = w13s + b_13s;
+    uint8_t* w2s = w2 + b_2;
+    bool okc = cudaMemcpy(wr, router_w, (size_t)c.num_experts * H * 4, cudaMemcpyDeviceToDevice) == cudaSuccess &&
+               cudaMemcpy(w13s, w13_scales, Eall * 2 * I * (H / 32), cudaMemcpyDeviceToDevice) == cudaSuccess &&
+               cudaMemcpy(w2, w2_codes, Eall * H * (I / 2), cudaMemcpyDeviceToDevice) == cudaSuccess &&
+               cudaMemcpy(w2s, w2_scales, Eall * H * (I / 32), cudaMemcpyDeviceToDevice) == cudaSuccess;
+    if (okc && ctx->variant == kTc) {
+      moe::k_repack_w13<<<ctx->sm_count * 8, 256>>>(w13_codes, w13, (int)Eall, (int)H, (int)I);
+      okc = cudaGetLastError() == cudaSuccess && cudaDeviceSynchronize() == cudaSuccess;
+      ctx->tws.repacked = 1;
+    } else if (okc) {
+      okc = cudaMemcpy(w13, w13_codes, Eall * 2 * I * (H / 2), cudaMemcpyDeviceToDevice) == cudaSuccess &&
+            cudaDeviceSynchronize() == cudaSuccess;
+    }
+    if (!okc) {
+      cudaGetLastError();
+      cudaFree(ctx->owned);
+      ctx->owned = nullptr;
+      ctx->tws.repacked = 0;
+      return MOE_ERR_CUDA;
+    }
+    router_w = wr;
+    w13_codes = w13;
+    w13_scales = w13s;
+    w2_codes = w2;
+    w2_scales = w2s;
+  }
   if (ctx->variant == kTc) {
-    const size_t Eall = c.num_experts + ((c.flags & MOE_FLAG_SHARED_EXPERT) ? 1 : 0);
-    if (!encode_w13_maps(w13_codes, Eall, c.hidden, c.inter, ctx->tplan.ks, ctx->maps.m)) return MOE_ERR_INVALID_ARG;
+    const bool enc_ok = ctx->tws.repacked
+                            ? encode_w13_maps_repacked(w13_codes, Eall, H, I, ctx->tplan.ks, ctx->maps.m)
+                            : encode_w13_maps(w13_codes, Eall, H, I, ctx->tplan.ks, ctx->maps.m);
+    if (!enc_ok) return MOE_ERR_INVALID_ARG;
   }
   ctx->wr = router_w;
   ctx->w13c = w13_codes;
@@ -612,7 +692,7 @@ moe_status moe_plan_query(const moe_config* cfg, int32_t sm_count, size_t smem_l
                          "\"o_sfb\": %d, \"o_ring_d\": %d, \"o_h\": %d, \"o_bar\": %d, \"o_misc\": %d, "
                          "\"o_ids\": %d, \"o_w\": %d, \"o_pm\": %d, \"o_ppos\": %d, \"o_union\": %d, "
                          "\"o_poff\": %d, \"o_dsm\": %d, \"sc_bytes\": %d, \"bx_bytes\": %d, "
-                         "\"max_pairs\": %d, \"max_union\": %d, \"o_lg\": %d, \"tmem_cols\": %d}}",
+                         "\"max_pairs\": %d, \"max_union\": %d, \"o_lg\": %d, \"tmem_cols\": %d, \"lg_own\": %d}}",
                          (tc || ok) ? "true" : "false", tc ? "tc" : "fused", pl.G, moe::kFusedThreads, pl.smem_bytes,
                          pl.slot_gu, pl.ns_gu, pl.slot_d, pl.ns_d, pl.rpc_max, pl.wr_bytes_max, pl.o_act, pl.o_dsm,
                          pl.o_ring_gu, pl.o_ring_d, pl.o_h, pl.hslot, pl.hpairs, pl.x_staged, tok ? "true" : "false",
@@ -620,7 +700,7 @@ moe_status moe_plan_query(const moe_config* cfg, int32_t sm_count, size_t smem_l
                          tp.ns_d, tp.slot_d, tp.rpc_max, tp.hslot, tp.hpairs, tp.wr_bytes_max, tp.x_staged,
                          tp.o_ring_gu, tp.o_bx, tp.o_sf, tp.o_sc, tp.o_sfb, tp.o_ring_d, tp.o_h, tp.o_bar, tp.o_misc,
                          tp.o_ids, tp.o_w, tp.o_pm, tp.o_ppos, tp.o_union, tp.o_poff, tp.o_dsm, tp.sc_bytes,
-                         tp.bx_bytes, tp.max_pairs, tp.max_union, tp.o_lg, tp.tmem_cols);
+                         tp.bx_bytes, tp.max_pairs, tp.max_union, tp.o_lg, tp.tmem_cols, tp.lg_own);
   if (n < 0 || (size_t)n >= len) return MOE_ERR_INVALID_ARG;
   return (tc || ok) ? MOE_OK : MOE_ERR_UNSUPPORTED;
 }

@@ -80,6 +80,8 @@ struct TcPlan {
   int wr_bytes_max;
   int x_staged;  // bf16 x fits in the down ring during routing
   int o_lg;      // gathered logits [maxM][E] fp32, then [E] union scratch (routing only)
+  int o_hready;  // [max_union] entry's h complete on every CTA (set by the gatekeeper warp)
+  int lg_own;    // o_lg is a region of its own (not in either ring)
   // shared-memory offsets from the 1024-aligned base
   int o_ring_gu, o_bx, o_sf, o_sc, o_ring_d, o_h, o_bar, o_misc, o_ids, o_w, o_pm, o_ppos, o_union, o_poff, o_dsm,
       o_sfb;
@@ -89,8 +91,10 @@ struct TcPlan {
   int smem_bytes;  // including 1 KB of alignment slack
 };
 
-constexpr int kTcCntStride = 8;  // u32 words between per-entry counters (32 bytes)
-constexpr int kTcTrace = 48;     // timestamps per CTA in the optional trace
+constexpr int kTcCntStride = 32;  // u32 words between per-entry counters (one 128-byte line each)
+constexpr int kTcMaxTiles = 64;   // gate/up tiles per CTA
+constexpr int kTcWarpGate = 3;    // polls the entry counters for the CTA
+constexpr int kTcTrace = 64;     // timestamps per CTA in the optional trace
 
 // The gate/up code maps, passed by value as a __grid_constant__ kernel
 // parameter (TMA reads its descriptor from parameter space).
@@ -99,9 +103,10 @@ struct TcMaps {
 };
 
 struct TcWs {
+  int repacked;                // gate/up codes in the private [E][I/4][H/128][8][64 B] layout (4-D maps)
   unsigned long long* logits;  // [maxM][E]  epoch << 32 | fp32 bits
   float* h;                    // [pairs][I] SwiGLU output per (token, slot) pair
-  unsigned* hcnt;              // [2][max_union * kTcCntStride] tiles done per entry, by launch parity
+  unsigned* hcnt;              // [2][max_union * kTcCntStride] gate/up tiles done per entry, by launch parity
   unsigned* epoch;             // launch counter
 };
 
@@ -121,12 +126,24 @@ __device__ __forceinline__ void red_release_add_u32(unsigned* p, unsigned v) {
   asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
+// try_wait without a suspend-time hint: the hardware's own short limit, so a
+// waiter on the stream's critical path resumes as soon as the phase completes.
+__device__ __forceinline__ bool mbar_try_wait_fast(uint64_t* bar, unsigned parity) {
+  uint32_t ok;
+  asm volatile(
+      "{.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;}"
+      : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+  return ok != 0;
+}
+
 // Bounded wait on an mbarrier phase; false (and the status word set) if the
 // wait ran out.
 __device__ __forceinline__ bool mbar_wait_ok(uint64_t* bar, unsigned parity, const Params& p) {
-  if (mbar_try_wait(bar, parity)) return true;
+  if (mbar_try_wait_fast(bar, parity)) return true;
   const long long t0 = clock64();
-  while (!mbar_try_wait(bar, parity)) {
+  while (!mbar_try_wait_fast(bar, parity)) {
     if (clock64() - t0 > p.spin_limit) {
       atomicOr(p.ws.ctrl, kStatusTimeout);
       return false;
@@ -209,6 +226,14 @@ __device__ __forceinline__ void tma_load_5d(void* dst, const CUtensorMap* map, i
       "l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4), "r"(smem_u32(bar))
       : "memory");
 }
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, int c0, int c1, int c2, int c3,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], "
+      "[%6];" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar))
+      : "memory");
+}
 __device__ __forceinline__ void prefetch_tensormap(const void* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
 }
@@ -232,14 +257,19 @@ __device__ __forceinline__ uint32_t sw128_offset(int r, int k, int groups) {
   return (uint32_t)(kc * groups * 1024 + (r >> 3) * 1024 + rr * 128 + ((((col >> 4) ^ rr) & 7) << 4) + (col & 15));
 }
 
-// Poll an entry's completion counter (one lane, acquire) until it reaches
-// `target`; the warp gets one verdict.
-__device__ __forceinline__ bool tc_wait_count(const Params& p, const unsigned* cnt, unsigned target) {
+// Wait (one lane, acquire at CTA scope) until a shared-memory flag is set;
+// the warp gets one verdict.
+__device__ __forceinline__ unsigned ld_acquire_cta_smem(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
+  return v;
+}
+__device__ __forceinline__ bool tc_wait_flag(const Params& p, const unsigned* flag) {
   bool ok = true;
-  if ((threadIdx.x & 31) == 0 && ld_acquire_u32g(cnt) < target) {
+  if ((threadIdx.x & 31) == 0 && ld_acquire_cta_smem(flag) == 0u) {
     const long long t0 = clock64();
-    while (ld_acquire_u32g(cnt) < target) {
-      __nanosleep(64);
+    while (ld_acquire_cta_smem(flag) == 0u) {
+      __nanosleep(32);
       if (clock64() - t0 > p.spin_limit) {
         atomicOr(p.ws.ctrl, kStatusTimeout);
         ok = false;
@@ -256,7 +286,7 @@ __device__ __forceinline__ bool tc_wait_count(const Params& p, const unsigned* c
 // quantisation) comes from the warp maximum of those values.
 template <bool kFp8H>
 __device__ __forceinline__ void tc_d_item(const Params& p, const TcWs& tw, const DChunk& ch, int a, int cnt, int pb,
-                                          int pe, float* dsm, int rpc) {
+                                          int pe, float* dsm, int rpc, int trace_base = -1) {
   const int lane = threadIdx.x & 31;
   const int I = p.I, nblk = I / 32;
   for (int pp = pb; pp < pe; ++pp) {
@@ -272,6 +302,7 @@ __device__ __forceinline__ void tc_d_item(const Params& p, const TcWs& tw, const
         mx = fmaxf(mx, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
       }
       mx = warp_max(mx);
+      if (trace_base >= 0) tc_trace(p, trace_base);
       uint32_t h2[16];
       float down;
       if constexpr (kFp8H) {
@@ -289,8 +320,10 @@ __device__ __forceinline__ void tc_d_item(const Params& p, const TcWs& tw, const
           h2[q] = *reinterpret_cast<uint32_t*>(&hh);
         }
       }
+      if (trace_base >= 0) tc_trace(p, trace_base + 1);
       d_rows(p, ch, a, cnt, lane, h2, down, dsm + (size_t)pp * rpc, true);
       __syncwarp();
+      if (trace_base >= 0) tc_trace(p, trace_base + 2);
     } else {
       // wide intermediate: the maximum first, then block by block
       float mx = 0.f;
@@ -341,15 +374,21 @@ __device__ __forceinline__ float fkey_value(unsigned k) {
 
 // Top-k (K <= 8) of one token's E <= 512 logits with every warp of the CTA:
 // warp w first takes the K best of experts 32w..32w+31 (one per lane; ties
-// to the lower lane, i.e. the lower expert), then warp 0 merges the
-// candidates (ties to the lower expert) and forms the softmax over the K
-// kept. Same result as topk_warp; all threads must call it.
+// to the lower lane, i.e. the lower expert); then every candidate's rank
+// among all of them is counted in parallel (larger logit first, ties to the
+// lower expert), and warp 0 forms the softmax over the K kept. Same result
+// as topk_warp; all threads must call it. s_ck, s_ce: 136 words each
+// (W*8 <= 128 candidates, then the K results).
 __device__ void topk_cta_small(const float* l, int E, int K, int* ids, float* wts, unsigned* s_ck, int* s_ce) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int W = (E + 31) / 32;
   if (warp < W) {
     const int e = 32 * warp + lane;
     unsigned key = (e < E) ? fkey(l[e]) : 0u;
+    if (lane < 8 && lane >= K) {
+      s_ck[warp * 8 + lane] = 0u;
+      s_ce[warp * 8 + lane] = 0x7fffffff;
+    }
     for (int r = 0; r < K; ++r) {
       const unsigned mx = __reduce_max_sync(0xffffffffu, key);
       const int win = __ffs(__ballot_sync(0xffffffffu, key == mx)) - 1;
@@ -361,41 +400,57 @@ __device__ void topk_cta_small(const float* l, int E, int K, int* ids, float* wt
     }
   }
   __syncthreads();
-  if (warp == 0) {
-    unsigned ck[4];
-    int ce[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int c = lane + 32 * j, w = c / K, r = c - w * K;
-      const bool v = c < W * K;
-      ck[j] = v ? s_ck[w * 8 + r] : 0u;
-      ce[j] = v ? s_ce[w * 8 + r] : 0x7fffffff;
-    }
-    float sel_v = 0.f, top = 0.f;
-    int sel_i = 0;
-    for (int r = 0; r < K; ++r) {
-      unsigned bk = 0u;
-      int be = 0x7fffffff, bj = 0;
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-        if (ck[j] > bk || (ck[j] == bk && ce[j] < be)) { bk = ck[j]; be = ce[j]; bj = j; }
-      const unsigned mx = __reduce_max_sync(0xffffffffu, bk);
-      const int emin = (int)__reduce_min_sync(0xffffffffu, (unsigned)((bk == mx) ? be : 0x7fffffff));
-      if (bk == mx && be == emin) {
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          if (j == bj) ck[j] = 0u;
+  // merge: the rank of candidate c among all W*8 slots (larger key first,
+  // then the lower expert), four threads per candidate, each counting over a
+  // quarter; ranks below K are the result, in order
+  {
+    const int c = threadIdx.x >> 2, part = threadIdx.x & 3, nc = W * 8;
+    int rank = 0;
+    unsigned kc = 0u;
+    int ec = 0x7fffffff;
+    if (c < nc) {
+      kc = s_ck[c];
+      ec = s_ce[c];
+      for (int d = part; d < nc; d += 4) {
+        const unsigned kd = s_ck[d];
+        const int ed = s_ce[d];
+        rank += (kd > kc) || (kd == kc && ed < ec);
       }
-      const float v = fkey_value(mx);
-      if (r == 0) top = v;
-      if (lane == r) { sel_v = v; sel_i = emin; }
     }
-    const float ex = (lane < K) ? expf(sel_v - top) : 0.f;
+    rank += __shfl_xor_sync(0xffffffffu, rank, 1);
+    rank += __shfl_xor_sync(0xffffffffu, rank, 2);
+    __syncthreads();
+    if (c < nc && part == 0 && kc != 0u && rank < K) {
+      s_ck[128 + rank] = kc;
+      s_ce[128 + rank] = ec;
+    }
+    __syncthreads();
+  }
+  if (warp == 0) {
+    const float top = fkey_value(s_ck[128]);
+    const float v = (lane < K) ? fkey_value(s_ck[128 + lane]) : 0.f;
+    const float ex = (lane < K) ? expf(v - top) : 0.f;
     const float z = warp_sum(ex);
     if (lane < K) {
-      ids[lane] = sel_i;
+      ids[lane] = s_ce[128 + lane];
       wts[lane] = ex / z;
     }
+  }
+}
+
+// Re-tiles gate/up codes [Eall][2I][H/2] into [Eall][I/4][H/128][8][64 B]:
+// block (e, j, c) holds rows 4j..4j+3 (gate) and I+4j..I+4j+3 (up) of
+// expert e, 64 bytes (128 codes) of K-chunk c each. 16 bytes per thread.
+__global__ void k_repack_w13(const uint8_t* __restrict__ src, uint8_t* __restrict__ dst, int Eall, int H, int I) {
+  const size_t KCH = H / 128, upe = I / 4;
+  const size_t total = (size_t)Eall * upe * KCH * 32;
+  for (size_t idx = blockIdx.x * (size_t)blockDim.x + threadIdx.x; idx < total; idx += (size_t)gridDim.x * blockDim.x) {
+    const size_t piece = idx & 31, blk = idx >> 5;
+    const size_t c = blk % KCH, u = blk / KCH, e = u / upe, j = u % upe;
+    const size_t i = piece >> 2, qq = piece & 3;
+    const size_t row = e * 2 * I + (i < 4 ? 4 * j + i : I + 4 * j + (i - 4));
+    const uint4 v = *reinterpret_cast<const uint4*>(src + row * (H / 2) + c * 64 + qq * 16);
+    *reinterpret_cast<uint4*>(dst + blk * 512 + i * 64 + qq * 16) = v;
   }
 }
 
@@ -431,6 +486,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc(Params p, TcWs tw, TcPlan 
   float* s_rn = s_xs + kMaxTokens;                             // [32]
   float* s_red = s_rn + kMaxTokens;                            // [kTcWarps][kMaxRowsPerCta * 4]
   int* s_int = reinterpret_cast<int*>(s_red + kTcWarps * kMaxRowsPerCta * 4);  // [0] U [1] epoch [2] queue [3] tmem
+  unsigned* s_tdone = reinterpret_cast<unsigned*>(s_int + 8);                  // [kTcMaxTiles] epilogue warps done
+  unsigned* s_hready = reinterpret_cast<unsigned*>(smem + pl.o_hready);         // [max_union]
   int* s_ids = reinterpret_cast<int*>(smem + pl.o_ids);
   float* s_w = reinterpret_cast<float*>(smem + pl.o_w);
   int* s_pm = reinterpret_cast<int*>(smem + pl.o_pm);
@@ -507,6 +564,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc(Params p, TcWs tw, TcPlan 
   }
   unsigned* s_amax_u = reinterpret_cast<unsigned*>(s_amax);
   if (tid < M) s_amax_u[tid] = 0u;
+  if (tid < kTcMaxTiles) s_tdone[tid] = 0u;
+  for (int i = tid; i < pl.max_union; i += kTcThreads) s_hready[i] = 0u;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -598,10 +657,54 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc(Params p, TcWs tw, TcPlan 
     }
     __syncthreads();
   }
-  // ---- A2: logits of the CTA's router rows, four tokens per pass
+  // ---- A2: logits of the CTA's router rows
   if (ne > 0 && !mbar_wait_ok(wr_bar, 0, p)) ok = false;
   tc_trace(p, 14);
-  for (int m0 = 0; m0 < M && ne > 0; m0 += 4) {
+  if (M == 1 && ne > 0 && ne <= 2) {
+    // one token: every thread takes a strided share of both rows at once;
+    // warp sums, then warp 0 sums the warps' partials
+    float acc0 = 0.f, acc1 = 0.f;
+    for (int i = tid; i < H / 8; i += kTcThreads) {
+      const uint4 x8 = ld_x8(i);
+      const uint32_t xw[4] = {x8.x, x8.y, x8.z, x8.w};
+      const float4* w0 = reinterpret_cast<const float4*>(wr_s) + 2 * i;
+      const float4 a0 = w0[0], a1 = w0[1];
+      const float4 b0 = (ne > 1) ? w0[H / 4] : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float4 b1 = (ne > 1) ? w0[H / 4 + 1] : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float2 x0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xw[0]));
+      const float2 x1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xw[1]));
+      const float2 x2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xw[2]));
+      const float2 x3 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xw[3]));
+      acc0 = fmaf(x0.x, a0.x, acc0); acc0 = fmaf(x0.y, a0.y, acc0); acc0 = fmaf(x1.x, a0.z, acc0);
+      acc0 = fmaf(x1.y, a0.w, acc0); acc0 = fmaf(x2.x, a1.x, acc0); acc0 = fmaf(x2.y, a1.y, acc0);
+      acc0 = fmaf(x3.x, a1.z, acc0); acc0 = fmaf(x3.y, a1.w, acc0);
+      acc1 = fmaf(x0.x, b0.x, acc1); acc1 = fmaf(x0.y, b0.y, acc1); acc1 = fmaf(x1.x, b0.z, acc1);
+      acc1 = fmaf(x1.y, b0.w, acc1); acc1 = fmaf(x2.x, b1.x, acc1); acc1 = fmaf(x2.y, b1.y, acc1);
+      acc1 = fmaf(x3.x, b1.z, acc1); acc1 = fmaf(x3.y, b1.w, acc1);
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+      acc0 += __shfl_xor_sync(0xffffffffu, acc0, o);
+      acc1 += __shfl_xor_sync(0xffffffffu, acc1, o);
+    }
+    if (lane == 0) {
+      s_red[warp] = acc0;
+      s_red[kTcWarps + warp] = acc1;
+    }
+    __syncthreads();
+    if (warp == 0) {
+      float v0 = (lane < kTcWarps) ? s_red[lane] : 0.f;
+      float v1 = (lane < kTcWarps) ? s_red[kTcWarps + lane] : 0.f;
+#pragma unroll
+      for (int o = kTcWarps / 2; o; o >>= 1) {
+        v0 += __shfl_xor_sync(0xffffffffu, v0, o);
+        v1 += __shfl_xor_sync(0xffffffffu, v1, o);
+      }
+      if (lane == 0) st_relaxed_u64(tw.logits + e0, tag_word(epoch, v0));
+      if (lane == 1 && ne > 1) st_relaxed_u64(tw.logits + e0 + 1, tag_word(epoch, v1));
+    }
+  }
+  for (int m0 = 0; m0 < M && ne > 0 && !(M == 1 && ne <= 2); m0 += 4) {
     const int mt = min(4, M - m0);
     for (int el = 0; el < ne; ++el) {
       float acc[4] = {0.f, 0.f, 0.f, 0.f};
@@ -694,6 +797,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc(Params p, TcWs tw, TcPlan 
     for (int i = tid; i < M * E; i += kTcThreads) {
       unsigned long long w = ld_relaxed_u64(tw.logits + i);
       while ((unsigned)(w >> 32) != want) {
+        __nanosleep(32);
         if (clock64() - t0 > p.spin_limit) {
           atomicOr(p.ws.ctrl, kStatusTimeout);
           ok = false;
@@ -712,7 +816,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc(Params p, TcWs tw, TcPlan 
   //      else one warp per token
   if (M == 1 && E <= 32 * kTcWarps && K <= 8) {
     topk_cta_small(s_logit, E, K, s_ids, s_w, reinterpret_cast<unsigned*>(s_red),
-                   reinterpret_cast<int*>(s_red) + kTcWarps * 8);
+                   reinterpret_cast<int*>(s_red) + 136);
     if (b == 0 && tid < K) {
       if (p.out_ids) p.out_ids[tid] = s_ids[tid];
       if (p.out_w) p.out_w[tid] = s_w[tid];
@@ -739,7 +843,22 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc(Params p, TcWs tw, TcPlan 
 
   // ---- A4: union (ascending ids) and the pairs of each entry in (token, slot) order
   const int np = M * K, pbase = kShared ? M : 0;
-  if (warp == 0 && np <= 32) {
+  if (M == 1) {
+    // one token: its K distinct experts, sorted; each entry has one pair
+    if (tid < K) {
+      const int id = s_ids[tid];
+      int rank = 0;
+      for (int j = 0; j < K; ++j) rank += s_ids[j] < id;
+      s_union[ub + rank] = id;
+      s_poff[ub + rank] = pbase + rank;
+      s_pm[pbase + rank] = 0;
+      s_ppos[tid] = pbase + rank;
+      if (rank == K - 1) {
+        s_poff[ub + K] = pbase + K;
+        s_int[0] = ub + K;
+      }
+    }
+  } else if (warp == 0 && np <= 32) {
     const int Us = union_small(s_ids, np, K, s_union + ub, s_poff + ub, s_pm, s_ppos, pbase);
     if (lane == 0) s_int[0] = ub + Us;
   } else if (warp == 0) {
@@ -792,8 +911,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc(Params p, TcWs tw, TcPlan 
     }
   }
   // ring_gu and ring_d held routing scratch (generic proxy): order that
-  // before the TMA writes into them
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  // before the TMA writes into them (not needed when the only generic
+  // accesses to them were the router-row and staged-x reads before the
+  // activation codes' fence)
+  if (!pl.lg_own) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   // one verdict for the CTA: after a routing wait ran out, no role starts
   ok = __syncthreads_and(ok ? 1 : 0) != 0;
   const int U = s_int[0];
@@ -827,11 +948,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc(Params p, TcWs tw, TcPlan 
         uint8_t* sc = scbuf + (size_t)sb * scb;
         // the tile's runs of units of one expert: at most 2 (a tile has at
         // most 16 units and an entry I/4 >= 32)
-        int rcoord[2], rn[2], rg[2], nrun = 0;
+        int rcoord[2], runit[2], rn[2], rg[2], nrun = 0;
         for (int f = f0; f < f1 && nrun < 2;) {
           const int u = f / upe, j = f % upe, n = min(f1 - f, upe - j);
           const int e = s_union[u];
-          rcoord[nrun] = e * (I / 2) + j;
+          rcoord[nrun] = e * (I / 2) + j;  // 5-D map: quad of gate rows 4j.. of expert e
+          runit[nrun] = e * upe + j;       // 4-D map over the re-tiled copy: unit j of expert e
           rn[nrun] = n;
           rg[nrun] = f - f0;
           ++nrun;
@@ -840,8 +962,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc(Params p, TcWs tw, TcPlan 
         if (it >= 2 && !mbar_wait_ok(sc_empty + sb, ((it >> 1) - 1) & 1, p)) { ok = false; break; }
         mbar_expect_tx(sc_full + sb, (unsigned)(8 * nu * (H / 32)));
         for (int r = 0; r < nrun; ++r) {
-          const int e = rcoord[r] / (I / 2), j = rcoord[r] % (I / 2);
-          const size_t grow = (size_t)e * 2 * I + 4 * j;
+          const size_t grow = (size_t)4 * rcoord[r];  // gate row 4j of expert e: 4 * (e*I/2 + j)
           tma_load_1d(sc + (size_t)4 * rg[r] * (H / 32), p.w13s + grow * (H / 32), (unsigned)(4 * rn[r] * (H / 32)),
                       sc_full + sb);
           tma_load_1d(sc + (size_t)(4 * pl.tu_max + 4 * rg[r]) * (H / 32), p.w13s + (grow + I) * (H / 32),
@@ -850,11 +971,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc(Params p, TcWs tw, TcPlan 
         const unsigned bytes = (unsigned)(nu * ks * 512);
         for (int k = 0; k < nstage; ++k, ++stage) {
           if (reuse && !mbar_wait_ok(empty_gu + slot, ph ^ 1u, p)) { ok = false; break; }
+          if (stage >= pl.ns_gu && stage < pl.ns_gu + 4) tc_trace(p, 42 + stage - pl.ns_gu);
           mbar_expect_tx(full_gu + slot, bytes);
           tc_trace(p, 32 + stage);
           uint8_t* dst = ring_gu + (size_t)slot * pl.slot_gu;
-          for (int r = 0; r < nrun; ++r)
-            tma_load_5d(dst + (size_t)rg[r] * ks * 1024, &maps.m[rn[r] - 1], 0, 0, 0, k * ks, rcoord[r], full_gu + slot);
+          for (int r = 0; r < nrun; ++r) {
+            if (tw.repacked)
+              tma_load_4d(dst + (size_t)rg[r] * ks * 1024, &maps.m[rn[r] - 1], 0, 0, k * ks, runit[r], full_gu + slot);
+            else
+              tma_load_5d(dst + (size_t)rg[r] * ks * 1024, &maps.m[rn[r] - 1], 0, 0, 0, k * ks, rcoord[r],
+                          full_gu + slot);
+          }
           if (++slot == pl.ns_gu) { slot = 0; ph ^= 1u; reuse = true; }
         }
       }
@@ -896,6 +1023,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc(Params p, TcWs tw, TcPlan 
           }
           tc_commit(empty_gu + slot);
           if (k == nstage - 1) tc_commit(acc_full + buf);
+          if (stage < 4) tc_trace(p, 26 + stage);
         }
         __syncwarp();
         if (++slot == pl.ns_gu) { slot = 0; ph ^= 1u; }
@@ -922,8 +1050,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc(Params p, TcWs tw, TcPlan 
         const unsigned codes = (unsigned)(nrd * I / 2);
         tma_load_1d(sp, p.w2c + ((size_t)e * H + r0) * (I / 2), codes, full_d + slot);
         tma_load_1d(sp + codes, p.w2s + sa0, sn, full_d + slot);
+        if (u == 0) tc_trace(p, 59);
         if (++slot == pl.ns_d) { slot = 0; ph ^= 1u; reuse = true; }
       }
+      tc_trace(p, 60);
     }
   }
 
@@ -976,6 +1106,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc(Params p, TcWs tw, TcPlan 
       const int f0 = t * tu, f1 = min(T, f0 + tu), nu = f1 - f0;
       const int buf = it & 1;
       if (!mbar_wait_warp(acc_full + buf, (it >> 1) & 1, p)) { ok = false; break; }
+      if (q == 0 && it == my_tiles - 1) tc_trace(p, 48);
       tc_fence_after();
       uint32_t v[32];
       tmem_ld32(tmem + (uint32_t)(buf * kTcAccCols) + ((uint32_t)(32 * q) << 16), v);
@@ -1002,18 +1133,49 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc(Params p, TcWs tw, TcPlan 
           tw.h[(size_t)pp * I + n] = gv / (1.f + expf(-gv)) * uv;
         }
       }
-      // publish: each of the four warps counts once per entry the tile
-      // touches, after its own stores (release at GPU scope)
+      // publish: the last of the four warps to finish the tile (CTA-scope
+      // acq_rel counter, so it sees the others' stores) adds one to the
+      // counter of every entry the tile touches, with release at GPU scope
       __syncwarp();
-      if (lane == 0)
+      if (q == 0 && it == my_tiles - 1) tc_trace(p, 49);
+      if (lane == 0 && atom_add_acqrel_cta_smem(s_tdone + it, 1u) == 3u)
         for (int u = f0 / upe; u <= (f1 - 1) / upe; ++u) red_release_add_u32(hcnt + u * kTcCntStride, 1u);
+      if (q == 0 && it == my_tiles - 1) tc_trace(p, 50);
     }
     tc_trace(p, 7);
   }
 
+  // ---------------- gatekeeper: one thread polls the entry counters in
+  //   order (acquire, GPU scope) and raises each entry's flag in shared
+  //   memory (release, CTA scope) once every tile covering it has published
+  //   its h; the down items wait on the flags. One poller per CTA keeps the
+  //   counters' L2 lines cool.
+  if (warp == kTcWarpGate && lane == 0) {
+    const long long t0 = clock64();
+    for (int u = 0; u < U && ok; ++u) {
+      const unsigned tiles = (unsigned)(((u + 1) * upe - 1) / tu - (u * upe) / tu + 1);
+      const unsigned* c = hcnt + u * kTcCntStride;
+      while (ld_acquire_u32g(c) < tiles) {
+        __nanosleep(128);
+        if (clock64() - t0 > p.spin_limit) {
+          atomicOr(p.ws.ctrl, kStatusTimeout);
+          ok = false;
+          break;
+        }
+      }
+      asm volatile("st.release.cta.shared::cta.u32 [%0], %1;" ::"r"(smem_u32(s_hready + u)), "r"(1u) : "memory");
+      if (u == 0) tc_trace(p, 30);
+    }
+    tc_trace(p, 31);
+  }
+  if (warp == kTcWarpGate) {
+    __syncwarp();
+    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+  }
+
   // ---------------- down (CUDA cores): every warp once its role is done.
   //   Items (entry, 9 output rows) in entry order; each waits for its
-  //   entry's h on every CTA (the entry's counter) and its chunk.
+  //   entry's flag (h complete on every CTA) and its chunk.
   {
     const int per = d_items;
     const int total = U * per;
@@ -1030,17 +1192,23 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc(Params p, TcWs tw, TcPlan 
       // below cannot see an earlier phase
       if (use > 0 && lane == 0) smem_count_wait(done_d + slot, (unsigned)(use * per), p);
       __syncwarp();
-      // every tile covering entry u arrives from its 4 epilogue warps
-      const unsigned tiles = (unsigned)(((u + 1) * upe - 1) / tu - (u * upe) / tu + 1);
-      if (!tc_wait_count(p, hcnt + u * kTcCntStride, 4u * tiles)) ok = false;
+      if (it == 0) tc_trace(p, 51);
+      if (it == total - 1) tc_trace(p, 54);
+      if (!tc_wait_flag(p, s_hready + u)) ok = false;
       if (u == U - 1 && gd == 0) tc_trace(p, 9);
+      if (it == 0) tc_trace(p, 52);
+      if (it == total - 1) tc_trace(p, 55);
       if (!mbar_wait_warp(full_d + slot, use & 1, p)) ok = false;
+      if (it == 0) tc_trace(p, 53);
+      if (it == total - 1) tc_trace(p, 56);
       DChunk ch;
       size_t sa0;
       unsigned sn;
       d_layout(p, s_union[u], r0, nrd, ring_d + (size_t)slot * pl.slot_d, &ch, &sa0, &sn);
       const int a = gd * kDownRowsPerItem, cnt = min(kDownRowsPerItem, nrd - a);
-      tc_d_item<kFp8H>(p, tw, ch, a, cnt, pb, pe, dsm, pl.rpc_max);
+      tc_d_item<kFp8H>(p, tw, ch, a, cnt, pb, pe, dsm, pl.rpc_max, it == 0 ? 61 : -1);
+      if (it == 0) tc_trace(p, 57);
+      if (it == total - 1) tc_trace(p, 58);
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(empty_d + slot);

@@ -27,6 +27,7 @@ MOE_FLAG_TENSOR_CORES = 0x20
 MOE_TC_MIN_TOKENS = 2
 MOE_LOAD_BORROW = 0x0
 MOE_LOAD_SKIP_VALIDATE = 0x1
+MOE_LOAD_COPY_REPACK = 0x2
 
 
 class MoEError(RuntimeError):
@@ -143,14 +144,16 @@ class MoELayer:
             raise MoEError(st, "moe_create")
         self._weights = None
 
-    def load_experts(self, router_w, w13_codes, w13_scales, w2_codes, w2_scales, validate: bool = True):
-        """Borrow device tensors (kept referenced here so they outlive the context)."""
-        flags = 0 if validate else MOE_LOAD_SKIP_VALIDATE
+    def load_experts(self, router_w, w13_codes, w13_scales, w2_codes, w2_scales, validate: bool = True,
+                     repack: bool = False):
+        """Borrow device tensors (kept referenced here so they outlive the
+        context), or with repack=True let the context copy (and re-tile) them."""
+        flags = (0 if validate else MOE_LOAD_SKIP_VALIDATE) | (MOE_LOAD_COPY_REPACK if repack else 0)
         st = lib().moe_load_experts(self._ctx, _ptr(router_w), _ptr(w13_codes), _ptr(w13_scales),
                                     _ptr(w2_codes), _ptr(w2_scales), flags)
         if st != MOE_OK:
             raise MoEError(st, "moe_load_experts")
-        self._weights = (router_w, w13_codes, w13_scales, w2_codes, w2_scales)
+        self._weights = None if repack else (router_w, w13_codes, w13_scales, w2_codes, w2_scales)
 
     def decode_raw(self, x, M: int, y, stream=None, topk_ids=None, topk_w=None, xq=None, xscale=None,
                    xnorm=None) -> int:

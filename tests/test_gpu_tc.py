@@ -162,3 +162,33 @@ def test_back_to_back_and_graph_replay():
     for L, c, y in zip(Ls, ctxs, ys):
         assert c.sync_status() == moe.MOE_OK
         assert torch.equal(L.run(c)["y"], y)
+
+
+@pytest.mark.parametrize("shape,M,mode", [((2560, 768, 256, 8), 1, "gap"), ((2560, 768, 256, 8), 4, "natural"),
+                                          ((512, 256, 40, 6), 5, "gap")])
+def test_copy_repack_matches_borrowed(shape, M, mode):
+    """MOE_LOAD_COPY_REPACK: the context's re-tiled copy gives the same bits
+    as the borrowed weights (the MMAs see the same operands), matches the
+    oracle, and keeps working after the caller's arrays are overwritten."""
+    H, I, E, K = shape
+    L = Layer(H, I, E, K, M, seed=51, mode=mode)
+    a = L.run(_ctx(L))
+    ctx = moe.MoELayer(H, I, E, K, M, flags=moe.MOE_FLAG_TENSOR_CORES)
+    ctx.load_experts(L.wr_d, *L.experts, repack=True)
+    b = L.run(ctx)
+    assert torch.equal(a["y"], b["y"])
+    compare(L, b, L.oracle())
+    # the context owns its copy: clobbering the caller's arrays changes nothing
+    for t in L.experts:
+        t.zero_()
+    L.wr_d.zero_()
+    c = L.run(ctx)
+    assert torch.equal(b["y"], c["y"])
+
+
+def test_copy_repack_cuda_core_kernel():
+    L = Layer(2560, 768, 256, 8, 2, seed=52, mode="natural")
+    ctx = moe.MoELayer(2560, 768, 256, 8, 2, flags=moe.MOE_FLAG_CUDA_CORES)
+    ctx.load_experts(L.wr_d, *L.experts, repack=True)
+    got = L.run(ctx)
+    compare(L, got, L.oracle())
