@@ -403,8 +403,7 @@ moe_status moe_create(const moe_config* cfg, moe_ctx** out) {
   const size_t o_pslot = take(NP * sizeof(int));
   const size_t o_pw = take(NP * sizeof(float));
   const size_t o_h = take(NPF * I * sizeof(float));
-  const size_t o_flog = take(MM * E * sizeof(float));
-  const size_t o_rcnt = take(sizeof(unsigned long long));
+  const size_t o_flog = take(MM * E * sizeof(unsigned long long));
   const size_t o_gcnt = take(UMAXF * moe::kCounterStride * sizeof(unsigned long long));
   const size_t o_tlog = take(MM * E * sizeof(unsigned long long));
   const size_t o_th = take(NPF * I * sizeof(float));
@@ -435,8 +434,7 @@ moe_status moe_create(const moe_config* cfg, moe_ctx** out) {
   w.pair_slot = reinterpret_cast<int*>(b + o_pslot);
   w.pair_w = reinterpret_cast<float*>(b + o_pw);
   w.h = reinterpret_cast<float*>(b + o_h);
-  ctx->fws.logits = reinterpret_cast<float*>(b + o_flog);
-  ctx->fws.route_cnt = reinterpret_cast<unsigned long long*>(b + o_rcnt);
+  ctx->fws.logits = reinterpret_cast<unsigned long long*>(b + o_flog);
   ctx->fws.gu_cnt = reinterpret_cast<unsigned long long*>(b + o_gcnt);
   ctx->fws.epoch = w.ctrl + 5;
   ctx->tws.logits = reinterpret_cast<unsigned long long*>(b + o_tlog);
@@ -621,7 +619,7 @@ moe_status moe_decode(moe_ctx* ctx, const void* x_bf16, int32_t M, void* y_bf16,
   p.out_xscale = xscale;
   p.spin_limit = ctx->spin_limit;
   p.force_stall = ctx->force_stall;
-  p.trace = ctx->variant == kTc ? ctx->trace : nullptr;
+  p.trace = ctx->trace;
   p.pre_rmsnorm = (c.flags & MOE_FLAG_PRE_RMSNORM) ? 1 : 0;
   p.out_xn = static_cast<__nv_bfloat16*>(xnorm_bf16);
   cudaStream_t st = static_cast<cudaStream_t>(stream);

@@ -62,6 +62,17 @@ struct Params {
   __nv_bfloat16* out_xn; // optional [M][H] normalised input
 };
 
+// Test hook: lane 0 of the calling warp stores the global timer into stamp
+// `slot` of this CTA's row of the trace array (kTraceSlots stamps per CTA).
+constexpr int kTraceSlots = 64;
+__device__ __forceinline__ void trace_stamp(const Params& p, int slot) {
+  if (p.trace && (threadIdx.x & 31) == 0 && slot < kTraceSlots) {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    p.trace[(size_t)blockIdx.x * kTraceSlots + slot] = t;
+  }
+}
+
 // ---------------------------------------------------------------- formats
 // E8M0 scale byte -> fp32 2^(b-127) (exact; b = 0 is the subnormal 2^-127).
 // 0xFF (NaN) is rejected when the weights are loaded.

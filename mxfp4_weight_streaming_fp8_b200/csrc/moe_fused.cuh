@@ -52,6 +52,7 @@ namespace moe {
 constexpr int kFusedThreads = 512;
 constexpr int kFusedWarps = kFusedThreads / 32;
 constexpr int kConsumers = kFusedWarps - 1;  // warp 0 produces
+constexpr int kDownLag = 8;                 // down items of entry k follow the gate/up items of entry k + kDownLag
 constexpr int kGuRowsPerItem = 2;           // intermediate rows per gate/up item
 constexpr int kDownRowsPerItem = 9;         // output rows per down item (two items per expert at 17-18 rows per CTA)
 constexpr int kHPairs = 4;                  // (token, slot) pairs of one expert whose h is staged in smem
@@ -59,7 +60,6 @@ constexpr int kMaxRowsPerCta = 8;           // router rows a CTA may own (E <= 8
 constexpr int kMaxSlots = 64;
 constexpr int kMaxPairTiles = 4;            // 8-pair MMA column tiles per entry (32 pairs)
 constexpr int kMmaMinPairs = 3;             // entries with at least this many pairs take the MMA gate/up path
-constexpr int kDownLag = 8;                 // down items of entry k follow the gate/up items of entry k + kDownLag
 constexpr int kCounterStride = 16;          // u64 words between per-entry counters (one 128-byte line)
 
 // Launch-invariant plan computed on the host at moe_create.
@@ -82,8 +82,7 @@ struct FusedPlan {
 
 // Workspace pieces only the persistent kernel uses.
 struct FusedWs {
-  float* logits;                  // [maxM][E]
-  unsigned long long* route_cnt;  // router arrivals; += G per launch
+  unsigned long long* logits;     // [maxM][E] tagged router logits (epoch, fp32)
   unsigned long long* gu_cnt;     // [max_union][kCounterStride] gate/up arrivals per entry; += G per launch
   unsigned* epoch;                // launch counter
 };
@@ -227,6 +226,33 @@ __device__ __forceinline__ void grid_wait(const unsigned long long* cnt, unsigne
       return;
     }
   }
+}
+
+// CTA-scope release/acquire on a shared-memory word (a ready flag).
+__device__ __forceinline__ unsigned ld_acquire_cta_smem(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_cta_smem(unsigned* p, unsigned v) {
+  asm volatile("st.release.cta.shared::cta.u32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
+}
+// Whole warp: wait (lane 0 polls, bounded) until a shared-memory flag is set;
+// false, with the status bit set, when the wait ran out.
+__device__ __forceinline__ bool wait_flag_warp(const Params& p, const unsigned* flag) {
+  bool ok = true;
+  if ((threadIdx.x & 31) == 0 && ld_acquire_cta_smem(flag) == 0u) {
+    const long long t0 = clock64();
+    while (ld_acquire_cta_smem(flag) == 0u) {
+      __nanosleep(32);
+      if (clock64() - t0 > p.spin_limit) {
+        atomicOr(p.ws.ctrl, kStatusTimeout);
+        ok = false;
+        break;
+      }
+    }
+  }
+  return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 
 // Wait (one thread) until a shared-memory count reaches `target`.
@@ -715,6 +741,191 @@ __device__ __forceinline__ void topk_warp(const float* l, int E, int K, int* ids
   }
 }
 
+// Router logit exchange word: the launch's epoch in the high half, the fp32
+// logit in the low half. A reader that sees its own epoch has the value of
+// this launch (one 64-bit store is single-copy atomic), so the word is its
+// own ready flag.
+__device__ __forceinline__ unsigned long long tag_word(unsigned epoch, float v) {
+  return ((unsigned long long)epoch << 32) | __float_as_uint(v);
+}
+
+// Order-preserving 32-bit image of a float, and back.
+__device__ __forceinline__ unsigned fkey(float v) {
+  const unsigned u = __float_as_uint(v);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float fkey_value(unsigned k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
+// Top-k (K <= 8) of one token's E <= 512 logits with every warp of the CTA.
+// Order: larger logit first, ties to the lower expert. Warp w ranks experts
+// 32w..32w+31 among themselves (each lane counts the keys ahead of its own
+// over the warp's shuffles) and keeps its K best; then every kept candidate
+// counts the candidates ahead of it over all warps (several threads per
+// candidate), and the K of rank < K are the result in order; warp 0 forms
+// the softmax over them. Same result as topk_warp; all threads must call it.
+// s_ck, s_ce: 136 words each (W*8 <= 128 candidates, then the K results).
+__device__ void topk_cta_small(const float* l, int E, int K, int* ids, float* wts, unsigned* s_ck, int* s_ce,
+                               const Params& p_trace) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int W = (E + 31) / 32;
+  if (warp < W) {
+    const int e = 32 * warp + lane;
+    const unsigned key = (e < E) ? fkey(l[e]) : 0u;  // 0 is below every float's key
+    int rank = 0;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const unsigned kj = __shfl_sync(0xffffffffu, key, j);
+      rank += (kj > key) || (kj == key && j < lane);
+    }
+    if (rank < 8) {
+      const bool keep = rank < K && key != 0u;
+      s_ck[warp * 8 + rank] = keep ? key : 0u;
+      s_ce[warp * 8 + rank] = keep ? e : 0x7fffffff;
+    }
+  }
+  trace_stamp(p_trace, 46);
+  __syncthreads();
+  {
+    const int nc = W * 8, tpc = (nc <= 64) ? 8 : 4;  // threads per candidate
+    const int c = threadIdx.x / tpc, part = threadIdx.x % tpc;
+    int rank = 0;
+    unsigned kc = 0u;
+    int ec = 0x7fffffff;
+    if (c < nc) {
+      kc = s_ck[c];
+      ec = s_ce[c];
+      for (int d = part; d < nc; d += tpc) {
+        const unsigned kd = s_ck[d];
+        const int ed = s_ce[d];
+        rank += (kd > kc) || (kd == kc && ed < ec);
+      }
+    }
+    for (int o = 1; o < tpc; o <<= 1) rank += __shfl_xor_sync(0xffffffffu, rank, o);
+    __syncthreads();
+    if (c < nc && part == 0 && kc != 0u && rank < K) {
+      s_ck[128 + rank] = kc;
+      s_ce[128 + rank] = ec;
+    }
+    __syncthreads();
+  }
+  trace_stamp(p_trace, 47);
+  if (warp == 0) {
+    const float top = fkey_value(s_ck[128]);
+    const float v = (lane < K) ? fkey_value(s_ck[128 + lane]) : 0.f;
+    const float ex = (lane < K) ? expf(v - top) : 0.f;
+    const float z = warp_sum(ex);
+    if (lane < K) {
+      ids[lane] = s_ce[128 + lane];
+      wts[lane] = ex / z;
+    }
+  }
+}
+
+// Logits of this CTA's ne <= 2 router rows (wr_s, fp32, row-major) for one
+// token: every thread takes a strided share of both rows; warp sums, then
+// warp 0 sums the warps' partials in warp order and stores the tagged words
+// out[0], out[1]. ld_x8(i) returns bf16 elements 8i..8i+7 of the token.
+// s_red: 2 * (blockDim.x / 32) floats. All threads must call it.
+template <class LdX8>
+__device__ __forceinline__ void router_logits_m1(LdX8 ld_x8, const float* wr_s, int H, int ne, unsigned epoch,
+                                                 unsigned long long* out, float* s_red) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
+  float acc0 = 0.f, acc1 = 0.f;
+  for (int i = tid; i < H / 8; i += blockDim.x) {
+    const uint4 x8 = ld_x8(i);
+    const uint32_t xw[4] = {x8.x, x8.y, x8.z, x8.w};
+    const float4* w0 = reinterpret_cast<const float4*>(wr_s) + 2 * i;
+    const float4 a0 = w0[0], a1 = w0[1];
+    const float4 b0 = (ne > 1) ? w0[H / 4] : make_float4(0.f, 0.f, 0.f, 0.f);
+    const float4 b1 = (ne > 1) ? w0[H / 4 + 1] : make_float4(0.f, 0.f, 0.f, 0.f);
+    const float2 x0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xw[0]));
+    const float2 x1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xw[1]));
+    const float2 x2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xw[2]));
+    const float2 x3 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xw[3]));
+    acc0 = fmaf(x0.x, a0.x, acc0); acc0 = fmaf(x0.y, a0.y, acc0); acc0 = fmaf(x1.x, a0.z, acc0);
+    acc0 = fmaf(x1.y, a0.w, acc0); acc0 = fmaf(x2.x, a1.x, acc0); acc0 = fmaf(x2.y, a1.y, acc0);
+    acc0 = fmaf(x3.x, a1.z, acc0); acc0 = fmaf(x3.y, a1.w, acc0);
+    acc1 = fmaf(x0.x, b0.x, acc1); acc1 = fmaf(x0.y, b0.y, acc1); acc1 = fmaf(x1.x, b0.z, acc1);
+    acc1 = fmaf(x1.y, b0.w, acc1); acc1 = fmaf(x2.x, b1.x, acc1); acc1 = fmaf(x2.y, b1.y, acc1);
+    acc1 = fmaf(x3.x, b1.z, acc1); acc1 = fmaf(x3.y, b1.w, acc1);
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    acc0 += __shfl_xor_sync(0xffffffffu, acc0, o);
+    acc1 += __shfl_xor_sync(0xffffffffu, acc1, o);
+  }
+  if (lane == 0) {
+    s_red[warp] = acc0;
+    s_red[nw + warp] = acc1;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    float v0 = (lane < nw) ? s_red[lane] : 0.f;
+    float v1 = (lane < nw) ? s_red[nw + lane] : 0.f;
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+      v0 += __shfl_xor_sync(0xffffffffu, v0, o);
+      v1 += __shfl_xor_sync(0xffffffffu, v1, o);
+    }
+    if (lane == 0) st_relaxed_u64(out, tag_word(epoch, v0));
+    if (lane == 1 && ne > 1) st_relaxed_u64(out + 1, tag_word(epoch, v1));
+  }
+}
+
+// Read n tagged logit words into s_logit until every one carries `want`
+// (eight independent loads in flight per thread, re-polling the stale ones).
+// Returns false, with the status bit set, when the wait runs out.
+__device__ __forceinline__ bool poll_tagged_logits(const Params& p, const unsigned long long* words, int n,
+                                                   unsigned want, float* s_logit) {
+  constexpr int kB = 8;
+  const long long t0 = clock64();
+  bool ok = true;
+  for (int i0 = threadIdx.x; i0 < n; i0 += kB * blockDim.x) {
+    unsigned long long w[kB];
+#pragma unroll
+    for (int j = 0; j < kB; ++j) {
+      const int i = i0 + j * blockDim.x;
+      w[j] = (i < n) ? ld_relaxed_u64(words + i) : ((unsigned long long)want << 32);
+    }
+#pragma unroll
+    for (int j = 0; j < kB; ++j) {
+      const int i = i0 + j * blockDim.x;
+      while ((unsigned)(w[j] >> 32) != want && ok) {
+        __nanosleep(32);
+        if (clock64() - t0 > p.spin_limit) {
+          atomicOr(p.ws.ctrl, kStatusTimeout);
+          ok = false;
+        }
+        w[j] = ld_relaxed_u64(words + i);
+      }
+      if (i < n) s_logit[i] = __uint_as_float((unsigned)w[j]);
+    }
+  }
+  return ok;
+}
+
+// One token: the union is its K distinct experts in ascending order, one
+// pair each (threads 0..K-1; pair positions from pbase, entries from ub).
+__device__ __forceinline__ void union_m1(const int* s_ids, int K, int ub, int pbase, int* s_union, int* s_poff,
+                                         int* s_pm, int* s_ppos, int* s_U) {
+  const int tid = threadIdx.x;
+  if (tid < K) {
+    const int id = s_ids[tid];
+    int rank = 0;
+    for (int j = 0; j < K; ++j) rank += s_ids[j] < id;
+    s_union[ub + rank] = id;
+    s_poff[ub + rank] = pbase + rank;
+    s_pm[pbase + rank] = 0;
+    s_ppos[tid] = pbase + rank;
+    if (rank == K - 1) {
+      s_poff[ub + K] = pbase + K;
+      *s_U = ub + K;
+    }
+  }
+}
+
 // One warp, M*K <= 32 pairs: the expert union (ascending ids) and the pairs
 // grouped by expert in (token, slot) order, from ranks computed with
 // shuffles (no shared-memory scratch). Pair i = (i / K, i % K); pair
@@ -845,6 +1056,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
     if (use > 0 && lane == 0) smem_count_wait(done_gu + slot, (unsigned)(use * gu_items), p);
     __syncwarp();
     mbar_wait(full_gu + slot, use & 1, p);
+    if (u == 0 && g == 0) trace_stamp(p, 5);
+    if (u == s_int[0] - 1 && g == gu_items - 1) trace_stamp(p, 16);
     GuChunk ch;
     size_t ga0, ua0;
     unsigned gn, un;
@@ -907,6 +1120,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
     }
     const int a = g * kGuRowsPerItem, cnt = min(kGuRowsPerItem, nr - a);
     gu_item(p, ch, a, cnt, n0, pb, pe, s_pm, act, s_xs);
+    if (u == 0 && g == 0) trace_stamp(p, 17);
+    if (u == s_int[0] - 1 && g == gu_items - 1) trace_stamp(p, 6);
     __syncwarp();
     if (lane == 0) {
       mbar_arrive(empty_gu + slot);
@@ -936,12 +1151,16 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
       tma_load_1d(wr_s, p.wr + (size_t)e0 * H, (unsigned)(ne * H * 4), wr_bar);
     }
   }
+  trace_stamp(p, 0);
   // Everything above is independent of the previous kernel on the stream.
   pdl_wait();
+  trace_stamp(p, 1);
   if (tid == 0) {
     s_int[1] = (int)(ld_relaxed_u32(fw.epoch) + 1u);
     s_int[2] = 0;  // gate/up queue head
     s_int[3] = 0;  // down queue head
+  }
+  if (tid == 0) {
     if constexpr (kShared) {
       s_union[0] = E;
       s_poff[0] = 0;
@@ -988,6 +1207,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
     if (mcur >= 0) atomicMax(&s_amax_u[mcur], __float_as_uint(a));
   }
   __syncthreads();
+  trace_stamp(p, 13);
   const uint4* xsrc = pl.x_staged ? x_s : reinterpret_cast<const uint4*>(p.x);
   // ---- A9 (stacked layers): x <- bf16(x / sqrt(mean(x^2) + 1e-6)) per token.
   //      One warp per token sums x^2 in a fixed order with IEEE fp32 ops, so
@@ -1045,7 +1265,17 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
   //          tokens per pass; warp partials go to shared memory and one block
   //          barrier per pass ends it
   if (ne > 0) mbar_wait(wr_bar, 0, p);
-  for (int m0 = 0; m0 < M && ne > 0; m0 += 4) {
+  trace_stamp(p, 14);
+  const bool lg_m1 = (M == 1 && ne > 0 && ne <= 2);
+  if (lg_m1) {
+    auto ld_x8 = [&](int i) -> uint4 {
+      uint4 v = pl.x_staged ? xsrc[i] : __ldcg(xsrc + i);
+      v.x = xn2(v.x, 0); v.y = xn2(v.y, 0); v.z = xn2(v.z, 0); v.w = xn2(v.w, 0);
+      return v;
+    };
+    router_logits_m1(ld_x8, wr_s, H, ne, epoch, fw.logits + e0, s_red);
+  }
+  for (int m0 = 0; m0 < M && ne > 0 && !lg_m1; m0 += 4) {
     const int mt = min(4, M - m0);
     for (int el = 0; el < ne; ++el) {
       float acc[4] = {0.f, 0.f, 0.f, 0.f};
@@ -1089,14 +1319,12 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
       if (t < mt) {
         float sum = 0.f;
         for (int w = 0; w < kFusedWarps; ++w) sum += s_red[w * (kMaxRowsPerCta * 4) + el * 4 + t];
-        fw.logits[(size_t)(m0 + t) * E + e0 + el] = sum;
+        st_relaxed_u64(fw.logits + (size_t)(m0 + t) * E + e0 + el, tag_word(epoch, sum));
       }
     }
     __syncthreads();
   }
-  // grid-wide: every CTA's logits are in L2 once the router count reaches
-  // epoch * G (the last arrival publishes the epoch to the flag copies)
-  if (tid == 0) grid_arrive(fw.route_cnt);
+  trace_stamp(p, 15);
   // ---- A1 (second half): E4M3 codes and scales, done while the other CTAs'
   //      logits arrive (the router works on the bf16 x, not on the codes)
   if (tid < M) {
@@ -1124,17 +1352,27 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
     if (b == 0 && p.out_xq) *reinterpret_cast<uint2*>(p.out_xq + (size_t)i * 8) = out;
   }
   if (b == 0 && p.out_xscale && tid < M) p.out_xscale[tid] = s_xs[tid];
+  trace_stamp(p, 2);
 
-  if (tid == 0)
-    grid_wait(fw.route_cnt, (unsigned long long)(p.force_stall ? epoch + 0x40000000u : epoch) * G, p);
+  // ---- A2 exchange: every logit word of this launch (the tag is the flag)
+  poll_tagged_logits(p, fw.logits, M * E, p.force_stall ? epoch + 0x40000000u : epoch, s_logit);
+  trace_stamp(p, 3);
   pdl_launch_dependents();
   __syncthreads();
+  trace_stamp(p, 20);
 
-  // ---- A3: gather all M*E logits into shared memory; one warp per token
-  //          selects the top-k (ties to the lower index) and its softmax
-  for (int i = tid; i < M * E; i += kFusedThreads) s_logit[i] = __ldcg(fw.logits + i);
-  __syncthreads();
-  for (int m = warp; m < M; m += kFusedWarps) {
+  // ---- A3: top-k (ties to the lower index) and its softmax: every warp on
+  //          the one token when M == 1, else one warp per token
+  const bool tk_m1 = (M == 1 && E <= 32 * kFusedWarps && K <= 8);
+  if (tk_m1) {
+    topk_cta_small(s_logit, E, K, s_ids, s_w, reinterpret_cast<unsigned*>(s_red),
+                   reinterpret_cast<int*>(s_red) + 136, p);
+    if (b == 0 && tid < K) {
+      if (p.out_ids) p.out_ids[tid] = s_ids[tid];
+      if (p.out_w) p.out_w[tid] = s_w[tid];
+    }
+  }
+  for (int m = warp; m < M && !tk_m1; m += kFusedWarps) {
     const float* lrow = s_logit + (size_t)m * E;
     int* ids = s_ids + m * K;
     float* ws = s_w + m * K;
@@ -1151,12 +1389,16 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
     }
   }
   __syncthreads();
+  trace_stamp(p, 8);
 
   // ---- A4: expert union (ascending ids) and the (token, slot) pairs of each
   //          entry in (token, slot) order; one warp, no block barriers
   // (with a shared expert, routed entries start at 1 and their pairs at M)
   const int np = M * K, pbase = kShared ? M : 0;
-  if (warp == 0 && np <= 32) {
+  if (M == 1) {
+    union_m1(s_ids, K, ub, pbase, s_union, s_poff, s_pm, s_ppos, &s_int[0]);
+    if (tid < K) s_cnt[ub + tid] = 0;  // per-entry gate/up item counters
+  } else if (warp == 0 && np <= 32) {
     const int Us = union_small(s_ids, np, K, s_union + ub, s_poff + ub, s_pm, s_ppos, pbase);
     if (lane == 0) s_int[0] = ub + Us;
     for (int u = lane; u < Us; u += 32) s_cnt[ub + u] = 0;  // per-entry gate/up item counters
@@ -1217,6 +1459,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
   }
   __syncthreads();
   const int U = s_int[0];
+  trace_stamp(p, 4);
 
   const int n_gu0 = (nr > 0) ? min(U, pl.ns_gu) : 0;
   const int n_d0 = (nrd > 0) ? min(U, pl.ns_d) : 0;
@@ -1227,6 +1470,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
     for (int u = ub + warp; u < n_gu0; u += kFusedWarps) issue_gu(u);
     for (int u = ub + warp; u < n_d0; u += kFusedWarps) issue_d(u);
   }
+  if (warp == 0) trace_stamp(p, 59);
+  if (warp == 0) trace_stamp(p, 59);
   if (warp == 0) {
     // refills of drained slots (more union entries than slots): one thread
     // polls both rings without suspending and issues whichever slot drains
@@ -1339,7 +1584,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
       }
     }
   }
+  trace_stamp(p, 10);
   consumers_sync();
+  trace_stamp(p, 11);
   // ---- A8: combine in slot order, bf16 out
   const int ct = tid - 32;
   for (int i = ct; i < M * nrd; i += kConsumers * 32) {
@@ -1354,6 +1601,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
     for (int u = U; u < pl.max_union; ++u) red_release_add_u64(gu_counter(fw, u), (unsigned long long)G);
     st_relaxed_u32(fw.epoch, epoch);
   }
+  trace_stamp(p, 12);
 }
 
 }  // namespace moe

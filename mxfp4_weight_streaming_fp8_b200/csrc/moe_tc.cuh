@@ -91,10 +91,10 @@ struct TcPlan {
   int smem_bytes;  // including 1 KB of alignment slack
 };
 
+constexpr int kTcXRegs = 8;    // uint4 of a token's x per lane per pass when M >= 2
 constexpr int kTcCntStride = 32;  // u32 words between per-entry counters (one 128-byte line each)
 constexpr int kTcMaxTiles = 64;   // gate/up tiles per CTA
 constexpr int kTcWarpGate = 3;    // polls the entry counters for the CTA
-constexpr int kTcTrace = 64;     // timestamps per CTA in the optional trace
 
 // The gate/up code maps, passed by value as a __grid_constant__ kernel
 // parameter (TMA reads its descriptor from parameter space).
@@ -110,13 +110,7 @@ struct TcWs {
   unsigned* epoch;             // launch counter
 };
 
-__device__ __forceinline__ void tc_trace(const Params& p, int slot) {
-  if (p.trace && (threadIdx.x & 31) == 0 && slot < kTcTrace) {
-    unsigned long long t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    p.trace[(size_t)blockIdx.x * kTcTrace + slot] = t;
-  }
-}
+__device__ __forceinline__ void tc_trace(const Params& p, int slot) { trace_stamp(p, slot); }
 __device__ __forceinline__ unsigned ld_acquire_u32g(const unsigned* p) {
   unsigned v;
   asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -246,9 +240,6 @@ __device__ __forceinline__ unsigned long long ld_relaxed_v2(const unsigned long 
 __device__ __forceinline__ void st_relaxed_v2(unsigned long long* p, unsigned long long a, unsigned long long b) {
   asm volatile("st.relaxed.gpu.global.v2.b64 [%0], {%1, %2};" ::"l"(p), "l"(a), "l"(b) : "memory");
 }
-__device__ __forceinline__ unsigned long long tag_word(unsigned epoch, float v) {
-  return ((unsigned long long)epoch << 32) | __float_as_uint(v);
-}
 
 // Byte offset of K element k of row r in a K-major 128-byte-swizzled operand
 // laid out as [K-chunk][8-row group][8][128 B] with `groups` row groups.
@@ -259,27 +250,6 @@ __device__ __forceinline__ uint32_t sw128_offset(int r, int k, int groups) {
 
 // Wait (one lane, acquire at CTA scope) until a shared-memory flag is set;
 // the warp gets one verdict.
-__device__ __forceinline__ unsigned ld_acquire_cta_smem(const unsigned* p) {
-  unsigned v;
-  asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
-  return v;
-}
-__device__ __forceinline__ bool tc_wait_flag(const Params& p, const unsigned* flag) {
-  bool ok = true;
-  if ((threadIdx.x & 31) == 0 && ld_acquire_cta_smem(flag) == 0u) {
-    const long long t0 = clock64();
-    while (ld_acquire_cta_smem(flag) == 0u) {
-      __nanosleep(32);
-      if (clock64() - t0 > p.spin_limit) {
-        atomicOr(p.ws.ctrl, kStatusTimeout);
-        ok = false;
-        break;
-      }
-    }
-  }
-  return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-}
-
 // Down item: rows [a, a+cnt) of one entry's chunk for each of its pairs. Lane
 // l takes 32-element block l of the pair's h, read once from L2 (I <= 1024:
 // one block per lane); the pair's power-of-two rescale (kFp8H: its E4M3
@@ -363,80 +333,6 @@ __device__ __forceinline__ void tc_d_item(const Params& p, const TcWs& tw, const
   }
 }
 
-// Order-preserving 32-bit image of a float, and back.
-__device__ __forceinline__ unsigned fkey(float v) {
-  const unsigned u = __float_as_uint(v);
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-__device__ __forceinline__ float fkey_value(unsigned k) {
-  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
-}
-
-// Top-k (K <= 8) of one token's E <= 512 logits with every warp of the CTA:
-// warp w first takes the K best of experts 32w..32w+31 (one per lane; ties
-// to the lower lane, i.e. the lower expert); then every candidate's rank
-// among all of them is counted in parallel (larger logit first, ties to the
-// lower expert), and warp 0 forms the softmax over the K kept. Same result
-// as topk_warp; all threads must call it. s_ck, s_ce: 136 words each
-// (W*8 <= 128 candidates, then the K results).
-__device__ void topk_cta_small(const float* l, int E, int K, int* ids, float* wts, unsigned* s_ck, int* s_ce) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int W = (E + 31) / 32;
-  if (warp < W) {
-    const int e = 32 * warp + lane;
-    unsigned key = (e < E) ? fkey(l[e]) : 0u;
-    if (lane < 8 && lane >= K) {
-      s_ck[warp * 8 + lane] = 0u;
-      s_ce[warp * 8 + lane] = 0x7fffffff;
-    }
-    for (int r = 0; r < K; ++r) {
-      const unsigned mx = __reduce_max_sync(0xffffffffu, key);
-      const int win = __ffs(__ballot_sync(0xffffffffu, key == mx)) - 1;
-      if (lane == win) {
-        s_ck[warp * 8 + r] = mx;
-        s_ce[warp * 8 + r] = (mx != 0u) ? e : 0x7fffffff;
-        key = 0u;
-      }
-    }
-  }
-  __syncthreads();
-  // merge: the rank of candidate c among all W*8 slots (larger key first,
-  // then the lower expert), four threads per candidate, each counting over a
-  // quarter; ranks below K are the result, in order
-  {
-    const int c = threadIdx.x >> 2, part = threadIdx.x & 3, nc = W * 8;
-    int rank = 0;
-    unsigned kc = 0u;
-    int ec = 0x7fffffff;
-    if (c < nc) {
-      kc = s_ck[c];
-      ec = s_ce[c];
-      for (int d = part; d < nc; d += 4) {
-        const unsigned kd = s_ck[d];
-        const int ed = s_ce[d];
-        rank += (kd > kc) || (kd == kc && ed < ec);
-      }
-    }
-    rank += __shfl_xor_sync(0xffffffffu, rank, 1);
-    rank += __shfl_xor_sync(0xffffffffu, rank, 2);
-    __syncthreads();
-    if (c < nc && part == 0 && kc != 0u && rank < K) {
-      s_ck[128 + rank] = kc;
-      s_ce[128 + rank] = ec;
-    }
-    __syncthreads();
-  }
-  if (warp == 0) {
-    const float top = fkey_value(s_ck[128]);
-    const float v = (lane < K) ? fkey_value(s_ck[128 + lane]) : 0.f;
-    const float ex = (lane < K) ? expf(v - top) : 0.f;
-    const float z = warp_sum(ex);
-    if (lane < K) {
-      ids[lane] = s_ce[128 + lane];
-      wts[lane] = ex / z;
-    }
-  }
-}
 
 // Re-tiles gate/up codes [Eall][2I][H/2] into [Eall][I/4][H/128][8][64 B]:
 // block (e, j, c) holds rows 4j..4j+3 (gate) and I+4j..I+4j+3 (up) of
@@ -599,6 +495,119 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc(Params p, TcWs tw, TcPlan 
     }
     return v;
   };
+  const int nbg = pl.nb_max / 8;
+  if (M >= 2) {
+    // ---- A9 + A1 + A2 for several tokens: one warp per token, over its x
+    //      row in chunks of kTcXRegs uint4 per lane (L2 reads). Pass 1: the
+    //      RMSNorm sum of squares (fixed order) and amax; the new amax is
+    //      bf16(fl32(amax * r)) (rounding is monotonic and symmetric). Pass 2:
+    //      the logits of the CTA's router rows (tagged stores) and the E4M3
+    //      codes straight into the MMA's B operand (K-major, 128-byte
+    //      swizzle; rows >= M are never read).
+    if (ne > 0 && !mbar_wait_ok(wr_bar, 0, p)) ok = false;
+    tc_trace(p, 14);
+    const int ng = H / 8;
+    if (tid < kMaxTokens) s_xs[tid] = 1.f;
+    __syncwarp();
+    for (int m = warp; m < M; m += kTcWarps) {
+      const uint4* xg = reinterpret_cast<const uint4*>(p.x) + (size_t)m * ng;
+      float ss = 0.f, a = 0.f;
+      for (int c0 = 0; c0 < ng; c0 += 32 * kTcXRegs) {
+        uint4 xr[kTcXRegs];
+#pragma unroll
+        for (int j = 0; j < kTcXRegs; ++j) {
+          const int i = c0 + lane + 32 * j;
+          xr[j] = (i < ng) ? __ldcg(xg + i) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int j = 0; j < kTcXRegs; ++j) {
+          const uint32_t w[4] = {xr[j].x, xr[j].y, xr[j].z, xr[j].w};
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[t]));
+            ss = __fmaf_rn(f.x, f.x, ss);
+            ss = __fmaf_rn(f.y, f.y, ss);
+            a = fmaxf(a, fmaxf(fabsf(f.x), fabsf(f.y)));
+          }
+        }
+      }
+      a = warp_max(a);
+      float r = 1.f;
+      if (p.pre_rmsnorm) {
+        ss = warp_sum(ss);
+        r = __fdiv_rn(1.f, __fsqrt_rn(__fadd_rn(__fdiv_rn(ss, (float)H), 1e-6f)));
+        a = __bfloat162float(__float2bfloat16_rn(__fmul_rn(a, r)));
+      }
+      const float inv = (a != 0.f) ? __fdiv_rn(448.f, a) : 0.f;
+      float acc[kMaxRowsPerCta];
+#pragma unroll
+      for (int el = 0; el < kMaxRowsPerCta; ++el) acc[el] = 0.f;
+      for (int c0 = 0; c0 < ng; c0 += 32 * kTcXRegs) {
+        uint4 xr[kTcXRegs];
+#pragma unroll
+        for (int j = 0; j < kTcXRegs; ++j) {
+          const int i = c0 + lane + 32 * j;
+          xr[j] = (i < ng) ? __ldcg(xg + i) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int j = 0; j < kTcXRegs; ++j) {
+          const int i = c0 + lane + 32 * j;
+          if (i >= ng) continue;
+          uint32_t w[4] = {xr[j].x, xr[j].y, xr[j].z, xr[j].w};
+          if (p.pre_rmsnorm) {
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+              const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[t]));
+              const __nv_bfloat162 o = __floats2bfloat162_rn(__fmul_rn(f.x, r), __fmul_rn(f.y, r));
+              w[t] = *reinterpret_cast<const uint32_t*>(&o);
+            }
+            if (b == 0 && p.out_xn)
+              reinterpret_cast<uint4*>(p.out_xn)[(size_t)m * ng + i] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+          float2 xf[4];
+#pragma unroll
+          for (int t = 0; t < 4; ++t) xf[t] = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[t]));
+#pragma unroll
+          for (int el = 0; el < kMaxRowsPerCta; ++el) {
+            if (el < ne) {
+              const float4* wrow = reinterpret_cast<const float4*>(wr_s + (size_t)el * H);
+              const float4 w0 = wrow[2 * i], w1 = wrow[2 * i + 1];
+              float v = acc[el];
+              v = fmaf(xf[0].x, w0.x, v); v = fmaf(xf[0].y, w0.y, v); v = fmaf(xf[1].x, w0.z, v);
+              v = fmaf(xf[1].y, w0.w, v); v = fmaf(xf[2].x, w1.x, v); v = fmaf(xf[2].y, w1.y, v);
+              v = fmaf(xf[3].x, w1.z, v); v = fmaf(xf[3].y, w1.w, v);
+              acc[el] = v;
+            }
+          }
+          uint2 out = make_uint2(0u, 0u);
+          if (a != 0.f) {
+            const uint32_t c0v = f32x2_to_e4m3x2(__fmul_rn(xf[0].x, inv), __fmul_rn(xf[0].y, inv));
+            const uint32_t c1v = f32x2_to_e4m3x2(__fmul_rn(xf[1].x, inv), __fmul_rn(xf[1].y, inv));
+            const uint32_t c2v = f32x2_to_e4m3x2(__fmul_rn(xf[2].x, inv), __fmul_rn(xf[2].y, inv));
+            const uint32_t c3v = f32x2_to_e4m3x2(__fmul_rn(xf[3].x, inv), __fmul_rn(xf[3].y, inv));
+            out = make_uint2(c0v | (c1v << 16), c2v | (c3v << 16));
+          }
+          *reinterpret_cast<uint2*>(bx + sw128_offset(m, 8 * i, nbg)) = out;
+          if (b == 0 && p.out_xq) *reinterpret_cast<uint2*>(p.out_xq + (size_t)m * H + 8 * i) = out;
+        }
+      }
+#pragma unroll
+      for (int el = 0; el < kMaxRowsPerCta; ++el) {
+        if (el < ne) {
+          const float v = warp_sum(acc[el]);
+          if (lane == 0) st_relaxed_u64(tw.logits + (size_t)m * E + e0 + el, tag_word(epoch, v));
+        }
+      }
+      if (lane == 0) {
+        s_amax[m] = a;
+        s_xs[m] = (a == 0.f) ? 1.f : __fdiv_rn(a, 448.f);
+        if (b == 0 && p.out_xscale) p.out_xscale[m] = s_xs[m];
+      }
+    }
+    tc_trace(p, 15);
+    // the B operand is read by the tensor cores (async proxy)
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  } else {
   // ---- A1 (first half): stage x (when it fits), per-token amax
   for (int i = tid; i < M * H / 8; i += kTcThreads) {
     const int m = (i * 8) / H;
@@ -660,50 +669,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc(Params p, TcWs tw, TcPlan 
   // ---- A2: logits of the CTA's router rows
   if (ne > 0 && !mbar_wait_ok(wr_bar, 0, p)) ok = false;
   tc_trace(p, 14);
-  if (M == 1 && ne > 0 && ne <= 2) {
-    // one token: every thread takes a strided share of both rows at once;
-    // warp sums, then warp 0 sums the warps' partials
-    float acc0 = 0.f, acc1 = 0.f;
-    for (int i = tid; i < H / 8; i += kTcThreads) {
-      const uint4 x8 = ld_x8(i);
-      const uint32_t xw[4] = {x8.x, x8.y, x8.z, x8.w};
-      const float4* w0 = reinterpret_cast<const float4*>(wr_s) + 2 * i;
-      const float4 a0 = w0[0], a1 = w0[1];
-      const float4 b0 = (ne > 1) ? w0[H / 4] : make_float4(0.f, 0.f, 0.f, 0.f);
-      const float4 b1 = (ne > 1) ? w0[H / 4 + 1] : make_float4(0.f, 0.f, 0.f, 0.f);
-      const float2 x0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xw[0]));
-      const float2 x1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xw[1]));
-      const float2 x2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xw[2]));
-      const float2 x3 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xw[3]));
-      acc0 = fmaf(x0.x, a0.x, acc0); acc0 = fmaf(x0.y, a0.y, acc0); acc0 = fmaf(x1.x, a0.z, acc0);
-      acc0 = fmaf(x1.y, a0.w, acc0); acc0 = fmaf(x2.x, a1.x, acc0); acc0 = fmaf(x2.y, a1.y, acc0);
-      acc0 = fmaf(x3.x, a1.z, acc0); acc0 = fmaf(x3.y, a1.w, acc0);
-      acc1 = fmaf(x0.x, b0.x, acc1); acc1 = fmaf(x0.y, b0.y, acc1); acc1 = fmaf(x1.x, b0.z, acc1);
-      acc1 = fmaf(x1.y, b0.w, acc1); acc1 = fmaf(x2.x, b1.x, acc1); acc1 = fmaf(x2.y, b1.y, acc1);
-      acc1 = fmaf(x3.x, b1.z, acc1); acc1 = fmaf(x3.y, b1.w, acc1);
-    }
-#pragma unroll
-    for (int o = 16; o; o >>= 1) {
-      acc0 += __shfl_xor_sync(0xffffffffu, acc0, o);
-      acc1 += __shfl_xor_sync(0xffffffffu, acc1, o);
-    }
-    if (lane == 0) {
-      s_red[warp] = acc0;
-      s_red[kTcWarps + warp] = acc1;
-    }
-    __syncthreads();
-    if (warp == 0) {
-      float v0 = (lane < kTcWarps) ? s_red[lane] : 0.f;
-      float v1 = (lane < kTcWarps) ? s_red[kTcWarps + lane] : 0.f;
-#pragma unroll
-      for (int o = kTcWarps / 2; o; o >>= 1) {
-        v0 += __shfl_xor_sync(0xffffffffu, v0, o);
-        v1 += __shfl_xor_sync(0xffffffffu, v1, o);
-      }
-      if (lane == 0) st_relaxed_u64(tw.logits + e0, tag_word(epoch, v0));
-      if (lane == 1 && ne > 1) st_relaxed_u64(tw.logits + e0 + 1, tag_word(epoch, v1));
-    }
-  }
+  if (M == 1 && ne > 0 && ne <= 2)
+    router_logits_m1(ld_x8, wr_s, H, ne, epoch, tw.logits + e0, s_red);
   for (int m0 = 0; m0 < M && ne > 0 && !(M == 1 && ne <= 2); m0 += 4) {
     const int mt = min(4, M - m0);
     for (int el = 0; el < ne; ++el) {
@@ -751,7 +718,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc(Params p, TcWs tw, TcPlan 
   tc_trace(p, 15);
   // ---- A1 (second half): E4M3 codes straight into the MMA's B operand
   //      (K-major, 128-byte swizzle, nb_max token rows; rows >= M are zero)
-  const int nbg = pl.nb_max / 8;
   if (tid < kMaxTokens) {
     const float a = (tid < M) ? s_amax[tid] : 0.f;
     s_xs[tid] = (a == 0.f) ? 1.f : __fdiv_rn(a, 448.f);
@@ -788,26 +754,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc(Params p, TcWs tw, TcPlan 
   if (b == 0 && p.out_xscale && tid < M) p.out_xscale[tid] = s_xs[tid];
   // the B operand is read by the tensor cores (async proxy)
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
   tc_trace(p, 2);
 
   // ---- A2 exchange: read every logit word until all carry this epoch
-  {
-    const long long t0 = clock64();
-    const unsigned want = p.force_stall ? epoch + 0x40000000u : epoch;
-    for (int i = tid; i < M * E; i += kTcThreads) {
-      unsigned long long w = ld_relaxed_u64(tw.logits + i);
-      while ((unsigned)(w >> 32) != want) {
-        __nanosleep(32);
-        if (clock64() - t0 > p.spin_limit) {
-          atomicOr(p.ws.ctrl, kStatusTimeout);
-          ok = false;
-          break;
-        }
-        w = ld_relaxed_u64(tw.logits + i);
-      }
-      s_logit[i] = __uint_as_float((unsigned)w);
-    }
-  }
+  if (!poll_tagged_logits(p, tw.logits, M * E, p.force_stall ? epoch + 0x40000000u : epoch, s_logit)) ok = false;
   pdl_launch_dependents();
   __syncthreads();
   tc_trace(p, 3);
@@ -816,7 +767,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc(Params p, TcWs tw, TcPlan 
   //      else one warp per token
   if (M == 1 && E <= 32 * kTcWarps && K <= 8) {
     topk_cta_small(s_logit, E, K, s_ids, s_w, reinterpret_cast<unsigned*>(s_red),
-                   reinterpret_cast<int*>(s_red) + 136);
+                   reinterpret_cast<int*>(s_red) + 136, p);
     if (b == 0 && tid < K) {
       if (p.out_ids) p.out_ids[tid] = s_ids[tid];
       if (p.out_w) p.out_w[tid] = s_w[tid];
@@ -844,20 +795,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc(Params p, TcWs tw, TcPlan 
   // ---- A4: union (ascending ids) and the pairs of each entry in (token, slot) order
   const int np = M * K, pbase = kShared ? M : 0;
   if (M == 1) {
-    // one token: its K distinct experts, sorted; each entry has one pair
-    if (tid < K) {
-      const int id = s_ids[tid];
-      int rank = 0;
-      for (int j = 0; j < K; ++j) rank += s_ids[j] < id;
-      s_union[ub + rank] = id;
-      s_poff[ub + rank] = pbase + rank;
-      s_pm[pbase + rank] = 0;
-      s_ppos[tid] = pbase + rank;
-      if (rank == K - 1) {
-        s_poff[ub + K] = pbase + K;
-        s_int[0] = ub + K;
-      }
-    }
+    union_m1(s_ids, K, ub, pbase, s_union, s_poff, s_pm, s_ppos, &s_int[0]);
   } else if (warp == 0 && np <= 32) {
     const int Us = union_small(s_ids, np, K, s_union + ub, s_poff + ub, s_pm, s_ppos, pbase);
     if (lane == 0) s_int[0] = ub + Us;
@@ -973,7 +911,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc(Params p, TcWs tw, TcPlan 
           if (reuse && !mbar_wait_ok(empty_gu + slot, ph ^ 1u, p)) { ok = false; break; }
           if (stage >= pl.ns_gu && stage < pl.ns_gu + 4) tc_trace(p, 42 + stage - pl.ns_gu);
           mbar_expect_tx(full_gu + slot, bytes);
-          tc_trace(p, 32 + stage);
+          if (stage < 10) tc_trace(p, 32 + stage);
           uint8_t* dst = ring_gu + (size_t)slot * pl.slot_gu;
           for (int r = 0; r < nrun; ++r) {
             if (tw.repacked)
@@ -1006,7 +944,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc(Params p, TcWs tw, TcPlan 
       tc_fence_after();
       for (int k = 0; k < nstage; ++k, ++stage) {
         if (!mbar_wait_warp(full_gu + slot, ph, p)) { ok = false; break; }
-        tc_trace(p, 16 + stage);
+        if (stage < 8) tc_trace(p, 16 + stage);
         if (lane == 0) {
           tc_fence_after();
           const uint64_t ads = ad0 + (uint64_t)slot * slot_step;
@@ -1194,7 +1132,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc(Params p, TcWs tw, TcPlan 
       __syncwarp();
       if (it == 0) tc_trace(p, 51);
       if (it == total - 1) tc_trace(p, 54);
-      if (!tc_wait_flag(p, s_hready + u)) ok = false;
+      if (!wait_flag_warp(p, s_hready + u)) ok = false;
       if (u == U - 1 && gd == 0) tc_trace(p, 9);
       if (it == 0) tc_trace(p, 52);
       if (it == total - 1) tc_trace(p, 55);
