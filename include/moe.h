@@ -125,6 +125,24 @@ typedef enum {
                                        runs. Setting both flags is
                                        MOE_ERR_INVALID_ARG */
 #define MOE_TC_MIN_TOKENS 2
+#define MOE_FLAG_TC_DOWN_MMA 0x40u   /* tensor-core kernel: run the down
+                                       projection on tcgen05 MMAs as well
+                                       (tiles of 128 output rows x up to 16
+                                       pairs of one expert; W2 decoded once
+                                       per tile, not once per pair). h enters
+                                       as per-pair-scaled E4M3 hi + lo/16
+                                       (within 2^-8 of h; with
+                                       MOE_FLAG_FP8_INTERMEDIATE, the FP8 h
+                                       codes alone). Needs I <= 1024, else
+                                       the tensor-core plan fails; also I <= H */
+#define MOE_FLAG_TC_DOWN_CUDA 0x80u  /* tensor-core kernel: keep the down
+                                       projection on CUDA cores. With neither
+                                       TC_DOWN flag the tensor cores take the
+                                       down projection from
+                                       MOE_TC_DOWN_MMA_MIN_TOKENS tokens of
+                                       max_tokens on. Both flags:
+                                       MOE_ERR_INVALID_ARG */
+#define MOE_TC_DOWN_MMA_MIN_TOKENS 8
 
 typedef struct {
   int32_t hidden;      /* H: multiple of 32, 32..8192                        */

@@ -36,8 +36,10 @@ moe_status validate_config(const moe_config& c) {
   if (c.top_k < 1 || c.top_k > c.num_experts || c.top_k > moe::kMaxTopK) return MOE_ERR_INVALID_ARG;
   if (c.max_tokens < 1 || c.max_tokens > moe::kMaxTokens) return MOE_ERR_INVALID_ARG;
   const uint32_t fused_only = MOE_FLAG_PRE_RMSNORM | MOE_FLAG_SHARED_EXPERT | MOE_FLAG_FP8_INTERMEDIATE;
-  if (c.flags & ~(MOE_FLAG_SPLIT_KERNELS | MOE_FLAG_CUDA_CORES | MOE_FLAG_TENSOR_CORES | fused_only))
+  if (c.flags & ~(MOE_FLAG_SPLIT_KERNELS | MOE_FLAG_CUDA_CORES | MOE_FLAG_TENSOR_CORES | MOE_FLAG_TC_DOWN_MMA |
+                  MOE_FLAG_TC_DOWN_CUDA | fused_only))
     return MOE_ERR_INVALID_ARG;
+  if ((c.flags & MOE_FLAG_TC_DOWN_MMA) && (c.flags & MOE_FLAG_TC_DOWN_CUDA)) return MOE_ERR_INVALID_ARG;
   if ((c.flags & MOE_FLAG_CUDA_CORES) && (c.flags & MOE_FLAG_TENSOR_CORES)) return MOE_ERR_INVALID_ARG;
   if ((c.flags & MOE_FLAG_TENSOR_CORES) && (c.flags & MOE_FLAG_SPLIT_KERNELS)) return MOE_ERR_INVALID_ARG;
   if ((c.flags & fused_only) && (c.flags & MOE_FLAG_SPLIT_KERNELS)) return MOE_ERR_UNSUPPORTED;
@@ -144,15 +146,27 @@ bool make_tc_plan(const moe_config& c, int sm_count, size_t smem_limit, moe::TcP
   pl->max_pairs = (int)NP;
   pl->max_union = (int)UMAX;
   const size_t units_max = UMAX * (I / 4);
-  const size_t tu_max = std::min<size_t>(moe::kTcMaxUnits, (units_max + G - 1) / G);
+  // down projection on tensor cores: forced by a flag, else from
+  // MOE_TC_DOWN_MMA_MIN_TOKENS tokens on; its W2 stages (128 rows x 128
+  // elements) take 16-unit gate/up slots of one K-chunk, a lane holds I/32
+  // values of h (I <= 1024), and I <= H
+  const bool mma_down = !(c.flags & MOE_FLAG_TC_DOWN_CUDA) &&
+                        ((c.flags & MOE_FLAG_TC_DOWN_MMA) || MM >= MOE_TC_DOWN_MMA_MIN_TOKENS) && I <= 1024 &&
+                        I <= H;  // a down tile's scale factors fit a gate/up tile's tensor-memory columns
+  if ((c.flags & MOE_FLAG_TC_DOWN_MMA) && !mma_down) return false;
+  const size_t tu_max =
+      mma_down ? moe::kTcMaxUnits : std::min<size_t>(moe::kTcMaxUnits, (units_max + G - 1) / G);
   pl->tu_max = (int)tu_max;
-  pl->ks = (tu_max <= 12 && KCH % 2 == 0) ? 2 : 1;
+  pl->ks = (!mma_down && tu_max <= 12 && KCH % 2 == 0) ? 2 : 1;
+  pl->mma_down = mma_down ? 1 : 0;
+  pl->dkch = (int)(I / 128);
+  pl->bd_bytes = (int)(I / 128 * 4 * 1024);
   const size_t ks = pl->ks, nstage = KCH / ks;
   pl->nb_max = (int)std::max<size_t>(8, (MM + 7) / 8 * 8);
   pl->slot_gu = (int)(tu_max * ks * 1024);
   pl->bx_bytes = (int)(KCH * (pl->nb_max / 8) * 1024);
   const size_t overread = (moe::kTcMaxUnits - tu_max) * ks * 1024;  // junk MMA rows past the last slot
-  pl->sc_bytes = (int)align_up(8 * tu_max * (H / 32), 128);
+  pl->sc_bytes = (int)align_up(std::max<size_t>(8 * tu_max * (H / 32), mma_down ? 128 * (I / 32) : 0), 128);
   const size_t nrd_max = (H + G - 1) / G;
   pl->rpc_max = (int)nrd_max;
   pl->slot_d = (int)align_up(nrd_max * (I / 2) + nrd_max * (I / 32) + 32, 128);
@@ -163,7 +177,7 @@ bool make_tc_plan(const moe_config& c, int sm_count, size_t smem_limit, moe::TcP
   const size_t lg_bytes = align_up(MM * E * 4 + E * 4, 128);  // gathered logits + union scratch
   // fixed regions
   size_t fixed = align_up(std::max<size_t>(pl->bx_bytes, overread), 1024) + 2 * pl->sc_bytes;
-  const size_t bar_bytes = (2 * moe::kTcMaxSlots + 4 + 3 * moe::kMaxSlots + 1 + 6) * 8 + moe::kMaxSlots * 4;
+  const size_t bar_bytes = (2 * moe::kTcMaxSlots + 4 + 3 * moe::kMaxSlots + 1 + 14) * 8 + moe::kMaxSlots * 4;
   // tensor memory: 2 accumulators of 32 columns, 2 tiles' scale factors (4
   // columns per K-chunk), 4 columns of token scale factors
   const size_t cols = 64 + 8 * KCH + 4;
@@ -173,13 +187,15 @@ bool make_tc_plan(const moe_config& c, int sm_count, size_t smem_limit, moe::TcP
   const size_t misc_bytes = (3 * moe::kMaxTokens + moe::kTcWarps * moe::kMaxRowsPerCta * 4 + 8 + moe::kTcMaxTiles) * 4;
   // tiles a CTA may get: at most one more than the rounds of tu_max-unit tiles
   if ((units_max + G * tu_max - 1) / (G * tu_max) + 1 > (size_t)moe::kTcMaxTiles) return false;
+  const size_t dsm_bytes = mma_down ? 0 : NP * nrd_max * 4;  // per-pair down rows (CUDA-core down)
   const size_t small = align_up(bar_bytes, 16) + align_up(misc_bytes, 16) + align_up(UMAX * 4, 16) + 4 * align_up(NP * 4, 16) +
-                       align_up(UMAX * 4, 16) + align_up((UMAX + 1) * 4, 16) + align_up(NP * nrd_max * 4, 16);
+                       align_up(UMAX * 4, 16) + align_up((UMAX + 1) * 4, 16) + align_up(dsm_bytes, 16);
   fixed += small + 1024 /* alignment slack */ + 4 * 128;
+  if (mma_down) fixed += 2 * (size_t)pl->bd_bytes + 1024 + 4 * moe::kTcDownPairs * 4 + align_up((UMAX + 1) * 4, 16);
   if (fixed >= smem_limit) return false;
   size_t room = smem_limit - fixed;
-  // down ring: up to 8 entries in flight, at least 2
-  size_t ns_d = std::min<size_t>(UMAX, 8), per_d = pl->slot_d + pl->hslot;
+  // down ring (CUDA-core down): up to 8 entries in flight, at least 2
+  size_t ns_d = mma_down ? 0 : std::min<size_t>(UMAX, 8), per_d = pl->slot_d + pl->hslot;
   while (ns_d > 2 && room < ns_d * per_d + 2 * (size_t)pl->slot_gu) --ns_d;
   if (room < ns_d * per_d) return false;
   room -= ns_d * per_d;
@@ -195,9 +211,11 @@ bool make_tc_plan(const moe_config& c, int sm_count, size_t smem_limit, moe::TcP
   const size_t ring_gu_bytes = ns_gu * (size_t)pl->slot_gu;
   const size_t ring_d_bytes = ns_d * (size_t)pl->slot_d + ns_d * (size_t)pl->hslot;
   const bool x_fits = MM * H * 2 <= ring_d_bytes;
-  // a region of its own when there is room (then no second proxy fence)
-  const bool lg_own = fixed + ns_gu * (size_t)pl->slot_gu + ns_d * per_d + lg_bytes + 128 <= smem_limit &&
-                      lg_bytes <= 16384;
+  // a region of its own when there is room (then no second proxy fence);
+  // with the tensor-core down, the B operand buffers (idle until routing ends)
+  const bool lg_in_bd = mma_down && lg_bytes <= 2 * (size_t)pl->bd_bytes;
+  const bool lg_own = lg_in_bd || (fixed + ns_gu * (size_t)pl->slot_gu + ns_d * per_d + lg_bytes + 128 <= smem_limit &&
+                                   lg_bytes <= 16384);
   const bool lg_in_gu = !lg_own && pl->wr_bytes_max + lg_bytes <= ring_gu_bytes;
   const bool lg_in_d = !lg_own && !lg_in_gu && (x_fits ? align_up(MM * H * 2, 128) : 0) + lg_bytes <= ring_d_bytes;
   size_t off = 0;
@@ -208,11 +226,15 @@ bool make_tc_plan(const moe_config& c, int sm_count, size_t smem_limit, moe::TcP
   pl->o_sf = (int)off;  // (no shared-memory scale-factor staging)
   pl->o_sc = (int)take(2 * (size_t)pl->sc_bytes, 128);
   pl->o_sfb = (int)off;
+  pl->o_bd = mma_down ? (int)take(2 * (size_t)pl->bd_bytes, 1024) : 0;
+  pl->o_dsc = mma_down ? (int)take(4 * moe::kTcDownPairs * 4, 16) : 0;
+  pl->o_dtoff = mma_down ? (int)take((UMAX + 1) * 4, 16) : 0;
   pl->o_ring_d = (int)take(ns_d * (size_t)pl->slot_d, 128);
   pl->o_h = (int)take(ns_d * (size_t)pl->hslot, 16);
   pl->x_staged = x_fits ? 1 : 0;
   pl->lg_own = lg_own ? 1 : 0;
-  pl->o_lg = lg_own ? (int)take(lg_bytes, 128)
+  pl->o_lg = lg_in_bd ? pl->o_bd
+             : lg_own ? (int)take(lg_bytes, 128)
              : lg_in_d ? pl->o_ring_d + (int)(x_fits ? align_up(MM * H * 2, 128) : 0)
                        : pl->o_ring_gu + pl->wr_bytes_max;
   pl->o_bar = (int)take(bar_bytes, 16);
@@ -224,7 +246,7 @@ bool make_tc_plan(const moe_config& c, int sm_count, size_t smem_limit, moe::TcP
   pl->o_ppos = (int)take(NP * 4, 16);
   pl->o_union = (int)take(UMAX * 4, 16);
   pl->o_poff = (int)take((UMAX + 1) * 4, 16);
-  pl->o_dsm = (int)take(NP * nrd_max * 4, 16);
+  pl->o_dsm = (int)take(dsm_bytes, 16);
   pl->smem_bytes = (int)(off + 1024);
   return (size_t)pl->smem_bytes <= smem_limit;
 }
@@ -291,6 +313,22 @@ bool encode_w13_maps_repacked(const void* w13r, size_t Eall, size_t H, size_t I,
       return false;
   }
   return true;
+}
+
+// The down code map of k_tc's tensor-core down over w2_codes [Eall*H][I]
+// (4-bit elements, I/2 bytes a row): a box is one 128-element K-chunk of 128
+// rows, unpacked to 16 bytes per 16 codes with a 128-byte swizzle.
+bool encode_w2_map(const void* w2c, size_t Eall, size_t H, size_t I, CUtensorMap* map) {
+  EncodeTiledFn enc = encode_tiled();
+  if (!enc) return false;
+  if (reinterpret_cast<uintptr_t>(w2c) & 31) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)I, (cuuint64_t)(Eall * H)};
+  const cuuint64_t strides[1] = {(cuuint64_t)(I / 2)};
+  const cuuint32_t box[2] = {128, 128};
+  const cuuint32_t es[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 2, const_cast<void*>(w2c), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
@@ -408,6 +446,8 @@ moe_status moe_create(const moe_config* cfg, moe_ctx** out) {
   const size_t o_tlog = take(MM * E * sizeof(unsigned long long));
   const size_t o_th = take(NPF * I * sizeof(float));
   const size_t o_tcnt = take(2 * UMAXF * moe::kTcCntStride * sizeof(unsigned));
+  const size_t o_typ = take(NPF * H * sizeof(float));
+  const size_t o_tdc = take(2 * moe::kTcCntStride * sizeof(unsigned));
   ctx->ws_bytes = off;
   if (cudaMalloc(&ctx->ws_base, ctx->ws_bytes) != cudaSuccess) {
     cudaGetLastError();
@@ -440,6 +480,8 @@ moe_status moe_create(const moe_config* cfg, moe_ctx** out) {
   ctx->tws.logits = reinterpret_cast<unsigned long long*>(b + o_tlog);
   ctx->tws.h = reinterpret_cast<float*>(b + o_th);
   ctx->tws.hcnt = reinterpret_cast<unsigned*>(b + o_tcnt);
+  ctx->tws.ypart = reinterpret_cast<float*>(b + o_typ);
+  ctx->tws.dcnt = reinterpret_cast<unsigned*>(b + o_tdc);
   ctx->tws.epoch = w.ctrl + 6;
 
   // launch shapes
@@ -570,6 +612,8 @@ moe_status moe_load_experts(moe_ctx* ctx, const float* router_w, const uint8_t* 
                             ? encode_w13_maps_repacked(w13_codes, Eall, H, I, ctx->tplan.ks, ctx->maps.m)
                             : encode_w13_maps(w13_codes, Eall, H, I, ctx->tplan.ks, ctx->maps.m);
     if (!enc_ok) return MOE_ERR_INVALID_ARG;
+    if (ctx->tplan.mma_down && (!encode_w2_map(w2_codes, Eall, H, I, &ctx->maps.w2) || !aligned16(w2_scales)))
+      return MOE_ERR_INVALID_ARG;
   }
   ctx->wr = router_w;
   ctx->w13c = w13_codes;
@@ -690,7 +734,9 @@ moe_status moe_plan_query(const moe_config* cfg, int32_t sm_count, size_t smem_l
                          "\"o_sfb\": %d, \"o_ring_d\": %d, \"o_h\": %d, \"o_bar\": %d, \"o_misc\": %d, "
                          "\"o_ids\": %d, \"o_w\": %d, \"o_pm\": %d, \"o_ppos\": %d, \"o_union\": %d, "
                          "\"o_poff\": %d, \"o_dsm\": %d, \"sc_bytes\": %d, \"bx_bytes\": %d, "
-                         "\"max_pairs\": %d, \"max_union\": %d, \"o_lg\": %d, \"tmem_cols\": %d, \"lg_own\": %d}}",
+                         "\"max_pairs\": %d, \"max_union\": %d, \"o_lg\": %d, \"tmem_cols\": %d, \"lg_own\": %d, "
+                         "\"mma_down\": %d, \"dkch\": %d, \"o_bd\": %d, \"bd_bytes\": %d, \"o_dsc\": %d, "
+                         "\"o_dtoff\": %d}}",
                          (tc || ok) ? "true" : "false", tc ? "tc" : "fused", pl.G, moe::kFusedThreads, pl.smem_bytes,
                          pl.slot_gu, pl.ns_gu, pl.slot_d, pl.ns_d, pl.rpc_max, pl.wr_bytes_max, pl.o_act, pl.o_dsm,
                          pl.o_ring_gu, pl.o_ring_d, pl.o_h, pl.hslot, pl.hpairs, pl.x_staged, tok ? "true" : "false",
@@ -698,7 +744,8 @@ moe_status moe_plan_query(const moe_config* cfg, int32_t sm_count, size_t smem_l
                          tp.ns_d, tp.slot_d, tp.rpc_max, tp.hslot, tp.hpairs, tp.wr_bytes_max, tp.x_staged,
                          tp.o_ring_gu, tp.o_bx, tp.o_sf, tp.o_sc, tp.o_sfb, tp.o_ring_d, tp.o_h, tp.o_bar, tp.o_misc,
                          tp.o_ids, tp.o_w, tp.o_pm, tp.o_ppos, tp.o_union, tp.o_poff, tp.o_dsm, tp.sc_bytes,
-                         tp.bx_bytes, tp.max_pairs, tp.max_union, tp.o_lg, tp.tmem_cols, tp.lg_own);
+                         tp.bx_bytes, tp.max_pairs, tp.max_union, tp.o_lg, tp.tmem_cols, tp.lg_own, tp.mma_down, tp.dkch,
+                         tp.o_bd, tp.bd_bytes, tp.o_dsc, tp.o_dtoff);
   if (n < 0 || (size_t)n >= len) return MOE_ERR_INVALID_ARG;
   return (tc || ok) ? MOE_OK : MOE_ERR_UNSUPPORTED;
 }
@@ -737,11 +784,11 @@ moe_status moe_query(const moe_ctx* ctx, char* buf, size_t len) {
                  "\"variant\": \"tc\", \"kernels\": [\"k_tc\"], \"grid\": [%d], \"threads\": %d, "
                  "\"smem\": %d, \"gate_up\": \"tcgen05.mma kind::mxf8f6f4 block_scale M=128 N=%d\", "
                  "\"units_per_tile\": %d, \"kchunks_per_stage\": %d, \"ring_gu\": [%d, %d], \"ring_d\": [%d, %d], "
-                 "\"x_staged\": %d, \"pdl\": true, \"pre_rmsnorm\": %s, \"shared_expert\": %s, "
+                 "\"x_staged\": %d, \"down\": \"%s\", \"pdl\": true, \"pre_rmsnorm\": %s, \"shared_expert\": %s, "
                  "\"fp8_intermediate\": %s, \"hidden\": %d, \"inter\": %d, \"num_experts\": %d, \"top_k\": %d, "
                  "\"max_tokens\": %d}",
                  ctx->dev, ctx->sm_count, tp.G, moe::kTcThreads, tp.smem_bytes, tp.nb_max, tp.tu_max, tp.ks, tp.ns_gu,
-                 tp.slot_gu, tp.ns_d, tp.slot_d, tp.x_staged, (c.flags & MOE_FLAG_PRE_RMSNORM) ? "true" : "false",
+                 tp.slot_gu, tp.ns_d, tp.slot_d, tp.x_staged, tp.mma_down ? "tensor_cores" : "cuda_cores", (c.flags & MOE_FLAG_PRE_RMSNORM) ? "true" : "false",
                  (c.flags & MOE_FLAG_SHARED_EXPERT) ? "true" : "false",
                  (c.flags & MOE_FLAG_FP8_INTERMEDIATE) ? "true" : "false", c.hidden, c.inter, c.num_experts, c.top_k,
                  c.max_tokens);

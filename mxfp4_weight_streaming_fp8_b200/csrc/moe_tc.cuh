@@ -89,17 +89,29 @@ struct TcPlan {
   int tmem_cols; // tensor-memory columns allocated (power of two)
   int bx_bytes;
   int smem_bytes;  // including 1 KB of alignment slack
+  // tensor-core down projection (mma_down): tiles of 128 output rows x up to
+  // kTcDownPairs pairs of one entry; W2 stages share the gate/up ring (16 KB
+  // slots), h of the pairs is the B operand (E4M3, two buffers)
+  int mma_down;
+  int dkch;      // K-chunks of the down projection (I / 128)
+  int o_bd;      // [2][dkch][4][8][128 B] B operand buffers
+  int bd_bytes;  // one buffer
+  int o_dsc;     // [2][kTcDownPairs] per-pair h scales
+  int o_dtoff;   // [max_union + 1] first down tile of each entry
 };
 
 constexpr int kTcXRegs = 8;    // uint4 of a token's x per lane per pass when M >= 2
 constexpr int kTcCntStride = 32;  // u32 words between per-entry counters (one 128-byte line each)
 constexpr int kTcMaxTiles = 64;   // gate/up tiles per CTA
 constexpr int kTcWarpGate = 3;    // polls the entry counters for the CTA
+constexpr int kTcDownPairs = 16;  // pairs per tensor-core down tile: N = 2 x pairs (h = hi + lo/16)
+constexpr int kTcWarpBuild = 8;   // warps 8..15 build the down tiles' B operands
 
 // The gate/up code maps, passed by value as a __grid_constant__ kernel
 // parameter (TMA reads its descriptor from parameter space).
 struct TcMaps {
   CUtensorMap m[kTcMaxUnits];  // map n-1 loads n units x ks K-chunks
+  CUtensorMap w2;              // down codes [Eall*H rows][I] 4-bit: 128 rows x one 128-element K-chunk
 };
 
 struct TcWs {
@@ -108,6 +120,8 @@ struct TcWs {
   float* h;                    // [pairs][I] SwiGLU output per (token, slot) pair
   unsigned* hcnt;              // [2][max_union * kTcCntStride] gate/up tiles done per entry, by launch parity
   unsigned* epoch;             // launch counter
+  float* ypart;                // [pairs][H] tensor-core down: each pair's down output (fp32)
+  unsigned* dcnt;              // [2][kTcCntStride] CTAs done with their down tiles, by launch parity
 };
 
 __device__ __forceinline__ void tc_trace(const Params& p, int slot) { trace_stamp(p, slot); }
@@ -226,6 +240,13 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, i
       "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], "
       "[%6];" ::"r"(smem_u32(dst)),
       "l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int c0, int c1, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          smem_u32(dst)),
+      "l"(map), "r"(c0), "r"(c1), "r"(smem_u32(bar))
       : "memory");
 }
 __device__ __forceinline__ void prefetch_tensormap(const void* map) {
@@ -376,7 +397,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc(Params p, TcWs tw, TcPlan 
   uint64_t* sc_full = wr_bar + 1;   // [2] a tile's scale bytes landed
   uint64_t* sc_empty = sc_full + 2;  // [2] its scale factors are in tensor memory (4 warps)
   uint64_t* sf_ready = sc_empty + 2; // [2] same, for the MMA warp
-  unsigned* done_d = reinterpret_cast<unsigned*>(sf_ready + 2);  // [kMaxSlots]
+  uint64_t* b_full = sf_ready + 2;   // [2] a down tile's B operand built (builder warps)
+  uint64_t* b_empty = b_full + 2;    // [2] its MMAs are done with it
+  uint64_t* dsc_full = b_empty + 2;  // [4] a down tile's pair scales written (builder warps)
+  unsigned* done_d = reinterpret_cast<unsigned*>(dsc_full + 4);  // [kMaxSlots]
   float* s_amax = reinterpret_cast<float*>(smem + pl.o_misc);  // [32]
   float* s_xs = s_amax + kMaxTokens;                           // [32]
   float* s_rn = s_xs + kMaxTokens;                             // [32]
@@ -391,6 +415,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc(Params p, TcWs tw, TcPlan 
   int* s_union = reinterpret_cast<int*>(smem + pl.o_union);
   int* s_poff = reinterpret_cast<int*>(smem + pl.o_poff);
   float* dsm = reinterpret_cast<float*>(smem + pl.o_dsm);
+  uint8_t* bd = smem + pl.o_bd;                                   // mma_down: [2] B operand buffers
+  float* s_dsc = reinterpret_cast<float*>(smem + pl.o_dsc);       // mma_down: [4][kTcDownPairs] pair h scales
+  int* s_dtoff = reinterpret_cast<int*>(smem + pl.o_dtoff);       // mma_down: [max_union + 1]
   uint8_t* ring_gu = smem + pl.o_ring_gu;
   uint8_t* bx = smem + pl.o_bx;
   uint8_t* scbuf = smem + pl.o_sc;
@@ -431,6 +458,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc(Params p, TcWs tw, TcPlan 
   }
   if (tid == 32 * kTcWarpProdGu) {
     for (int n = 0; n < kTcMaxUnits; ++n) prefetch_tensormap(&maps.m[n]);
+    if (pl.mma_down) prefetch_tensormap(&maps.w2);
   }
   if (tid == 0) {
     mbar_init(wr_bar, 1);
@@ -438,6 +466,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc(Params p, TcWs tw, TcPlan 
       mbar_init(sc_full + i, 1);
       mbar_init(sc_empty + i, 4);
       mbar_init(sf_ready + i, 4);
+      mbar_init(b_full + i, kTcWarps - kTcWarpBuild);
+      mbar_init(b_empty + i, 1);
+      mbar_init(dsc_full + 2 * i, kTcWarps - kTcWarpBuild);
+      mbar_init(dsc_full + 2 * i + 1, kTcWarps - kTcWarpBuild);
     }
     fence_mbar_init();
     if (ne > 0) {
@@ -449,6 +481,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc(Params p, TcWs tw, TcPlan 
   if (tid == 0) {
     s_int[1] = (int)(ld_relaxed_u32(tw.epoch) + 1u);
     s_int[2] = 0;
+    s_int[5] = 0;  // epilogue warps done with their down tiles
     if constexpr (kShared) {
       s_union[0] = E;
       s_poff[0] = 0;
@@ -475,6 +508,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc(Params p, TcWs tw, TcPlan 
   if (b == 0) {
     unsigned* other = tw.hcnt + (size_t)((epoch + 1) & 1) * cstride;
     for (int i = tid; i < pl.max_union; i += kTcThreads) other[i * kTcCntStride] = 0u;
+    if (tid == 0) tw.dcnt[(size_t)((epoch + 1) & 1) * kTcCntStride] = 0u;
   }
 
   // 8 bf16 of x (group i of M*H/8), normalised when the layer normalises
@@ -856,6 +890,38 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc(Params p, TcWs tw, TcPlan 
   // one verdict for the CTA: after a routing wait ran out, no role starts
   ok = __syncthreads_and(ok ? 1 : 0) != 0;
   const int U = s_int[0];
+  // tensor-core down tiles, entry-major: entry u has ceil(pairs / kTcDownPairs)
+  // pair groups x H/128 row blocks; s_dtoff[u] = first tile of entry u
+  const int RB = H / 128;
+  if (pl.mma_down) {
+    if (warp == 0) {
+      const int per = (U + 31) / 32, ua = min(U, lane * per), ubd = min(U, ua + per);
+      int cnt = 0;
+      for (int u = ua; u < ubd; ++u) cnt += (s_poff[u + 1] - s_poff[u] + kTcDownPairs - 1) / kTcDownPairs * RB;
+      int ex = cnt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, ex, o);
+        if (lane >= o) ex += y;
+      }
+      ex -= cnt;
+      for (int u = ua; u < ubd; ++u) {
+        s_dtoff[u] = ex;
+        ex += (s_poff[u + 1] - s_poff[u] + kTcDownPairs - 1) / kTcDownPairs * RB;
+      }
+      if (lane == 31) s_dtoff[U] = ex + 0;  // lane 31 holds the total (its range may be empty)
+    }
+    __syncthreads();
+  }
+  const int D = pl.mma_down ? s_dtoff[U] : 0;
+  const int my_dtiles = (b < D) ? (D - b + G - 1) / G : 0;
+  // down tile d -> entry u (hint: advances monotonically), pair group g, row block R
+  auto dtile_of = [&](int d, int& u, int& g, int& R) {
+    while (s_dtoff[u + 1] <= d) ++u;
+    const int rem = d - s_dtoff[u];
+    g = rem / RB;
+    R = rem - g * RB;
+  };
   tc_trace(p, 4);
 
   // ---------------- gate/up schedule: flat units, tiles dealt round robin
@@ -923,6 +989,28 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc(Params p, TcWs tw, TcPlan 
           if (++slot == pl.ns_gu) { slot = 0; ph ^= 1u; reuse = true; }
         }
       }
+      // tensor-core down tiles: the 128 rows' E8M0 scales (one copy, 128 x
+      // I/32 bytes), then one stage per K-chunk of 128: a 128 x 128 box of
+      // W2 codes (16 KB unpacked, the same slot shape as a 16-unit gate/up
+      // stage)
+      int du = 0;
+      for (int k = 0; k < my_dtiles && ok; ++k) {
+        int g, R;
+        dtile_of(b + k * G, du, g, R);
+        const int it = my_tiles + k, sb = it & 1;
+        const int row0 = s_union[du] * H + R * 128;
+        if (it >= 2 && !mbar_wait_ok(sc_empty + sb, ((it >> 1) - 1) & 1, p)) { ok = false; break; }
+        mbar_expect_tx(sc_full + sb, (unsigned)(128 * (I / 32)));
+        tma_load_1d(scbuf + (size_t)sb * scb, p.w2s + (size_t)row0 * (I / 32), (unsigned)(128 * (I / 32)),
+                    sc_full + sb);
+        for (int kc = 0; kc < pl.dkch; ++kc, ++stage) {
+          if (reuse && !mbar_wait_ok(empty_gu + slot, ph ^ 1u, p)) { ok = false; break; }
+          mbar_expect_tx(full_gu + slot, 128u * 64u);
+          tma_load_2d(ring_gu + (size_t)slot * pl.slot_gu, &maps.w2, kc * 128, row0, full_gu + slot);
+          if (++slot == pl.ns_gu) { slot = 0; ph ^= 1u; reuse = true; }
+        }
+      }
+      if (my_dtiles > 0) tc_trace(p, 59);
     }
   } else if (warp == kTcWarpMma) {
     // ---------------- MMA issue (one thread); descriptors move by adding the
@@ -967,10 +1055,52 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc(Params p, TcWs tw, TcPlan 
         if (++slot == pl.ns_gu) { slot = 0; ph ^= 1u; }
       }
     }
+    // tensor-core down tiles: A = 128 W2 rows (slot, SBO 1 KB), B = the
+    // tile's h codes (buffer k & 1: K-chunk kc at kc * 4 KB, N <= 32 rows),
+    // scale factors of A in the tile buffer's columns, B's all 1.0
+    const uint64_t bdd0 = umma_desc_sw128(smem_u32(bd), 1024u);
+    int du = 0;
+    for (int k = 0; k < my_dtiles && ok; ++k) {
+      int g, R;
+      dtile_of(b + k * G, du, g, R);
+      const int np_t = min(kTcDownPairs, s_poff[du + 1] - s_poff[du] - kTcDownPairs * g);
+      const int nn = kFp8H ? np_t : 2 * np_t;
+      uint32_t idd[4];
+#pragma unroll
+      for (int kb = 0; kb < 4; ++kb) idd[kb] = umma_idesc_mx(max(8, (nn + 7) / 8 * 8), kb);
+      const int it = my_tiles + k, buf = it & 1, bb = k & 1;
+      const uint32_t acc_col = tmem + (uint32_t)(buf * kTcAccCols);
+      const uint32_t sf_base = tmem + (uint32_t)(kTcSfCol + 4 * KCH * buf);
+      if (it >= 2 && !mbar_wait_warp(acc_empty + buf, ((it >> 1) - 1) & 1, p)) { ok = false; break; }
+      if (!mbar_wait_warp(sf_ready + buf, (it >> 1) & 1, p)) { ok = false; break; }
+      if (!mbar_wait_warp(b_full + bb, (k >> 1) & 1, p)) { ok = false; break; }
+      tc_fence_after();
+      const uint64_t bdb = bdd0 + (uint64_t)((bb * pl.bd_bytes) >> 4);
+      for (int kc = 0; kc < pl.dkch; ++kc, ++stage) {
+        if (!mbar_wait_warp(full_gu + slot, ph, p)) { ok = false; break; }
+        if (lane == 0) {
+          tc_fence_after();
+          const uint64_t adc = ad0 + (uint64_t)slot * slot_step;
+          const uint64_t bdc = bdb + (uint64_t)kc * 256u;  // 4 KB per K-chunk
+          const uint32_t sfa = sf_base + 4u * (uint32_t)kc;
+          umma_mx(acc_col, adc, bdc, idd[0], kc > 0 ? 1u : 0u, sfa, sfb_col);
+          umma_mx(acc_col, adc + 2, bdc + 2, idd[1], 1u, sfa, sfb_col);
+          umma_mx(acc_col, adc + 4, bdc + 4, idd[2], 1u, sfa, sfb_col);
+          umma_mx(acc_col, adc + 6, bdc + 6, idd[3], 1u, sfa, sfb_col);
+          tc_commit(empty_gu + slot);
+          if (kc == pl.dkch - 1) {
+            tc_commit(acc_full + buf);
+            tc_commit(b_empty + bb);
+          }
+        }
+        __syncwarp();
+        if (++slot == pl.ns_gu) { slot = 0; ph ^= 1u; }
+      }
+    }
     tc_trace(p, 6);
   } else if (warp == kTcWarpProdD) {
     // ---------------- down producer: rows [r0, r0+nrd) of every entry, in order
-    if (lane == 0 && nrd > 0) {
+    if (lane == 0 && nrd > 0 && !pl.mma_down) {
       // the gate/up stream goes first: wait for its first stage to land
       if (my_tiles > 0 && !mbar_wait_ok(full_gu, 0, p)) ok = false;
       int slot = 0;
@@ -1003,21 +1133,29 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc(Params p, TcWs tw, TcPlan 
     // holds, in column 4*kc + j, the scale word (4 E8M0 bytes, K blocks
     // 4kc..4kc+3) of tile row L + 32j (unit (L+32j)/8; its rows 0..3 gate,
     // 4..7 up). The first call also writes the tokens' unit scales.
+    // A down tile (ti >= my_tiles): row r is W2 row row0 + r, whose scale
+    // bytes sit at r * I/32 in the buffer; dkch K-chunks.
     auto write_sf = [&](int ti) -> bool {
       const int sb = ti & 1;
       if (!mbar_wait_warp(sc_full + sb, (ti >> 1) & 1, p)) return false;
-      const int t = b + ti * G;
-      const int f0 = t * tu, nu = min(T, f0 + tu) - f0;
       const uint8_t* sc = scbuf + (size_t)sb * scb;
       const uint32_t lane_base = (uint32_t)(32 * q) << 16;
       const uint32_t col = tmem + (uint32_t)(kTcSfCol + 4 * KCH * sb) + lane_base;
-      int rowoff[4];
+      int rowoff[4], nkc = KCH;
+      if (ti < my_tiles) {
+        const int t = b + ti * G;
+        const int f0 = t * tu, nu = min(T, f0 + tu) - f0;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int r = lane + 32 * j, g = r >> 3, i8 = r & 7;
-        rowoff[j] = (g < nu) ? ((i8 < 4) ? 4 * g + i8 : 4 * pl.tu_max + 4 * g + (i8 - 4)) * (H / 32) : -1;
+        for (int j = 0; j < 4; ++j) {
+          const int r = lane + 32 * j, g = r >> 3, i8 = r & 7;
+          rowoff[j] = (g < nu) ? ((i8 < 4) ? 4 * g + i8 : 4 * pl.tu_max + 4 * g + (i8 - 4)) * (H / 32) : -1;
+        }
+      } else {
+        nkc = pl.dkch;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) rowoff[j] = (lane + 32 * j) * (I / 32);
       }
-      for (int kc = 0; kc < KCH; ++kc) {
+      for (int kc = 0; kc < nkc; ++kc) {
         uint32_t w[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j)
@@ -1037,9 +1175,46 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc(Params p, TcWs tw, TcPlan 
       }
       return true;
     };
-    if (ok && my_tiles > 0 && !write_sf(0)) ok = false;
-    if (ok && my_tiles > 1 && !write_sf(1)) ok = false;
-    for (int it = 0; it < my_tiles && ok; ++it) {
+    const int all_tiles = my_tiles + my_dtiles;
+    if (ok && all_tiles > 0 && !write_sf(0)) ok = false;
+    if (ok && all_tiles > 1 && !write_sf(1)) ok = false;
+    int du = 0;
+    for (int it = 0; it < all_tiles && ok; ++it) {
+      if (it >= my_tiles) {
+        // ---- tensor-core down tile: y of each pair of the group for the
+        //      tile's 128 output rows (lane = row), h = scale * (hi + lo/16)
+        const int k = it - my_tiles, buf = it & 1;
+        int g, R;
+        dtile_of(b + k * G, du, g, R);
+        const int pb0 = s_poff[du] + kTcDownPairs * g, np_t = min(kTcDownPairs, s_poff[du + 1] - pb0);
+        if (!mbar_wait_warp(acc_full + buf, (it >> 1) & 1, p)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t v[32];
+        tmem_ld32(tmem + (uint32_t)(buf * kTcAccCols) + ((uint32_t)(32 * q) << 16), v);
+        // the pair scales of tile k (ring of 4: the builders reuse this entry
+        // for tile k + 4 only after tile k + 2's MMAs, which wait for this
+        // epilogue to release the accumulator below)
+        if (!mbar_wait_warp(dsc_full + (k & 3), (k >> 2) & 1, p)) { ok = false; break; }
+        float dsc[kTcDownPairs];
+#pragma unroll
+        for (int qq = 0; qq < kTcDownPairs; ++qq) dsc[qq] = s_dsc[(k & 3) * kTcDownPairs + qq];
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(acc_empty + buf);
+        if (it + 2 < all_tiles && !write_sf(it + 2)) { ok = false; break; }
+        const int row = R * 128 + 32 * q + lane;
+#pragma unroll
+        for (int qq = 0; qq < kTcDownPairs; ++qq) {
+          if (qq < np_t) {
+            const float val = kFp8H ? __uint_as_float(v[qq]) * dsc[qq]
+                                    : (__uint_as_float(v[2 * qq]) + __uint_as_float(v[2 * qq + 1]) * 0.0625f) * dsc[qq];
+            tw.ypart[(size_t)(pb0 + qq) * H + row] = val;
+          }
+        }
+        if (q == 0 && k == 0) tc_trace(p, 24);
+        if (q == 0 && k == my_dtiles - 1) tc_trace(p, 25);
+        continue;
+      }
       const int t = b + it * G;
       const int f0 = t * tu, f1 = min(T, f0 + tu), nu = f1 - f0;
       const int buf = it & 1;
@@ -1051,8 +1226,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc(Params p, TcWs tw, TcPlan 
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(acc_empty + buf);
-      // the MMAs of tile it are complete: its scale-factor buffer takes tile it+2
-      if (it + 2 < my_tiles && !write_sf(it + 2)) { ok = false; break; }
       const int r = 32 * q + lane, g = r >> 3, i8 = r & 7;
       float upv[32];
 #pragma unroll
@@ -1079,6 +1252,19 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc(Params p, TcWs tw, TcPlan 
       if (lane == 0 && atom_add_acqrel_cta_smem(s_tdone + it, 1u) == 3u)
         for (int u = f0 / upe; u <= (f1 - 1) / upe; ++u) red_release_add_u32(hcnt + u * kTcCntStride, 1u);
       if (q == 0 && it == my_tiles - 1) tc_trace(p, 50);
+      // the MMAs of tile it are complete: its scale-factor buffer takes tile
+      // it+2. Only after the publish: tile it+2 may be a down tile, whose
+      // scales the producer issues behind down stages that wait (through the
+      // B operand) for every CTA's h, this one's included.
+      if (it + 2 < all_tiles && !write_sf(it + 2)) { ok = false; break; }
+    }
+    if (pl.mma_down && ok) {
+      // this CTA's down tiles are all in ypart: the last of the four warps
+      // (CTA-scope acq_rel, so it sees the others' stores) counts the CTA in,
+      // with release at GPU scope
+      __syncwarp();
+      if (lane == 0 && atom_add_acqrel_cta_smem(reinterpret_cast<unsigned*>(s_int + 5), 1u) == 3u)
+        red_release_add_u32(tw.dcnt + (size_t)(epoch & 1) * kTcCntStride, 1u);
     }
     tc_trace(p, 7);
   }
@@ -1111,59 +1297,148 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc(Params p, TcWs tw, TcPlan 
     ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
   }
 
-  // ---------------- down (CUDA cores): every warp once its role is done.
-  //   Items (entry, 9 output rows) in entry order; each waits for its
-  //   entry's flag (h complete on every CTA) and its chunk.
-  {
-    const int per = d_items;
-    const int total = U * per;
-    for (;;) {
-      if (!ok) break;  // a wait of this warp ran out: the step's output is lost anyway
-      int it = 0;
-      if (lane == 0) it = atomicAdd(&s_int[2], 1);
-      it = __shfl_sync(0xffffffffu, it, 0);
-      if (it >= total) break;
-      const int u = it / per, gd = it - u * per;
-      const int slot = u % pl.ns_d, use = u / pl.ns_d;
-      const int pb = s_poff[u], pe = s_poff[u + 1];
-      // the slot's previous use is fully consumed, so the parity waits
-      // below cannot see an earlier phase
-      if (use > 0 && lane == 0) smem_count_wait(done_d + slot, (unsigned)(use * per), p);
-      __syncwarp();
-      if (it == 0) tc_trace(p, 51);
-      if (it == total - 1) tc_trace(p, 54);
-      if (!wait_flag_warp(p, s_hready + u)) ok = false;
-      if (u == U - 1 && gd == 0) tc_trace(p, 9);
-      if (it == 0) tc_trace(p, 52);
-      if (it == total - 1) tc_trace(p, 55);
-      if (!mbar_wait_warp(full_d + slot, use & 1, p)) ok = false;
-      if (it == 0) tc_trace(p, 53);
-      if (it == total - 1) tc_trace(p, 56);
-      DChunk ch;
-      size_t sa0;
-      unsigned sn;
-      d_layout(p, s_union[u], r0, nrd, ring_d + (size_t)slot * pl.slot_d, &ch, &sa0, &sn);
-      const int a = gd * kDownRowsPerItem, cnt = min(kDownRowsPerItem, nrd - a);
-      tc_d_item<kFp8H>(p, tw, ch, a, cnt, pb, pe, dsm, pl.rpc_max, it == 0 ? 61 : -1);
-      if (it == 0) tc_trace(p, 57);
-      if (it == total - 1) tc_trace(p, 58);
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(empty_d + slot);
-        atomicAdd(done_d + slot, 1u);
+  if (pl.mma_down) {
+    // ---------------- tensor-core down: the builder warps turn each tile's
+    //   pairs' h (read from L2 once the entry is complete on every CTA) into
+    //   the B operand: per pair an fp32 scale amax/448 and E4M3 codes of
+    //   h/scale (row 2q), plus (unless kFp8H) the codes of 16x the rounding
+    //   residual (row 2q+1), so the MMA sums hi + lo/16, within 2^-8 of h.
+    //   Then every CTA waits for all CTAs' tiles and combines its rows.
+    if (warp >= kTcWarpBuild && ok) {
+      const int wb = warp - kTcWarpBuild, nwb = kTcWarps - kTcWarpBuild;
+      const int nf4 = I / 128;  // float4 of h per lane (I <= 1024)
+      int du = 0;
+      for (int k = 0; k < my_dtiles; ++k) {
+        int g, R;
+        dtile_of(b + k * G, du, g, R);
+        const int pb0 = s_poff[du] + kTcDownPairs * g, np_t = min(kTcDownPairs, s_poff[du + 1] - pb0);
+        const int bb = k & 1;
+        if (!wait_flag_warp(p, s_hready + du)) { ok = false; break; }
+        if (k >= 2 && !mbar_wait_warp(b_empty + bb, ((k >> 1) - 1) & 1, p)) { ok = false; break; }
+        uint8_t* bdb = bd + (size_t)bb * pl.bd_bytes;
+        for (int qq = wb; qq < np_t; qq += nwb) {
+          const float4* hp = reinterpret_cast<const float4*>(tw.h + (size_t)(pb0 + qq) * I) + lane * nf4;
+          float4 hv[8];
+          float mx = 0.f;
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            hv[t] = (t < nf4) ? __ldcg(hp + t) : make_float4(0.f, 0.f, 0.f, 0.f);
+            mx = fmaxf(mx, fmaxf(fmaxf(fabsf(hv[t].x), fabsf(hv[t].y)), fmaxf(fabsf(hv[t].z), fabsf(hv[t].w))));
+          }
+          const float amax = warp_max(mx), inv = h_fp8_inv(amax);
+          const int nhi = kFp8H ? qq : 2 * qq;
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            if (t < nf4) {
+              const int kk = (lane * nf4 + t) * 4;
+              const float y0 = __fmul_rn(hv[t].x, inv), y1 = __fmul_rn(hv[t].y, inv);
+              const float y2 = __fmul_rn(hv[t].z, inv), y3 = __fmul_rn(hv[t].w, inv);
+              const uint32_t c01 = f32x2_to_e4m3x2(y0, y1), c23 = f32x2_to_e4m3x2(y2, y3);
+              *reinterpret_cast<uint32_t*>(bdb + sw128_offset(nhi, kk, 4)) = c01 | (c23 << 16);
+              if constexpr (!kFp8H) {
+                const uint32_t h01 = e4m3x2_to_f16x2((uint16_t)c01), h23 = e4m3x2_to_f16x2((uint16_t)c23);
+                const float2 q01 = __half22float2(*reinterpret_cast<const __half2*>(&h01));
+                const float2 q23 = __half22float2(*reinterpret_cast<const __half2*>(&h23));
+                const uint32_t l01 = f32x2_to_e4m3x2((y0 - q01.x) * 16.f, (y1 - q01.y) * 16.f);
+                const uint32_t l23 = f32x2_to_e4m3x2((y2 - q23.x) * 16.f, (y3 - q23.y) * 16.f);
+                *reinterpret_cast<uint32_t*>(bdb + sw128_offset(nhi + 1, kk, 4)) = l01 | (l23 << 16);
+              }
+            }
+          }
+          if (lane == 0) s_dsc[(k & 3) * kTcDownPairs + qq] = h_fp8_scale(amax);
+        }
+        // the codes are read by the tensor cores (async proxy)
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(b_full + bb);
+          mbar_arrive(dsc_full + (k & 3));
+        }
+        if (k == 0) tc_trace(p, 51);
       }
+      tc_trace(p, 52);
     }
     tc_trace(p, 10);
-    __syncthreads();
+    // grid-wide: every CTA's down tiles are in ypart once the count reaches G
+    if (tid == 0 && ok) {
+      const unsigned* c = tw.dcnt + (size_t)(epoch & 1) * kTcCntStride;
+      const long long t0 = clock64();
+      while (ld_acquire_u32g(c) < (unsigned)G) {
+        __nanosleep(128);
+        if (clock64() - t0 > p.spin_limit) {
+          atomicOr(p.ws.ctrl, kStatusTimeout);
+          ok = false;
+          break;
+        }
+      }
+    }
+    const bool all_ok = __syncthreads_and(ok ? 1 : 0) != 0;
     tc_trace(p, 11);
     // ---- A8: combine in slot order, bf16 out
-    for (int i = tid; i < M * nrd; i += kTcThreads) {
-      const int m = i / nrd, rl = i % nrd;
+    for (int i = tid; i < M * nrd && all_ok; i += kTcThreads) {
+      const int m = i / nrd, r = r0 + i % nrd;
       float acc = 0.f;
-      for (int s = 0; s < K; ++s) acc = fmaf(s_w[m * K + s], dsm[(size_t)s_ppos[m * K + s] * pl.rpc_max + rl], acc);
-      if constexpr (kShared) acc += dsm[(size_t)m * pl.rpc_max + rl];
-      p.y[(size_t)m * H + r0 + rl] = __float2bfloat16_rn(acc);
+      for (int s = 0; s < K; ++s)
+        acc = fmaf(s_w[m * K + s], __ldcg(tw.ypart + (size_t)s_ppos[m * K + s] * H + r), acc);
+      if constexpr (kShared) acc += __ldcg(tw.ypart + (size_t)m * H + r);
+      p.y[(size_t)m * H + r] = __float2bfloat16_rn(acc);
     }
+  } else {
+    // ---------------- down (CUDA cores): every warp once its role is done.
+    //   Items (entry, 9 output rows) in entry order; each waits for its
+    //   entry's flag (h complete on every CTA) and its chunk.
+    {
+      const int per = d_items;
+      const int total = U * per;
+      for (;;) {
+        if (!ok) break;  // a wait of this warp ran out: the step's output is lost anyway
+        int it = 0;
+        if (lane == 0) it = atomicAdd(&s_int[2], 1);
+        it = __shfl_sync(0xffffffffu, it, 0);
+        if (it >= total) break;
+        const int u = it / per, gd = it - u * per;
+        const int slot = u % pl.ns_d, use = u / pl.ns_d;
+        const int pb = s_poff[u], pe = s_poff[u + 1];
+        // the slot's previous use is fully consumed, so the parity waits
+        // below cannot see an earlier phase
+        if (use > 0 && lane == 0) smem_count_wait(done_d + slot, (unsigned)(use * per), p);
+        __syncwarp();
+        if (it == 0) tc_trace(p, 51);
+        if (it == total - 1) tc_trace(p, 54);
+        if (!wait_flag_warp(p, s_hready + u)) ok = false;
+        if (u == U - 1 && gd == 0) tc_trace(p, 9);
+        if (it == 0) tc_trace(p, 52);
+        if (it == total - 1) tc_trace(p, 55);
+        if (!mbar_wait_warp(full_d + slot, use & 1, p)) ok = false;
+        if (it == 0) tc_trace(p, 53);
+        if (it == total - 1) tc_trace(p, 56);
+        DChunk ch;
+        size_t sa0;
+        unsigned sn;
+        d_layout(p, s_union[u], r0, nrd, ring_d + (size_t)slot * pl.slot_d, &ch, &sa0, &sn);
+        const int a = gd * kDownRowsPerItem, cnt = min(kDownRowsPerItem, nrd - a);
+        tc_d_item<kFp8H>(p, tw, ch, a, cnt, pb, pe, dsm, pl.rpc_max, it == 0 ? 61 : -1);
+        if (it == 0) tc_trace(p, 57);
+        if (it == total - 1) tc_trace(p, 58);
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(empty_d + slot);
+          atomicAdd(done_d + slot, 1u);
+        }
+      }
+      tc_trace(p, 10);
+      __syncthreads();
+      tc_trace(p, 11);
+      // ---- A8: combine in slot order, bf16 out
+      for (int i = tid; i < M * nrd; i += kTcThreads) {
+        const int m = i / nrd, rl = i % nrd;
+        float acc = 0.f;
+        for (int s = 0; s < K; ++s) acc = fmaf(s_w[m * K + s], dsm[(size_t)s_ppos[m * K + s] * pl.rpc_max + rl], acc);
+        if constexpr (kShared) acc += dsm[(size_t)m * pl.rpc_max + rl];
+        p.y[(size_t)m * H + r0 + rl] = __float2bfloat16_rn(acc);
+      }
+    }
+  
   }
 
   // ---------------- teardown

@@ -25,6 +25,9 @@ MOE_FLAG_FP8_INTERMEDIATE = 0x8
 MOE_FLAG_CUDA_CORES = 0x10
 MOE_FLAG_TENSOR_CORES = 0x20
 MOE_TC_MIN_TOKENS = 2
+MOE_FLAG_TC_DOWN_MMA = 0x40
+MOE_FLAG_TC_DOWN_CUDA = 0x80
+MOE_TC_DOWN_MMA_MIN_TOKENS = 8
 MOE_LOAD_BORROW = 0x0
 MOE_LOAD_SKIP_VALIDATE = 0x1
 MOE_LOAD_COPY_REPACK = 0x2

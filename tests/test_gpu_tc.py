@@ -192,3 +192,62 @@ def test_copy_repack_cuda_core_kernel():
     ctx.load_experts(L.wr_d, *L.experts, repack=True)
     got = L.run(ctx)
     compare(L, got, L.oracle())
+
+
+# ---- the down projection on tensor cores (MOE_FLAG_TC_DOWN_MMA; the default
+#      from MOE_TC_DOWN_MMA_MIN_TOKENS tokens of max_tokens on)
+
+def _ctx_down(L, mma, flags=0, max_tokens=None):
+    f = flags | moe.MOE_FLAG_TENSOR_CORES | (moe.MOE_FLAG_TC_DOWN_MMA if mma else moe.MOE_FLAG_TC_DOWN_CUDA)
+    ctx = L.make_ctx(f, max_tokens=max_tokens)
+    q = ctx.query()
+    assert q["variant"] == "tc" and q["down"] == ("tensor_cores" if mma else "cuda_cores"), q
+    return ctx
+
+
+@pytest.mark.parametrize("shape,M,mode", [((256, 128, 16, 2), 3, "gap"), ((512, 256, 40, 6), 5, "gap"),
+                                          ((128, 128, 8, 8), 3, "natural"), ((1024, 512, 64, 8), 7, "zipf"),
+                                          ((384, 128, 12, 4), 4, "shared")])
+def test_mma_down_small_layers(shape, M, mode):
+    """Tiles of 128 output rows over several row blocks, pair groups of one
+    to many pairs, ragged unions."""
+    H, I, E, K = shape
+    L = Layer(H, I, E, K, M, seed=61, mode=mode)
+    got = L.run(_ctx_down(L, True))
+    worst = compare(L, got, L.oracle(), check_ids=(mode != "natural" or K < E))
+    print(f"k_tc down on tensor cores {shape} M={M}: worst y error {worst:.3f} of the bound")
+
+
+@pytest.mark.parametrize("M,mode", [(1, "gap"), (4, "distinct"), (8, "zipf"), (16, "shared")])
+def test_mma_down_ling(M, mode):
+    L = Layer(2560, 768, 256, 8, M, seed=62, mode=mode)
+    ctx = _ctx_down(L, True)
+    got = L.run(ctx)
+    compare(L, got, L.oracle())
+    assert torch.equal(L.run(ctx)["y"], got["y"])  # repeatable
+
+
+def test_mma_down_is_default_from_min_tokens():
+    L = Layer(2560, 768, 256, 8, 2, seed=63, mode="gap")
+    ctx = L.make_ctx(0, max_tokens=moe.MOE_TC_DOWN_MMA_MIN_TOKENS)
+    assert ctx.query()["down"] == "tensor_cores"
+    compare(L, L.run(ctx), L.oracle())
+    ctx = L.make_ctx(0, max_tokens=moe.MOE_TC_DOWN_MMA_MIN_TOKENS - 1)
+    assert ctx.query()["down"] == "cuda_cores"
+
+
+def test_mma_down_agrees_with_cuda_core_down():
+    L = Layer(2560, 768, 256, 8, 8, seed=64, mode="zipf")
+    a, b = L.run(_ctx_down(L, True)), L.run(_ctx_down(L, False))
+    assert np.array_equal(a["ids"], b["ids"])
+    ya, yb = a["y"].float(), b["y"].float()
+    assert torch.all((ya - yb).abs() <= 4e-3 * yb.norm(dim=1, keepdim=True))
+
+
+@pytest.mark.parametrize("M,mode", [(2, "gap"), (12, "zipf")])
+def test_mma_down_shared_expert_and_fp8_intermediate(M, mode):
+    from test_gpu_parity import _check_a8
+    L = Layer(2560, 768, 256, 8, M, seed=65, mode=mode, shared=True)
+    compare(L, L.run(_ctx_down(L, True, moe.MOE_FLAG_SHARED_EXPERT)), L.oracle())
+    L = Layer(2560, 768, 256, 8, M, seed=66, mode=mode, a8=True)
+    _check_a8(L, L.run(_ctx_down(L, True, moe.MOE_FLAG_FP8_INTERMEDIATE)))
