@@ -823,6 +823,59 @@ __device__ void topk_cta_small(const float* l, int E, int K, int* ids, float* wt
   }
 }
 
+// Top-k (K <= 8) of one token's E <= 512 logits with half a warp (lanes
+// 16h..16h+15, so a warp takes two tokens): lane l holds experts l + 16j;
+// K rounds of (lane's best untaken, the half's largest key, the lowest expert
+// holding it; shuffle butterflies within the half), ties to the lower expert;
+// softmax over the K kept as in topk_warp. Same result as topk_warp.
+template <int NJ2>
+__device__ __forceinline__ void topk_half(const float* l, int E, int K, int* ids, float* w) {
+  const int lane = threadIdx.x & 31, hl = lane & 15;
+  const unsigned hm = 0xFFFFu << (lane & 16);
+  unsigned key[NJ2];
+#pragma unroll
+  for (int j = 0; j < NJ2; ++j) {
+    const int e = hl + 16 * j;
+    key[j] = (e < E) ? fkey(l[e]) : 0u;  // 0: absent or taken (below every float's key)
+  }
+  unsigned sel = 0u;
+  int sel_e = 0;
+  for (int r = 0; r < K; ++r) {
+    unsigned bk = 0u;
+    int bj = 0;
+#pragma unroll
+    for (int j = 0; j < NJ2; ++j)
+      if (key[j] > bk) {
+        bk = key[j];
+        bj = j;
+      }
+    // the half's largest key, then the lowest expert holding it (butterflies
+    // within the half)
+    unsigned kmax = bk;
+#pragma unroll
+    for (int o = 8; o; o >>= 1) kmax = max(kmax, __shfl_xor_sync(hm, kmax, o));
+    int win = (bk == kmax && bk != 0u) ? hl + 16 * bj : 0x7fffffff;
+#pragma unroll
+    for (int o = 8; o; o >>= 1) win = min(win, __shfl_xor_sync(hm, win, o));
+#pragma unroll
+    for (int j = 0; j < NJ2; ++j)
+      if (hl + 16 * j == win) key[j] = 0u;
+    if (hl == r) {
+      sel = kmax;
+      sel_e = win;
+    }
+  }
+  const float top = fkey_value(__shfl_sync(hm, sel, lane & 16));
+  float ex = (hl < K) ? expf(fkey_value(sel) - top) : 0.f;
+  float z = ex;
+#pragma unroll
+  for (int o = 8; o; o >>= 1) z += __shfl_xor_sync(hm, z, o);
+  if (hl < K) {
+    ids[hl] = sel_e;
+    w[hl] = ex / z;
+  }
+}
+
 // Logits of this CTA's ne <= 2 router rows (wr_s, fp32, row-major) for one
 // token: every thread takes a strided share of both rows; warp sums, then
 // warp 0 sums the warps' partials in warp order and stores the tagged words

@@ -100,7 +100,7 @@ struct TcPlan {
   int o_dtoff;   // [max_union + 1] first down tile of each entry
 };
 
-constexpr int kTcXRegs = 8;    // uint4 of a token's x per lane per pass when M >= 2
+constexpr int kTcXU2 = 20;     // 4-element groups of a token's x a lane holds when M >= 2 (H <= 2560: one read)
 constexpr int kTcCntStride = 32;  // u32 words between per-entry counters (one 128-byte line each)
 constexpr int kTcMaxTiles = 64;   // gate/up tiles per CTA
 constexpr int kTcWarpGate = 3;    // polls the entry counters for the CTA
@@ -125,6 +125,13 @@ struct TcWs {
 };
 
 __device__ __forceinline__ void tc_trace(const Params& p, int slot) { trace_stamp(p, slot); }
+// An 8-byte L2 load the compiler may not repeat (asm volatile): a row loaded
+// once stays in registers instead of being re-read from L2.
+__device__ __forceinline__ uint2 ld_cg_v2_once(const uint2* p) {
+  uint2 v;
+  asm volatile("ld.global.cg.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+  return v;
+}
 __device__ __forceinline__ unsigned ld_acquire_u32g(const unsigned* p) {
   unsigned v;
   asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -531,41 +538,48 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc(Params p, TcWs tw, TcPlan 
   };
   const int nbg = pl.nb_max / 8;
   if (M >= 2) {
-    // ---- A9 + A1 + A2 for several tokens: one warp per token, over its x
-    //      row in chunks of kTcXRegs uint4 per lane (L2 reads). Pass 1: the
-    //      RMSNorm sum of squares (fixed order) and amax; the new amax is
-    //      bf16(fl32(amax * r)) (rounding is monotonic and symmetric). Pass 2:
-    //      the logits of the CTA's router rows (tagged stores) and the E4M3
-    //      codes straight into the MMA's B operand (K-major, 128-byte
-    //      swizzle; rows >= M are never read).
+    // ---- A9 + A1 + A2 for several tokens: one warp per token. Lane l holds
+    //      the 4-element groups l + 32j of the row (a single L2 read when the
+    //      row fits kTcXU2 groups per lane; else chunks, read twice). Pass 1:
+    //      the RMSNorm sum of squares (fixed order) and amax (the normalised
+    //      amax is bf16(fl32(amax * r)): rounding is monotonic and symmetric),
+    //      and without RMSNorm the router logits; pass 2: the logits of the
+    //      normalised row (with RMSNorm) and the E4M3 codes straight into the
+    //      MMA's B operand (K-major, 128-byte swizzle; rows >= M never read).
+    //      A lane's router values are one float4 per row and group, so the
+    //      warp reads each router row contiguously.
     if (ne > 0 && !mbar_wait_ok(wr_bar, 0, p)) ok = false;
     tc_trace(p, 14);
-    const int ng = H / 8;
+    const int n2 = H / 4;
+    const bool one = n2 <= 32 * kTcXU2;
     if (tid < kMaxTokens) s_xs[tid] = 1.f;
     __syncwarp();
     for (int m = warp; m < M; m += kTcWarps) {
-      const uint4* xg = reinterpret_cast<const uint4*>(p.x) + (size_t)m * ng;
-      float ss = 0.f, a = 0.f;
-      for (int c0 = 0; c0 < ng; c0 += 32 * kTcXRegs) {
-        uint4 xr[kTcXRegs];
+      const uint2* xg = reinterpret_cast<const uint2*>(p.x) + (size_t)m * n2;
+      uint2 xr[kTcXU2];
+      auto load_chunk = [&](int c0) {
 #pragma unroll
-        for (int j = 0; j < kTcXRegs; ++j) {
+        for (int j = 0; j < kTcXU2; ++j) {
           const int i = c0 + lane + 32 * j;
-          xr[j] = (i < ng) ? __ldcg(xg + i) : make_uint4(0u, 0u, 0u, 0u);
+          xr[j] = (i < n2) ? ld_cg_v2_once(xg + i) : make_uint2(0u, 0u);
         }
+      };
+      float ss = 0.f, a = 0.f;
+      for (int c0 = 0; c0 < n2; c0 += 32 * kTcXU2) {
+        load_chunk(c0);
 #pragma unroll
-        for (int j = 0; j < kTcXRegs; ++j) {
-          const uint32_t w[4] = {xr[j].x, xr[j].y, xr[j].z, xr[j].w};
-#pragma unroll
-          for (int t = 0; t < 4; ++t) {
-            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[t]));
-            ss = __fmaf_rn(f.x, f.x, ss);
-            ss = __fmaf_rn(f.y, f.y, ss);
-            a = fmaxf(a, fmaxf(fabsf(f.x), fabsf(f.y)));
-          }
+        for (int j = 0; j < kTcXU2; ++j) {
+          const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xr[j].x));
+          const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xr[j].y));
+          ss = __fmaf_rn(f0.x, f0.x, ss);
+          ss = __fmaf_rn(f0.y, f0.y, ss);
+          ss = __fmaf_rn(f1.x, f1.x, ss);
+          ss = __fmaf_rn(f1.y, f1.y, ss);
+          a = fmaxf(a, fmaxf(fmaxf(fabsf(f0.x), fabsf(f0.y)), fmaxf(fabsf(f1.x), fabsf(f1.y))));
         }
       }
       a = warp_max(a);
+      if (m == warp) tc_trace(p, 36);
       float r = 1.f;
       if (p.pre_rmsnorm) {
         ss = warp_sum(ss);
@@ -573,70 +587,76 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc(Params p, TcWs tw, TcPlan 
         a = __bfloat162float(__float2bfloat16_rn(__fmul_rn(a, r)));
       }
       const float inv = (a != 0.f) ? __fdiv_rn(448.f, a) : 0.f;
-      float acc[kMaxRowsPerCta];
+      // (reloaded) chunk, normalised in place with RMSNorm
+      auto norm_chunk = [&](int c0) {
+        if (!p.pre_rmsnorm) return;
 #pragma unroll
-      for (int el = 0; el < kMaxRowsPerCta; ++el) acc[el] = 0.f;
-      for (int c0 = 0; c0 < ng; c0 += 32 * kTcXRegs) {
-        uint4 xr[kTcXRegs];
-#pragma unroll
-        for (int j = 0; j < kTcXRegs; ++j) {
-          const int i = c0 + lane + 32 * j;
-          xr[j] = (i < ng) ? __ldcg(xg + i) : make_uint4(0u, 0u, 0u, 0u);
+        for (int j = 0; j < kTcXU2; ++j) {
+          const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xr[j].x));
+          const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xr[j].y));
+          const __nv_bfloat162 o0 = __floats2bfloat162_rn(__fmul_rn(f0.x, r), __fmul_rn(f0.y, r));
+          const __nv_bfloat162 o1 = __floats2bfloat162_rn(__fmul_rn(f1.x, r), __fmul_rn(f1.y, r));
+          xr[j] = make_uint2(*reinterpret_cast<const uint32_t*>(&o0), *reinterpret_cast<const uint32_t*>(&o1));
         }
+      };
+      for (int c0 = 0; c0 < n2; c0 += 32 * kTcXU2) {
+        if (!one) load_chunk(c0);
+        norm_chunk(c0);
 #pragma unroll
-        for (int j = 0; j < kTcXRegs; ++j) {
+        for (int j = 0; j < kTcXU2; ++j) {
           const int i = c0 + lane + 32 * j;
-          if (i >= ng) continue;
-          uint32_t w[4] = {xr[j].x, xr[j].y, xr[j].z, xr[j].w};
-          if (p.pre_rmsnorm) {
-#pragma unroll
-            for (int t = 0; t < 4; ++t) {
-              const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[t]));
-              const __nv_bfloat162 o = __floats2bfloat162_rn(__fmul_rn(f.x, r), __fmul_rn(f.y, r));
-              w[t] = *reinterpret_cast<const uint32_t*>(&o);
+          if (i < n2) {
+            if (p.pre_rmsnorm && b == 0 && p.out_xn) reinterpret_cast<uint2*>(p.out_xn)[(size_t)m * n2 + i] = xr[j];
+            uint32_t out = 0u;
+            if (a != 0.f) {
+              const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xr[j].x));
+              const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xr[j].y));
+              const uint32_t c0v = f32x2_to_e4m3x2(__fmul_rn(f0.x, inv), __fmul_rn(f0.y, inv));
+              const uint32_t c1v = f32x2_to_e4m3x2(__fmul_rn(f1.x, inv), __fmul_rn(f1.y, inv));
+              out = c0v | (c1v << 16);
             }
-            if (b == 0 && p.out_xn)
-              reinterpret_cast<uint4*>(p.out_xn)[(size_t)m * ng + i] = make_uint4(w[0], w[1], w[2], w[3]);
+            *reinterpret_cast<uint32_t*>(bx + sw128_offset(m, 4 * i, nbg)) = out;
+            if (b == 0 && p.out_xq) *reinterpret_cast<uint32_t*>(p.out_xq + (size_t)m * H + 4 * i) = out;
           }
-          float2 xf[4];
-#pragma unroll
-          for (int t = 0; t < 4; ++t) xf[t] = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[t]));
-#pragma unroll
-          for (int el = 0; el < kMaxRowsPerCta; ++el) {
-            if (el < ne) {
-              const float4* wrow = reinterpret_cast<const float4*>(wr_s + (size_t)el * H);
-              const float4 w0 = wrow[2 * i], w1 = wrow[2 * i + 1];
-              float v = acc[el];
-              v = fmaf(xf[0].x, w0.x, v); v = fmaf(xf[0].y, w0.y, v); v = fmaf(xf[1].x, w0.z, v);
-              v = fmaf(xf[1].y, w0.w, v); v = fmaf(xf[2].x, w1.x, v); v = fmaf(xf[2].y, w1.y, v);
-              v = fmaf(xf[3].x, w1.z, v); v = fmaf(xf[3].y, w1.w, v);
-              acc[el] = v;
-            }
-          }
-          uint2 out = make_uint2(0u, 0u);
-          if (a != 0.f) {
-            const uint32_t c0v = f32x2_to_e4m3x2(__fmul_rn(xf[0].x, inv), __fmul_rn(xf[0].y, inv));
-            const uint32_t c1v = f32x2_to_e4m3x2(__fmul_rn(xf[1].x, inv), __fmul_rn(xf[1].y, inv));
-            const uint32_t c2v = f32x2_to_e4m3x2(__fmul_rn(xf[2].x, inv), __fmul_rn(xf[2].y, inv));
-            const uint32_t c3v = f32x2_to_e4m3x2(__fmul_rn(xf[3].x, inv), __fmul_rn(xf[3].y, inv));
-            out = make_uint2(c0v | (c1v << 16), c2v | (c3v << 16));
-          }
-          *reinterpret_cast<uint2*>(bx + sw128_offset(m, 8 * i, nbg)) = out;
-          if (b == 0 && p.out_xq) *reinterpret_cast<uint2*>(p.out_xq + (size_t)m * H + 8 * i) = out;
         }
       }
+      if (m == warp) tc_trace(p, 37);
+      // logits of the CTA's router rows, two at a time
+      for (int el0 = 0; el0 < ne; el0 += 2) {
+        float acc0 = 0.f, acc1 = 0.f;
+        const bool two = el0 + 1 < ne;
+        const float4* w0 = reinterpret_cast<const float4*>(wr_s + (size_t)el0 * H);
+        const float4* w1 = reinterpret_cast<const float4*>(wr_s + (size_t)(el0 + (two ? 1 : 0)) * H);
+        for (int c0 = 0; c0 < n2; c0 += 32 * kTcXU2) {
+          if (!one) {
+            load_chunk(c0);
+            norm_chunk(c0);
+          }
 #pragma unroll
-      for (int el = 0; el < kMaxRowsPerCta; ++el) {
-        if (el < ne) {
-          const float v = warp_sum(acc[el]);
-          if (lane == 0) st_relaxed_u64(tw.logits + (size_t)m * E + e0 + el, tag_word(epoch, v));
+          for (int j = 0; j < kTcXU2; ++j) {
+            const int i = c0 + lane + 32 * j;
+            if (i < n2) {
+              const float2 x01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xr[j].x));
+              const float2 x23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xr[j].y));
+              const float4 u = w0[i], v = w1[i];
+              acc0 = fmaf(x01.x, u.x, acc0); acc0 = fmaf(x01.y, u.y, acc0);
+              acc0 = fmaf(x23.x, u.z, acc0); acc0 = fmaf(x23.y, u.w, acc0);
+              acc1 = fmaf(x01.x, v.x, acc1); acc1 = fmaf(x01.y, v.y, acc1);
+              acc1 = fmaf(x23.x, v.z, acc1); acc1 = fmaf(x23.y, v.w, acc1);
+            }
+          }
         }
+        acc0 = warp_sum(acc0);
+        acc1 = warp_sum(acc1);
+        if (lane == 0) st_relaxed_u64(tw.logits + (size_t)m * E + e0 + el0, tag_word(epoch, acc0));
+        if (lane == 0 && two) st_relaxed_u64(tw.logits + (size_t)m * E + e0 + el0 + 1, tag_word(epoch, acc1));
       }
       if (lane == 0) {
         s_amax[m] = a;
         s_xs[m] = (a == 0.f) ? 1.f : __fdiv_rn(a, 448.f);
         if (b == 0 && p.out_xscale) p.out_xscale[m] = s_xs[m];
       }
+      if (m == warp) tc_trace(p, 38);
     }
     tc_trace(p, 15);
     // the B operand is read by the tensor cores (async proxy)
@@ -807,7 +827,28 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc(Params p, TcWs tw, TcPlan 
       if (p.out_w) p.out_w[tid] = s_w[tid];
     }
   }
-  for (int m = warp; m < M && !(M == 1 && E <= 32 * kTcWarps && K <= 8); m += kTcWarps) {
+  if (M >= 2 && E <= 512 && K <= 8) {
+    // two tokens per warp, one per half
+    for (int m = 2 * warp + (lane >> 4); m < M; m += 2 * kTcWarps) {
+      const float* lrow = s_logit + (size_t)m * E;
+      int* ids = s_ids + m * K;
+      float* ws = s_w + m * K;
+      if (E <= 16) topk_half<1>(lrow, E, K, ids, ws);
+      else if (E <= 32) topk_half<2>(lrow, E, K, ids, ws);
+      else if (E <= 64) topk_half<4>(lrow, E, K, ids, ws);
+      else if (E <= 128) topk_half<8>(lrow, E, K, ids, ws);
+      else if (E <= 256) topk_half<16>(lrow, E, K, ids, ws);
+      else topk_half<32>(lrow, E, K, ids, ws);
+      if (b == 0 && (lane & 15) < K) {
+        if (p.out_ids) p.out_ids[m * K + (lane & 15)] = ids[lane & 15];
+        if (p.out_w) p.out_w[m * K + (lane & 15)] = ws[lane & 15];
+      }
+      if (m == 2 * warp) tc_trace(p, 39);
+    }
+    tc_trace(p, 40);
+  }
+  for (int m = warp; m < M && !(M == 1 && E <= 32 * kTcWarps && K <= 8) && !(M >= 2 && E <= 512 && K <= 8);
+       m += kTcWarps) {
     const float* lrow = s_logit + (size_t)m * E;
     int* ids = s_ids + m * K;
     float* ws = s_w + m * K;
@@ -830,28 +871,43 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc(Params p, TcWs tw, TcPlan 
   const int np = M * K, pbase = kShared ? M : 0;
   if (M == 1) {
     union_m1(s_ids, K, ub, pbase, s_union, s_poff, s_pm, s_ppos, &s_int[0]);
-  } else if (warp == 0 && np <= 32) {
-    const int Us = union_small(s_ids, np, K, s_union + ub, s_poff + ub, s_pm, s_ppos, pbase);
-    if (lane == 0) s_int[0] = ub + Us;
-  } else if (warp == 0) {
-    for (int e = lane; e < E; e += 32) s_ec[e] = 0;
-    __syncwarp();
-    for (int i = lane; i < np; i += 32) atomicAdd(&s_ec[s_ids[i]], 1);
-    __syncwarp();
-    const int per = (E + 31) / 32;
-    const int ea = min(E, lane * per), eb = min(E, ea + per);
+  } else if (np <= 32) {
+    if (warp == 0) {
+      const int Us = union_small(s_ids, np, K, s_union + ub, s_poff + ub, s_pm, s_ppos, pbase);
+      if (lane == 0) s_int[0] = ub + Us;
+    }
+  } else {
+    // many pairs: the whole CTA. Counts per expert, a block-wide exclusive
+    // scan over the experts (ascending: the union and each entry's first
+    // pair position), then each pair's place among the earlier pairs of its
+    // expert (token, slot order)
+    int* s_ws = reinterpret_cast<int*>(s_red);  // [kTcWarps][2] warp totals
+    for (int e = tid; e < E; e += kTcThreads) s_ec[e] = 0;
+    __syncthreads();
+    tc_trace(p, 41);
+    for (int i = tid; i < np; i += kTcThreads) atomicAdd(&s_ec[s_ids[i]], 1);
+    __syncthreads();
+    const int per = (E + kTcThreads - 1) / kTcThreads;
+    const int ea = min(E, tid * per), eb = min(E, ea + per);
     int nz = 0, cs = 0;
     for (int e = ea; e < eb; ++e) { nz += s_ec[e] > 0; cs += s_ec[e]; }
-    int nz_ex = nz, cs_ex = cs;
+    int nz_in = nz, cs_in = cs;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const int x1 = __shfl_up_sync(0xffffffffu, nz_ex, o);
-      const int x2 = __shfl_up_sync(0xffffffffu, cs_ex, o);
-      if (lane >= o) { nz_ex += x1; cs_ex += x2; }
+      const int x1 = __shfl_up_sync(0xffffffffu, nz_in, o);
+      const int x2 = __shfl_up_sync(0xffffffffu, cs_in, o);
+      if (lane >= o) { nz_in += x1; cs_in += x2; }
     }
-    nz_ex -= nz;
-    cs_ex -= cs;
-    __syncwarp();
+    if (lane == 31) {
+      s_ws[2 * warp] = nz_in;
+      s_ws[2 * warp + 1] = cs_in;
+    }
+    __syncthreads();
+    int nz_ex = nz_in - nz, cs_ex = cs_in - cs;
+    for (int w = 0; w < warp; ++w) {
+      nz_ex += s_ws[2 * w];
+      cs_ex += s_ws[2 * w + 1];
+    }
     for (int e = ea; e < eb; ++e) {
       const int c = s_ec[e];
       if (c > 0) {
@@ -860,26 +916,28 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc(Params p, TcWs tw, TcPlan 
         ++nz_ex;
         cs_ex += c;
       }
-      s_ec[e] = pbase + cs_ex - c;
+      s_ec[e] = pbase + cs_ex - c;  // first pair position of expert e
     }
-    if (lane == 31) {
+    if (tid == kTcThreads - 1) {
       s_poff[ub + nz_ex] = pbase + cs_ex;
       s_int[0] = ub + nz_ex;
     }
-    __syncwarp();
-    for (int base = 0; base < np; base += 32) {
-      const int i = base + lane;
-      const int e = (i < np) ? s_ids[i] : -1 - lane;
-      const unsigned same = __match_any_sync(0xffffffffu, e);
-      const int rank = __popc(same & ((1u << lane) - 1u));
-      if (i < np) {
-        const int pos = s_ec[e] + rank;
-        s_pm[pos] = i / K;
-        s_ppos[i] = pos;
+    __syncthreads();
+    tc_trace(p, 34);
+    for (int i = tid; i < np; i += kTcThreads) {
+      const int e = s_ids[i];
+      // earlier pairs of the same expert: whole int4 blocks (16-byte aligned
+      // s_ids), then the rest
+      int rank = 0, j2 = 0;
+      const int4* ids4 = reinterpret_cast<const int4*>(s_ids);
+      for (; j2 + 4 <= i; j2 += 4) {
+        const int4 v = ids4[j2 >> 2];
+        rank += (v.x == e) + (v.y == e) + (v.z == e) + (v.w == e);
       }
-      __syncwarp();
-      if (i < np && rank == 0) s_ec[e] += __popc(same);
-      __syncwarp();
+      for (; j2 < i; ++j2) rank += s_ids[j2] == e;
+      const int pos = s_ec[e] + rank;
+      s_pm[pos] = i / K;
+      s_ppos[i] = pos;
     }
   }
   // ring_gu and ring_d held routing scratch (generic proxy): order that
@@ -977,7 +1035,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc(Params p, TcWs tw, TcPlan 
           if (reuse && !mbar_wait_ok(empty_gu + slot, ph ^ 1u, p)) { ok = false; break; }
           if (stage >= pl.ns_gu && stage < pl.ns_gu + 4) tc_trace(p, 42 + stage - pl.ns_gu);
           mbar_expect_tx(full_gu + slot, bytes);
-          if (stage < 10) tc_trace(p, 32 + stage);
+          if (stage < 2) tc_trace(p, 32 + stage);
           uint8_t* dst = ring_gu + (size_t)slot * pl.slot_gu;
           for (int r = 0; r < nrun; ++r) {
             if (tw.repacked)
