@@ -218,6 +218,7 @@ def run_ours(args):
     flags = {"split": moe.MOE_FLAG_SPLIT_KERNELS, "cuda": moe.MOE_FLAG_CUDA_CORES,
              "tc": moe.MOE_FLAG_TENSOR_CORES}.get(args.variant, 0)
     flags |= moe.MOE_FLAG_FP8_INTERMEDIATE if args.fp8_intermediate else 0
+    flags |= moe.MOE_FLAG_SPLITK_DOWN if args.splitk_down else 0
     x, ctxs, _weights = build_pool(device, M, args.routing, layers=L, flags=flags, stack=args.stack,
                                    shared=args.shared_expert, repack=args.repack)
     n_shared = int(args.shared_expert)
@@ -715,6 +716,8 @@ def main():
                     help="load the layers with MOE_LOAD_COPY_REPACK (context-owned, kernel-private weight layout)")
     ap.add_argument("--shared-expert", action="store_true",
                     help="one always-active shared expert per layer besides the top-8 routed ones")
+    ap.add_argument("--splitk-down", action="store_true",
+                    help="down projection split over K with CTA-local h (max 4 tokens)")
     ap.add_argument("--fp8-intermediate", action="store_true",
                     help="quantise the SwiGLU output to E4M3 per (token, expert) before the down projection")
     ap.add_argument("--stack", action="store_true",

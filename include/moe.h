@@ -88,6 +88,13 @@ typedef enum {
                                        Persistent kernel only: with
                                        MOE_FLAG_SPLIT_KERNELS, moe_create
                                        returns MOE_ERR_UNSUPPORTED */
+#define MOE_FLAG_SPLITK_DOWN 0x100u  /* down projection split over K (each CTA
+                                       multiplies its own h slice by a K-major
+                                       copy of W2 that moe_load_experts makes;
+                                       partial outputs summed in a fixed
+                                       order). max_tokens <= 4; not with
+                                       MOE_FLAG_FP8_INTERMEDIATE or
+                                       MOE_FLAG_SPLIT_KERNELS */
 #define MOE_FLAG_FP8_INTERMEDIATE 0x8u /* FP8 input to the down projection too
                                        (W4A8 on the same page, section "Why
                                        is MoE decoding on DGX Spark

@@ -35,14 +35,19 @@ moe_status validate_config(const moe_config& c) {
   if (c.num_experts < 1 || c.num_experts > moe::kMaxExperts) return MOE_ERR_INVALID_ARG;
   if (c.top_k < 1 || c.top_k > c.num_experts || c.top_k > moe::kMaxTopK) return MOE_ERR_INVALID_ARG;
   if (c.max_tokens < 1 || c.max_tokens > moe::kMaxTokens) return MOE_ERR_INVALID_ARG;
-  const uint32_t fused_only = MOE_FLAG_PRE_RMSNORM | MOE_FLAG_SHARED_EXPERT | MOE_FLAG_FP8_INTERMEDIATE;
+  const uint32_t fused_only =
+      MOE_FLAG_PRE_RMSNORM | MOE_FLAG_SHARED_EXPERT | MOE_FLAG_FP8_INTERMEDIATE | MOE_FLAG_SPLITK_DOWN;
   if (c.flags & ~(MOE_FLAG_SPLIT_KERNELS | MOE_FLAG_CUDA_CORES | MOE_FLAG_TENSOR_CORES | MOE_FLAG_TC_DOWN_MMA |
                   MOE_FLAG_TC_DOWN_CUDA | fused_only))
     return MOE_ERR_INVALID_ARG;
   if ((c.flags & MOE_FLAG_TC_DOWN_MMA) && (c.flags & MOE_FLAG_TC_DOWN_CUDA)) return MOE_ERR_INVALID_ARG;
   if ((c.flags & MOE_FLAG_CUDA_CORES) && (c.flags & MOE_FLAG_TENSOR_CORES)) return MOE_ERR_INVALID_ARG;
-  if ((c.flags & MOE_FLAG_TENSOR_CORES) && (c.flags & MOE_FLAG_SPLIT_KERNELS)) return MOE_ERR_INVALID_ARG;
+  if ((c.flags & MOE_FLAG_TENSOR_CORES) && (c.flags & (MOE_FLAG_SPLIT_KERNELS | MOE_FLAG_SPLITK_DOWN)))
+    return MOE_ERR_INVALID_ARG;
   if ((c.flags & fused_only) && (c.flags & MOE_FLAG_SPLIT_KERNELS)) return MOE_ERR_UNSUPPORTED;
+  if ((c.flags & MOE_FLAG_SPLITK_DOWN) &&
+      ((c.flags & MOE_FLAG_FP8_INTERMEDIATE) || c.max_tokens > moe::kSkMaxTokens))
+    return MOE_ERR_UNSUPPORTED;
   return MOE_OK;
 }
 
@@ -62,6 +67,7 @@ bool make_plan(const moe_config& c, int sm_count, size_t smem_limit, moe::FusedP
   size_t NP, UMAX;
   union_bounds(c, &NP, &UMAX);
   const bool shared = (c.flags & MOE_FLAG_SHARED_EXPERT) != 0;
+  const bool splitk = (c.flags & MOE_FLAG_SPLITK_DOWN) != 0;
   const size_t n_cnt = shared ? E + 1 : E;
   const size_t nr_max = (I + G - 1) / G, nrd_max = (H + G - 1) / G;
   *pl = moe::FusedPlan{};
@@ -72,13 +78,16 @@ bool make_plan(const moe_config& c, int sm_count, size_t smem_limit, moe::FusedP
   pl->rpc_max = (int)nrd_max;
   pl->slot_gu = (int)align_up(nr_max * H + 2 * (nr_max * H / 32 + 32), 128);
   pl->slot_d = (int)align_up(nrd_max * (I / 2) + nrd_max * (I / 32) + 32, 128);
+  pl->nr_max = (int)nr_max;
+  pl->dchunks = (int)((H + moe::kSkChunk - 1) / moe::kSkChunk);
+  if (splitk) pl->slot_d = (int)align_up(nr_max * (H / 2) + 2 * H, 128);  // K rows + <= 2 scale rows
   // MMA partials of entries with several pairs: per gate/up slot, one float4
   // per lane for each (K chunk = item, 8-row group, 8-pair tile)
   const size_t gu_items_max = (nr_max + moe::kGuRowsPerItem - 1) / moe::kGuRowsPerItem;
   pl->part_ct = (int)std::min<size_t>(moe::kMaxPairTiles, (MM + 7) / 8);
   pl->part_slot = (MM >= (size_t)moe::kMmaMinPairs) ? (int)(gu_items_max * ((nr_max + 7) / 8) * pl->part_ct * 32 * 16) : 0;
   pl->hpairs = (int)std::min<size_t>(moe::kHPairs, MM);
-  pl->hslot = (int)align_up((size_t)pl->hpairs * I * 2 + moe::kHPairs * 4, 16);
+  pl->hslot = splitk ? 0 : (int)align_up((size_t)pl->hpairs * I * 2 + moe::kHPairs * 4, 16);
   const size_t kMaxSlots = moe::kMaxSlots;
   size_t off = 0;
   auto take = [&](size_t bytes, size_t a) { off = align_up(off, a); size_t o = off; off += bytes; return o; };
@@ -92,7 +101,13 @@ bool make_plan(const moe_config& c, int sm_count, size_t smem_limit, moe::FusedP
   pl->o_poff = (int)take((UMAX + 1) * 4, 16);
   pl->o_cnt = (int)take(n_cnt * 4, 16);
   pl->o_act = (int)take(MM * H, 16);
-  pl->o_dsm = (int)take(NP * nrd_max * 4, 16);
+  pl->o_dsm = (int)take(splitk ? 0 : NP * nrd_max * 4, 16);
+  if (splitk) {
+    pl->o_hsm = (int)take(UMAX * MM * nr_max * 4, 16);
+    pl->o_ycta = (int)take(std::max<size_t>(MM * H, moe::kConsumers * 32) * 4, 16);
+    pl->o_chunk = (int)take((pl->dchunks + UMAX) * 4, 16);
+    pl->o_pw = (int)take(NP * 4, 16);
+  }
   off = align_up(off, 128);
   if (off >= smem_limit) return false;
   // each down slot carries its staged h
@@ -331,6 +346,25 @@ bool encode_w2_map(const void* w2c, size_t Eall, size_t H, size_t I, CUtensorMap
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// K-major copy of W2 for the split-K down projection:
+//   kc[e][n][j] = code of W2[e][2j][n] | code of W2[e][2j+1][n] << 4
+//   ks[e][nb][r] = scale byte of W2[e][r][32nb .. 32nb+31]
+__global__ void k_repack_w2(const uint8_t* w2c, const uint8_t* w2s, int E, int H, int I, uint8_t* kc, uint8_t* ks) {
+  const size_t step = (size_t)gridDim.x * blockDim.x;
+  const size_t nc = (size_t)E * I * (H / 2);
+  for (size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x; idx < nc; idx += step) {
+    const size_t j = idx % (H / 2), n = (idx / (H / 2)) % I, e = idx / ((size_t)(H / 2) * I);
+    const uint8_t b0 = w2c[(e * H + 2 * j) * (I / 2) + n / 2], b1 = w2c[(e * H + 2 * j + 1) * (I / 2) + n / 2];
+    const uint8_t v0 = (n & 1) ? (b0 >> 4) : (b0 & 0xF), v1 = (n & 1) ? (b1 >> 4) : (b1 & 0xF);
+    kc[idx] = (uint8_t)(v0 | (v1 << 4));
+  }
+  const size_t ns = (size_t)E * (I / 32) * H;
+  for (size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x; idx < ns; idx += step) {
+    const size_t r = idx % H, nb = (idx / H) % (I / 32), e = idx / ((size_t)H * (I / 32));
+    ks[idx] = w2s[(e * H + r) * (I / 32) + nb];
+  }
+}
+
 }  // namespace
 
 struct moe_ctx {
@@ -354,6 +388,8 @@ struct moe_ctx {
   int force_stall = 0;
   unsigned long long* trace = nullptr;
   void (*fused)(moe::Params, moe::FusedWs, moe::FusedPlan) = nullptr;  // k_fused instantiation
+  uint8_t* w2k = nullptr;  // split-K: context-owned K-major W2 (codes, then scales)
+  size_t w2k_codes = 0, w2k_bytes = 0;
   moe::FusedPlan plan{};
   moe::FusedWs fws{};
   void (*tc)(moe::Params, moe::TcWs, moe::TcPlan, const moe::TcMaps) = nullptr;  // k_tc instantiation
@@ -402,16 +438,21 @@ moe_status moe_create(const moe_config* cfg, moe_ctx** out) {
   ctx->spin_limit = kDefaultSpinLimit;
   {
     const bool sh = (c.flags & MOE_FLAG_SHARED_EXPERT) != 0, f8 = (c.flags & MOE_FLAG_FP8_INTERMEDIATE) != 0;
-    ctx->fused = sh ? (f8 ? moe::k_fused<true, true> : moe::k_fused<true, false>)
-                    : (f8 ? moe::k_fused<false, true> : moe::k_fused<false, false>);
+    const bool sk = (c.flags & MOE_FLAG_SPLITK_DOWN) != 0;
+    if (sk)
+      ctx->fused = sh ? moe::k_fused<true, false, true> : moe::k_fused<false, false, true>;
+    else
+      ctx->fused = sh ? (f8 ? moe::k_fused<true, true, false> : moe::k_fused<true, false, false>)
+                      : (f8 ? moe::k_fused<false, true, false> : moe::k_fused<false, false, false>);
     ctx->tc = sh ? (f8 ? moe::k_tc<true, true> : moe::k_tc<true, false>)
                  : (f8 ? moe::k_tc<false, true> : moe::k_tc<false, false>);
   }
   // the tensor-core kernel when asked for, or by default from
-  // MOE_TC_MIN_TOKENS tokens on, wherever its shape rules hold
+  // MOE_TC_MIN_TOKENS tokens on, wherever its shape rules hold (the split-K
+  // down projection is a CUDA-core kernel option)
   {
     const bool want_tc = (c.flags & MOE_FLAG_TENSOR_CORES) ||
-                         (!(c.flags & MOE_FLAG_CUDA_CORES) && c.max_tokens >= MOE_TC_MIN_TOKENS);
+                         (!(c.flags & (MOE_FLAG_CUDA_CORES | MOE_FLAG_SPLITK_DOWN)) && c.max_tokens >= MOE_TC_MIN_TOKENS);
     const bool tc_ok = make_tc_plan(c, prop.multiProcessorCount, (size_t)prop.sharedMemPerBlockOptin, &ctx->tplan) &&
                        encode_tiled() != nullptr;
     if ((c.flags & MOE_FLAG_TENSOR_CORES) && !tc_ok) {
@@ -448,6 +489,9 @@ moe_status moe_create(const moe_config* cfg, moe_ctx** out) {
   const size_t o_tcnt = take(2 * UMAXF * moe::kTcCntStride * sizeof(unsigned));
   const size_t o_typ = take(NPF * H * sizeof(float));
   const size_t o_tdc = take(2 * moe::kTcCntStride * sizeof(unsigned));
+  const bool splitk = (c.flags & MOE_FLAG_SPLITK_DOWN) != 0;
+  const size_t o_ypart = take(splitk ? (size_t)ctx->sm_count * MM * H * sizeof(float) : 0);
+  const size_t o_fcnt = take(sizeof(unsigned long long));
   ctx->ws_bytes = off;
   if (cudaMalloc(&ctx->ws_base, ctx->ws_bytes) != cudaSuccess) {
     cudaGetLastError();
@@ -483,6 +527,8 @@ moe_status moe_create(const moe_config* cfg, moe_ctx** out) {
   ctx->tws.ypart = reinterpret_cast<float*>(b + o_typ);
   ctx->tws.dcnt = reinterpret_cast<unsigned*>(b + o_tdc);
   ctx->tws.epoch = w.ctrl + 6;
+  ctx->fws.ypart = reinterpret_cast<float*>(b + o_ypart);
+  ctx->fws.fin_cnt = reinterpret_cast<unsigned long long*>(b + o_fcnt);
 
   // launch shapes
   ctx->grid_route = (int)(E < (size_t)ctx->sm_count ? E : (size_t)ctx->sm_count);
@@ -531,6 +577,7 @@ void moe_destroy(moe_ctx* ctx) {
   DeviceGuard guard(ctx->dev);
   if (ctx->ws_base) cudaFree(ctx->ws_base);
   if (ctx->owned) cudaFree(ctx->owned);
+  if (ctx->w2k) cudaFree(ctx->w2k);
   delete ctx;
 }
 
@@ -615,6 +662,26 @@ moe_status moe_load_experts(moe_ctx* ctx, const float* router_w, const uint8_t* 
     if (ctx->tplan.mma_down && (!encode_w2_map(w2_codes, Eall, H, I, &ctx->maps.w2) || !aligned16(w2_scales)))
       return MOE_ERR_INVALID_ARG;
   }
+  if (c.flags & MOE_FLAG_SPLITK_DOWN) {
+    // the K-major W2 copy the split-K down projection streams
+    const size_t E = c.num_experts + ((c.flags & MOE_FLAG_SHARED_EXPERT) ? 1 : 0), H = c.hidden, I = c.inter;
+    const size_t nc = E * I * (H / 2), ns = E * (I / 32) * H;
+    if (!ctx->w2k) {
+      if (cudaMalloc(&ctx->w2k, nc + ns) != cudaSuccess) {
+        cudaGetLastError();
+        ctx->w2k = nullptr;
+        ctx->loaded = false;
+        return MOE_ERR_OOM;
+      }
+      ctx->w2k_codes = nc;
+      ctx->w2k_bytes = nc + ns;
+    }
+    k_repack_w2<<<ctx->sm_count * 8, 256>>>(w2_codes, w2_scales, (int)E, (int)H, (int)I, ctx->w2k, ctx->w2k + nc);
+    if (cudaGetLastError() != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
+      ctx->loaded = false;
+      return MOE_ERR_CUDA;
+    }
+  }
   ctx->wr = router_w;
   ctx->w13c = w13_codes;
   ctx->w13s = w13_scales;
@@ -656,6 +723,8 @@ moe_status moe_decode(moe_ctx* ctx, const void* x_bf16, int32_t M, void* y_bf16,
   p.w13s = ctx->w13s;
   p.w2c = ctx->w2c;
   p.w2s = ctx->w2s;
+  p.w2kc = ctx->w2k;
+  p.w2ks = ctx->w2k ? ctx->w2k + ctx->w2k_codes : nullptr;
   p.ws = ctx->ws;
   p.out_ids = topk_ids;
   p.out_w = topk_w;

@@ -50,6 +50,8 @@ struct Params {
   const uint8_t* w13s;
   const uint8_t* w2c;
   const uint8_t* w2s;
+  const uint8_t* w2kc;  // split-K down: W2 codes K-major [E][I][H/2] (low nibble = even output row)
+  const uint8_t* w2ks;  // split-K down: W2 scales [E][I/32][H]
   Workspace ws;
   int* out_ids;
   float* out_w;

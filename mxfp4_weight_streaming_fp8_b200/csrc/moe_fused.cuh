@@ -61,6 +61,9 @@ constexpr int kMaxSlots = 64;
 constexpr int kMaxPairTiles = 4;            // 8-pair MMA column tiles per entry (32 pairs)
 constexpr int kMmaMinPairs = 3;             // entries with at least this many pairs take the MMA gate/up path
 constexpr int kCounterStride = 16;          // u64 words between per-entry counters (one 128-byte line)
+constexpr int kSkMaxTokens = 4;             // split-K down: tokens per call (partial y of a CTA in smem)
+constexpr int kSkRowsPerLane = 8;           // split-K down: output rows per lane of a chunk (one code word)
+constexpr int kSkChunk = 32 * kSkRowsPerLane;  // output rows per down chunk
 
 // Launch-invariant plan computed on the host at moe_create.
 struct FusedPlan {
@@ -78,6 +81,9 @@ struct FusedPlan {
   int smem_bytes;
   int wr_bytes_max;     // router rows staged per CTA (alias ring_gu)
   int x_staged;         // bf16 x fits in ring_d and is staged there during routing
+  // split-K down (kSplitK): CTA-local h [max_union][max_tokens][nr_max],
+  // partial y [max_tokens][H], per-chunk entry progress, pair weights
+  int nr_max, dchunks, o_hsm, o_ycta, o_chunk, o_pw;
 };
 
 // Workspace pieces only the persistent kernel uses.
@@ -85,6 +91,8 @@ struct FusedWs {
   unsigned long long* logits;     // [maxM][E] tagged router logits (epoch, fp32)
   unsigned long long* gu_cnt;     // [max_union][kCounterStride] gate/up arrivals per entry; += G per launch
   unsigned* epoch;                // launch counter
+  float* ypart;                   // split-K: [G][max_tokens][H] partial y of every CTA
+  unsigned long long* fin_cnt;    // split-K: partial-y arrivals; += G per launch
 };
 
 // Counter of union entry u, alone on its L2 line.
@@ -197,6 +205,30 @@ __device__ __forceinline__ unsigned atom_add_acqrel_cta_smem(unsigned* p, unsign
   return old;
 }
 
+// CTA-scope release/acquire on a shared-memory word (a ready flag).
+__device__ __forceinline__ void st_release_cta_smem(unsigned* p, unsigned v) {
+  asm volatile("st.release.cta.shared::cta.u32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
+}
+__device__ __forceinline__ unsigned ld_acquire_cta_smem(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
+  return v;
+}
+// Wait (one thread) until a shared-memory word written with a CTA-scope
+// release reaches `target`; acquire, so the writer's earlier stores are
+// visible after it returns.
+__device__ __forceinline__ void smem_acquire_wait(const unsigned* c, unsigned target, const Params& p) {
+  if (ld_acquire_cta_smem(c) >= target) return;
+  const long long t0 = clock64();
+  while (ld_acquire_cta_smem(c) < target) {
+    __nanosleep(32);
+    if (clock64() - t0 > p.spin_limit) {
+      atomicOr(p.ws.ctrl, kStatusTimeout);
+      return;
+    }
+  }
+}
+
 __device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* p) {
   unsigned long long v;
   asm volatile("ld.acquire.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
@@ -228,15 +260,6 @@ __device__ __forceinline__ void grid_wait(const unsigned long long* cnt, unsigne
   }
 }
 
-// CTA-scope release/acquire on a shared-memory word (a ready flag).
-__device__ __forceinline__ unsigned ld_acquire_cta_smem(const unsigned* p) {
-  unsigned v;
-  asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
-  return v;
-}
-__device__ __forceinline__ void st_release_cta_smem(unsigned* p, unsigned v) {
-  asm volatile("st.release.cta.shared::cta.u32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
-}
 // Whole warp: wait (lane 0 polls, bounded) until a shared-memory flag is set;
 // false, with the status bit set, when the wait ran out.
 __device__ __forceinline__ bool wait_flag_warp(const Params& p, const unsigned* flag) {
@@ -335,8 +358,8 @@ __device__ __forceinline__ unsigned d_layout(const Params& p, int e, int r0, int
 // expert. Lane owns half-blocks hb = lane + 32j (16 elements, 8 code bytes).
 // Products E2M1 x E4M3 are exact in f16; each f16x2 half sums 8 of them
 // (|sum| <= 8*6*448 = 21504) before the fp32 block-scale FMA.
-__device__ __forceinline__ void gu_item(const Params& p, const GuChunk& ch, int a, int cnt, int n0,
-                                        int pb, int pe, const int* s_pm, const uint8_t* act,
+__device__ __forceinline__ void gu_item(const Params& p, const GuChunk& ch, int a, int cnt, float* hout,
+                                        size_t hstride, int pb, int pe, const int* s_pm, const uint8_t* act,
                                         const float* s_xs) {
   const int lane = threadIdx.x & 31;
   const int H = p.H, nhb = H / 16;
@@ -398,7 +421,7 @@ __device__ __forceinline__ void gu_item(const Params& p, const GuChunk& ch, int 
 #pragma unroll
     for (int r = 0; r < kGuRowsPerItem; ++r) {
       const float g = ag[r] * s, u = au[r] * s;
-      if (lane == 0 && r < cnt) p.ws.h[(size_t)pp * p.I + n0 + a + r] = g / (1.f + expf(-g)) * u;
+      if (lane == 0 && r < cnt) hout[(size_t)(pp - pb) * hstride + a + r] = g / (1.f + expf(-g)) * u;
     }
   }
 }
@@ -684,6 +707,64 @@ __device__ __forceinline__ void d_item(const Params& p, const DChunk& ch, int a,
       }
       d_rows(p, ch, a, cnt, blk, h2, down, dsm + (size_t)pp * rpc, b0 == 0);
       __syncwarp();
+    }
+  }
+}
+
+// Split-K down chunk: output rows [c*kSkChunk, (c+1)*kSkChunk) of one entry
+// over this CTA's K slice [n0, n0+nr): lane owns rows r..r+7 (one code word
+// per K row). slot: codes [nr][H/2] (K-major, byte j = rows 2j, 2j+1), then
+// scale rows [nskb][H] of the 32-blocks from skb0. hu[q * hstride + j] is
+// h of pair pb + q at K row n0 + j. Adds w * partial into the CTA's
+// partial y of each pair's token.
+__device__ __forceinline__ void sk_down_chunk(const Params& p, const uint8_t* slot, int n0, int nr, int skb0, int c,
+                                              int pb, int pe, const float* hu, int hstride, const int* s_pm,
+                                              const float* s_pw, float* ycta) {
+  const int lane = threadIdx.x & 31, H = p.H;
+  const int r = c * kSkChunk + lane * kSkRowsPerLane;
+  if (r >= H) return;  // H % 8 == 0: a lane's rows are all in range or all out
+  const uint8_t* codes = slot;
+  const uint8_t* scl = slot + (size_t)nr * (H / 2);
+  const int np = pe - pb;
+  float acc[kSkMaxTokens][kSkRowsPerLane];
+#pragma unroll
+  for (int q = 0; q < kSkMaxTokens; ++q)
+#pragma unroll
+    for (int i = 0; i < kSkRowsPerLane; ++i) acc[q][i] = 0.f;
+  for (int j = 0; j < nr; ++j) {
+    const uint32_t cw = *reinterpret_cast<const uint32_t*>(codes + (size_t)j * (H / 2) + r / 2);
+    const uint2 sw = *reinterpret_cast<const uint2*>(scl + (size_t)((n0 + j) / 32 - skb0) * H + r);
+    uint32_t f[4];
+    e2m1x8_to_f16x2x4(cw, f);
+    const uint32_t sb[2] = {sw.x, sw.y};
+    float wv[kSkRowsPerLane];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const float2 v = __half22float2(*reinterpret_cast<const __half2*>(&f[t]));
+      wv[2 * t] = v.x * e8m0_to_f32((sb[t >> 1] >> (16 * (t & 1))) & 0xFFu);
+      wv[2 * t + 1] = v.y * e8m0_to_f32((sb[t >> 1] >> (16 * (t & 1) + 8)) & 0xFFu);
+    }
+#pragma unroll
+    for (int q = 0; q < kSkMaxTokens; ++q) {
+      if (q < np) {
+        const float hv = hu[(size_t)q * hstride + j];
+#pragma unroll
+        for (int i = 0; i < kSkRowsPerLane; ++i) acc[q][i] = fmaf(wv[i], hv, acc[q][i]);
+      }
+    }
+  }
+#pragma unroll
+  for (int q = 0; q < kSkMaxTokens; ++q) {
+    if (q < np) {
+      const float w = s_pw[pb + q];
+      float4* yr = reinterpret_cast<float4*>(ycta + (size_t)s_pm[pb + q] * H + r);
+      float4 y0 = yr[0], y1 = yr[1];
+      y0.x = fmaf(w, acc[q][0], y0.x); y0.y = fmaf(w, acc[q][1], y0.y);
+      y0.z = fmaf(w, acc[q][2], y0.z); y0.w = fmaf(w, acc[q][3], y0.w);
+      y1.x = fmaf(w, acc[q][4], y1.x); y1.y = fmaf(w, acc[q][5], y1.y);
+      y1.z = fmaf(w, acc[q][6], y1.z); y1.w = fmaf(w, acc[q][7], y1.w);
+      yr[0] = y0;
+      yr[1] = y1;
     }
   }
 }
@@ -1022,8 +1103,12 @@ __device__ __forceinline__ int union_small(const int* s_ids, int np, int K, int*
 // logits arrive measured slower: the wait for the router is shorter than an
 // item, so they lengthened routing.)
 // kFp8H: the FP8 intermediate (see h_fp8x2) for every expert.
-template <bool kShared, bool kFp8H>
+// kSplitK: the down projection is split over K instead of output rows (see
+// the split-K block below); needs max_tokens <= kSkMaxTokens and the
+// K-major W2 copy (w2kc, w2ks).
+template <bool kShared, bool kFp8H, bool kSplitK>
 __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw, FusedPlan pl) {
+  static_assert(!(kSplitK && kFp8H), "the FP8 intermediate needs the whole h of a pair");
   extern __shared__ __align__(128) unsigned char smem[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int b = blockIdx.x, G = gridDim.x;
@@ -1055,6 +1140,12 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
   float* dsm = reinterpret_cast<float*>(smem + pl.o_dsm);
   uint8_t* hstage = smem + pl.o_h;
   uint8_t* ring_gu = smem + pl.o_ring_gu;
+  // split-K down: CTA-local h, partial y, chunk progress, per-entry h ready
+  float* hsm = reinterpret_cast<float*>(smem + pl.o_hsm);     // [max_union][max_tokens][nr_max]
+  float* ycta = reinterpret_cast<float*>(smem + pl.o_ycta);   // [max_tokens][H]
+  unsigned* s_chunk = reinterpret_cast<unsigned*>(smem + pl.o_chunk);  // [dchunks] entries done
+  unsigned* s_hrdy = s_chunk + pl.dchunks;                              // [max_union] h of the entry complete
+  float* s_pw = reinterpret_cast<float*>(smem + pl.o_pw);    // [pairs] routing weight per pair position
   uint8_t* ring_d = smem + pl.o_ring_d;
   float* wr_s = reinterpret_cast<float*>(ring_gu + (kShared ? pl.slot_gu : 0));  // router rows (routing phase only)
   float* s_logit = wr_s;                                                          // gathered logits (after them)
@@ -1066,7 +1157,12 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
   const int n0 = (int)((long long)I * b / G), nr = (int)((long long)I * (b + 1) / G) - n0;
   const int r0 = (int)((long long)H * b / G), nrd = (int)((long long)H * (b + 1) / G) - r0;
   const int gu_items = (nr > 0) ? (nr + kGuRowsPerItem - 1) / kGuRowsPerItem : 0;  // per expert
-  const int d_items = (nrd > 0) ? (nrd + kDownRowsPerItem - 1) / kDownRowsPerItem : 0;
+  // down items per entry: output-row items, or (split-K) output chunks of the
+  // CTA's K slice
+  const int d_items = kSplitK ? ((nr > 0) ? pl.dchunks : 0)
+                              : ((nrd > 0) ? (nrd + kDownRowsPerItem - 1) / kDownRowsPerItem : 0);
+  // split-K: scale-block rows of W2 the CTA's K slice touches
+  const int skb0 = n0 / 32, nskb = (nr > 0) ? (n0 + nr - 1) / 32 - skb0 + 1 : 0;
 
   // ---------------- weight stream. Each bulk copy costs its issuing thread
   //   about a hundred nanoseconds, so the first use of every ring slot is
@@ -1093,6 +1189,15 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
     const int e = s_union[u];
     const int slot = u % pl.ns_d;
     uint8_t* sp = ring_d + (size_t)slot * pl.slot_d;
+    if constexpr (kSplitK) {
+      // codes of W2 columns [n0, n0+nr) for every output row (K-major rows
+      // n, each H/2 bytes), then the scale rows of their 32-blocks
+      const unsigned codes = (unsigned)(nr * H / 2), sb = (unsigned)(nskb * H);
+      mbar_expect_tx(full_d + slot, codes + sb);
+      tma_load_1d(sp, p.w2kc + ((size_t)e * I + n0) * (H / 2), codes, full_d + slot);
+      tma_load_1d(sp + codes, p.w2ks + ((size_t)e * (I / 32) + skb0) * H, sb, full_d + slot);
+      return;
+    }
     DChunk ch;
     size_t sa0;
     unsigned sn;
@@ -1116,6 +1221,10 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
     unsigned gn, un;
     gu_layout(p, s_union[u], n0, nr, ring_gu + (size_t)slot * pl.slot_gu, &ch, &ga0, &gn, &ua0, &un);
     const int pb = s_poff[u], pe = s_poff[u + 1];
+    // h of pair pb + q, local row j: hout[q * hstride + j] (global h, or the
+    // CTA-local copy for the split-K down)
+    float* hout = kSplitK ? hsm + (size_t)u * pl.max_tokens * pl.nr_max : p.ws.h + (size_t)pb * I + n0;
+    const size_t hstride = kSplitK ? (size_t)pl.nr_max : (size_t)I;
     if (pe - pb >= kMmaMinPairs && pl.part_slot > 0) {
       // several pairs: the entry's items split K; each runs warp MMAs over
       // all rows and pairs, and the last one to finish sums the partials
@@ -1153,15 +1262,18 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
               if (q < pe - pb && row < nr) {
                 const float sx = s_xs[s_pm[pb + q]];
                 const float gv = gg[i] * sx, uv = uu[i] * sx;
-                p.ws.h[(size_t)(pb + q) * I + n0 + row] = gv / (1.f + expf(-gv)) * uv;
+                hout[(size_t)q * hstride + row] = gv / (1.f + expf(-gv)) * uv;
               }
             }
           }
         }
         __syncwarp();
         // orders the warp's h stores (through the warp barrier) before the
-        // GPU-wide arrival for the entry
-        if (lane == 0) grid_arrive(gu_counter(fw, u));
+        // GPU-wide arrival for the entry (split-K: the CTA-local ready flag)
+        if (lane == 0) {
+          if constexpr (kSplitK) st_release_cta_smem(s_hrdy + u, 1u);
+          else grid_arrive(gu_counter(fw, u));
+        }
       }
       __syncwarp();
       if (lane == 0) {
@@ -1172,7 +1284,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
       return;
     }
     const int a = g * kGuRowsPerItem, cnt = min(kGuRowsPerItem, nr - a);
-    gu_item(p, ch, a, cnt, n0, pb, pe, s_pm, act, s_xs);
+    gu_item(p, ch, a, cnt, hout, hstride, pb, pe, s_pm, act, s_xs);
     if (u == 0 && g == 0) trace_stamp(p, 17);
     if (u == s_int[0] - 1 && g == gu_items - 1) trace_stamp(p, 6);
     __syncwarp();
@@ -1182,7 +1294,10 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
       // acq_rel at CTA scope: the warp completing the entry sees every
       // other warp's h stores, then releases them GPU-wide
       const unsigned done = atom_add_acqrel_cta_smem(reinterpret_cast<unsigned*>(s_cnt + u), 1u) + 1u;
-      if ((int)done == gu_items) grid_arrive(gu_counter(fw, u));
+      if ((int)done == gu_items) {
+        if constexpr (kSplitK) st_release_cta_smem(s_hrdy + u, 1u);
+        else grid_arrive(gu_counter(fw, u));
+      }
     }
     __syncwarp();
   };
@@ -1195,6 +1310,10 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
     }
     done_gu[tid] = done_d[tid] = 0u;
     fence_mbar_init();
+  }
+  if constexpr (kSplitK) {
+    for (int i = tid; i < M * H; i += kFusedThreads) ycta[i] = 0.f;
+    for (int i = tid; i < pl.dchunks + pl.max_union; i += kFusedThreads) s_chunk[i] = 0u;  // and s_hrdy
   }
   if (tid == 0) {
     mbar_init(wr_bar, 1);
@@ -1223,6 +1342,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
   }
   if constexpr (kShared) {
     if (tid < M) s_pm[tid] = tid;
+    if constexpr (kSplitK) {
+      if (tid < M) s_pw[tid] = 1.f;  // the shared expert's weight
+    }
   }
   unsigned* s_amax_u = reinterpret_cast<unsigned*>(s_amax);
   if (tid < M) s_amax_u[tid] = 0u;
@@ -1232,7 +1354,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
     // the shared entry's chunks, into slot 0 of each ring (its barriers were
     // initialised before the block barrier above)
     if (lane == 0 && warp == kFusedWarps - 1 && nr > 0) issue_gu(0);
-    if (lane == 0 && warp == kFusedWarps - 2 && nrd > 0) issue_d(0);
+    if (lane == 0 && warp == kFusedWarps - 2 && (kSplitK ? nr > 0 : nrd > 0)) issue_d(0);
   }
 
   // ---- A1: per-token amax (unsigned max of |x| bit patterns) and, when it
@@ -1510,12 +1632,20 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
     __syncwarp();
     for (int u = ub + lane; u < U; u += 32) s_cnt[u] = 0;  // per-entry gate/up item counters
   }
+  if constexpr (kSplitK) {
+    // routing weight of every routed pair position
+    if (warp == 0) {
+      __syncwarp();
+      for (int i = lane; i < np; i += 32) s_pw[s_ppos[i]] = s_w[i];
+    }
+  }
   __syncthreads();
   const int U = s_int[0];
   trace_stamp(p, 4);
 
   const int n_gu0 = (nr > 0) ? min(U, pl.ns_gu) : 0;
-  const int n_d0 = (nrd > 0) ? min(U, pl.ns_d) : 0;
+  const bool has_d = kSplitK ? (nr > 0) : (nrd > 0);  // this CTA streams down chunks
+  const int n_d0 = has_d ? min(U, pl.ns_d) : 0;
   if (lane == 0 && (ub + warp < n_gu0 || ub + warp < n_d0)) {
     // ring_gu and ring_d were read and written through the generic proxy
     // during routing; order that before the async-proxy (TMA) writes
@@ -1530,7 +1660,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
     // polls both rings without suspending and issues whichever slot drains
     // first, in entry order per ring, so neither ring waits behind the other
     if (lane == 0) {
-      int ug = (nr > 0) ? n_gu0 : U, ud = (nrd > 0) ? n_d0 : U;
+      int ug = (nr > 0) ? n_gu0 : U, ud = has_d ? n_d0 : U;
       if (ug < U || ud < U) {
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         long long t0 = clock64();
@@ -1566,7 +1696,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
   //   gate/up of the entry on every CTA, which never waits on down work, so
   //   the second cannot deadlock either.
   const unsigned long long tgt = (unsigned long long)epoch * G;
-  if (gu_items == 0 && warp == 1 && lane == 0) {
+  if (!kSplitK && gu_items == 0 && warp == 1 && lane == 0) {
     // no gate/up rows here: this CTA's part of every entry is trivially done
     for (int u = 0; u < U; ++u) grid_arrive(gu_counter(fw, u));
   }
@@ -1602,6 +1732,27 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
     }
     if (!is_down) {
       gu_work(u, sub);
+    } else if constexpr (kSplitK) {
+      // split-K down chunk `sub` of entry u over this CTA's K slice; chunk c
+      // of entry u accumulates after chunk c of entry u - 1 (fixed order)
+      const int c = sub;
+      const int slot = u % pl.ns_d, use = u / pl.ns_d;
+      const int pb = s_poff[u], pe = s_poff[u + 1];
+      if (lane == 0) {
+        if (use > 0) smem_count_wait(done_d + slot, (unsigned)(use * d_items), p);
+        smem_acquire_wait(s_hrdy + u, 1u, p);
+        smem_acquire_wait(s_chunk + c, (unsigned)u, p);
+      }
+      __syncwarp();
+      mbar_wait(full_d + slot, use & 1, p);
+      sk_down_chunk(p, ring_d + (size_t)slot * pl.slot_d, n0, nr, skb0, c, pb, pe,
+                    hsm + (size_t)u * pl.max_tokens * pl.nr_max, pl.nr_max, s_pm, s_pw, ycta);
+      __syncwarp();
+      if (lane == 0) {
+        st_release_cta_smem(s_chunk + c, (unsigned)(u + 1));
+        mbar_arrive(empty_d + slot);
+        atomicAdd(done_d + slot, 1u);
+      }
     } else {
       const int gd = sub;
       const int slot = u % pl.ns_d, use = u / pl.ns_d;
@@ -1640,8 +1791,44 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
   trace_stamp(p, 10);
   consumers_sync();
   trace_stamp(p, 11);
-  // ---- A8: combine in slot order, bf16 out
   const int ct = tid - 32;
+  if constexpr (kSplitK) {
+    // ---- A8 (split-K): publish this CTA's partial y, one grid barrier, then
+    //      rows [r0, r0+nrd) of every token summed over the G partials: thread
+    //      (o, j) adds partials [j*G/T, (j+1)*G/T) of output o, and the T sums
+    //      of an output are added in j order (deterministic)
+    float4* dst = reinterpret_cast<float4*>(fw.ypart + (size_t)b * pl.max_tokens * H);
+    const float4* src = reinterpret_cast<const float4*>(ycta);
+    for (int i = ct; i < M * H / 4; i += kConsumers * 32) dst[i] = src[i];
+    consumers_sync();
+    if (ct == 0) {
+      __threadfence();
+      grid_arrive(fw.fin_cnt);
+      grid_wait(fw.fin_cnt, (unsigned long long)epoch * G, p);
+    }
+    consumers_sync();
+    const int nout = M * nrd;
+    if (nout > 0) {
+      const int tpo = max(1, (kConsumers * 32) / nout);
+      float* red = ycta;  // [nout][tpo], free once published
+      const int o = ct / tpo, j = ct % tpo;
+      if (o < nout) {
+        const int m = o / nrd, rl = o % nrd;
+        const int c0 = j * G / tpo, c1 = (j + 1) * G / tpo;
+        float acc = 0.f;
+        for (int c = c0; c < c1; ++c) acc += __ldcg(fw.ypart + ((size_t)c * pl.max_tokens + m) * H + r0 + rl);
+        red[o * tpo + j] = acc;
+      }
+      consumers_sync();
+      if (ct < nout) {
+        float acc = 0.f;
+        for (int j2 = 0; j2 < tpo; ++j2) acc += red[ct * tpo + j2];
+        p.y[(size_t)(ct / nrd) * H + r0 + ct % nrd] = __float2bfloat16_rn(acc);
+      }
+    }
+    if (b == 0 && ct == 0) st_relaxed_u32(fw.epoch, epoch);
+  } else {
+  // ---- A8: combine in slot order, bf16 out
   for (int i = ct; i < M * nrd; i += kConsumers * 32) {
     const int m = i / nrd, rl = i % nrd;
     float acc = 0.f;
@@ -1653,6 +1840,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
     // keep every entry's counter at epoch * G for the next launch
     for (int u = U; u < pl.max_union; ++u) red_release_add_u64(gu_counter(fw, u), (unsigned long long)G);
     st_relaxed_u32(fw.epoch, epoch);
+  }
   }
   trace_stamp(p, 12);
 }

@@ -109,7 +109,7 @@ moe_status moe_decode_static(const moe_config* cfg, const float* router_w, const
   if (c.num_experts < 1 || c.num_experts > moe::kMaxExperts) return MOE_ERR_INVALID_ARG;
   if (c.top_k < 1 || c.top_k > c.num_experts || c.top_k > moe::kMaxTopK) return MOE_ERR_INVALID_ARG;
   if (M < 0 || M > moe::kMaxTokens) return MOE_ERR_INVALID_ARG;
-  if (c.flags & (MOE_FLAG_SHARED_EXPERT | MOE_FLAG_PRE_RMSNORM | MOE_FLAG_FP8_INTERMEDIATE))
+  if (c.flags & (MOE_FLAG_SHARED_EXPERT | MOE_FLAG_PRE_RMSNORM | MOE_FLAG_FP8_INTERMEDIATE | MOE_FLAG_SPLITK_DOWN))
     return MOE_ERR_UNSUPPORTED;
   if (M == 0) return MOE_OK;
   if (!router_w || !w13_codes || !w13_scales || !w2_codes || !w2_scales || !x_bf16 || !y_bf16)

@@ -28,6 +28,7 @@ MOE_TC_MIN_TOKENS = 2
 MOE_FLAG_TC_DOWN_MMA = 0x40
 MOE_FLAG_TC_DOWN_CUDA = 0x80
 MOE_TC_DOWN_MMA_MIN_TOKENS = 8
+MOE_FLAG_SPLITK_DOWN = 0x100
 MOE_LOAD_BORROW = 0x0
 MOE_LOAD_SKIP_VALIDATE = 0x1
 MOE_LOAD_COPY_REPACK = 0x2

@@ -53,7 +53,7 @@ def test_create_rejects_bad_config_without_gpu(L):
            moe.moe_config(256, 64, 16, 17, 1, 0, 0),  # top_k > E
            moe.moe_config(256, 64, 16, 2, 33, 0, 0),  # max_tokens > 32
            moe.moe_config(256, 64, 2000, 2, 1, 0, 0),  # E > 1024
-           moe.moe_config(256, 64, 16, 2, 1, 0x100, 0)]  # unknown flag
+           moe.moe_config(256, 64, 16, 2, 1, 0x200, 0)]  # unknown flag
     for c in bad:
         assert L.moe_create(ctypes.byref(c), ctypes.byref(out)) == 1
         assert not out.value
@@ -99,8 +99,8 @@ def test_shared_expert_flag_without_gpu(L):
     assert L.moe_create(ctypes.byref(c), ctypes.byref(out)) == 2 and not out.value
     c = moe.moe_config(256, 64, 16, 2, 1, moe.MOE_FLAG_FP8_INTERMEDIATE | moe.MOE_FLAG_SPLIT_KERNELS, 0)
     assert L.moe_create(ctypes.byref(c), ctypes.byref(out)) == 2 and not out.value
-    # an unknown flag bit is refused as an invalid argument (0x10..0x80 are kernel choices)
-    c = moe.moe_config(256, 64, 16, 2, 1, moe.MOE_FLAG_SHARED_EXPERT | moe.MOE_FLAG_PRE_RMSNORM | 0x100, 0)
+    # an unknown flag bit is refused as an invalid argument (0x10..0x100 are kernel choices)
+    c = moe.moe_config(256, 64, 16, 2, 1, moe.MOE_FLAG_SHARED_EXPERT | moe.MOE_FLAG_PRE_RMSNORM | 0x200, 0)
     assert L.moe_create(ctypes.byref(c), ctypes.byref(out)) == 1 and not out.value
     for shape in [(2560, 768, 256, 8, 1), (2560, 768, 256, 8, 32), (128, 64, 8, 8, 3), (256, 64, 16, 2, 1)]:
         st0, base = moe.plan_query(*shape)
@@ -131,6 +131,18 @@ def test_fp8_intermediate_flag_without_gpu(L):
     out = ctypes.c_void_p()
     c = moe.moe_config(256, 64, 16, 2, 1, F8 | moe.MOE_FLAG_SPLIT_KERNELS, 0)
     assert L.moe_create(ctypes.byref(c), ctypes.byref(out)) == 2 and not out.value
+
+
+def test_splitk_flag_rules_without_gpu(L):
+    out = ctypes.c_void_p()
+    SK = moe.MOE_FLAG_SPLITK_DOWN
+    for flags, mt in ((SK | moe.MOE_FLAG_SPLIT_KERNELS, 1), (SK | moe.MOE_FLAG_FP8_INTERMEDIATE, 1), (SK, 5)):
+        c = moe.moe_config(256, 64, 16, 2, mt, flags, 0)
+        assert L.moe_create(ctypes.byref(c), ctypes.byref(out)) == 2 and not out.value
+    for shape in [(2560, 768, 256, 8, 1), (2560, 768, 256, 8, 4), (256, 64, 16, 2, 1), (128, 64, 8, 8, 3)]:
+        for extra in (0, moe.MOE_FLAG_SHARED_EXPERT):
+            st, pl = moe.plan_query(*shape, flags=SK | extra)
+            assert st == 0 and pl["ok"] and pl["smem"] <= 232448, (shape, pl)
 
 
 def test_plan_rejects_what_does_not_fit(L):

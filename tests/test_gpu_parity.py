@@ -189,6 +189,26 @@ def test_fp8_intermediate_m32_sampled():
     _check_a8(L, got, tokens=[0, 17, 31])
 
 
+@pytest.mark.parametrize("shape,M,mode,shared", [((256, 64, 16, 2), 1, "natural", False),
+                                                 ((160, 96, 12, 4), 3, "gap", False),
+                                                 ((2560, 768, 256, 8), 1, "gap", False),
+                                                 ((2560, 768, 256, 8), 4, "natural", False),
+                                                 ((2560, 768, 256, 8), 4, "shared", False),
+                                                 ((2560, 768, 256, 8), 1, "gap", True),
+                                                 ((2560, 768, 256, 8), 3, "natural", True),
+                                                 ((128, 64, 8, 8), 3, "natural", False)])
+def test_splitk_down(shape, M, mode, shared):
+    """Down projection split over K (CTA-local h, K-major W2 copy, fixed-order
+    reduction of the per-CTA partial outputs), every token checked, and the
+    same bits on a second call."""
+    H, I, E, K = shape
+    L = Layer(H, I, E, K, M, seed=41, mode=mode, shared=shared)
+    ctx = L.make_ctx(moe.MOE_FLAG_SPLITK_DOWN)
+    got = L.run(ctx)
+    compare(L, got, L.oracle(), check_ids=E != K)
+    assert torch.equal(got["y"], L.run(ctx)["y"])
+
+
 @pytest.mark.parametrize("M,mode", [(1, "gap"), (2, "zipf"), (4, "gap"), (3, "shared")])
 def test_deep_ring_reuse(M, mode):
     """A context sized for 32 tokens leaves 4 ring slots, so every slot is
