@@ -219,6 +219,7 @@ def run_ours(args):
              "tc": moe.MOE_FLAG_TENSOR_CORES}.get(args.variant, 0)
     flags |= moe.MOE_FLAG_FP8_INTERMEDIATE if args.fp8_intermediate else 0
     flags |= moe.MOE_FLAG_SPLITK_DOWN if args.splitk_down else 0
+    flags |= {"mma": moe.MOE_FLAG_TC_DOWN_MMA, "cuda": moe.MOE_FLAG_TC_DOWN_CUDA}.get(args.tc_down, 0)
     x, ctxs, _weights = build_pool(device, M, args.routing, layers=L, flags=flags, stack=args.stack,
                                    shared=args.shared_expert, repack=args.repack)
     n_shared = int(args.shared_expert)
@@ -327,7 +328,8 @@ def run_ours(args):
                    "l2": "inputs larger than L2: each layer-step reads a different layer of the pool",
                    "step": (f"{L}-layer stack (RMSNorm between layers) in one CUDA graph" if args.stack
                             else f"{L} layer-steps in one CUDA graph"), "parallelism": f"replicas x{ws}",
-                   "variant": info["variant"]},
+                   "variant": info["variant"], **({"down": info["down"]} if "down" in info else {}),
+                   **({"splitk_down": True} if args.splitk_down else {})},
         "us_per_layer_step": round(us_per_layer, 3),
         "union_experts": U_mean,
         "expert_gbs": round(exp_b / (us_per_layer * 1e-6) / 1e9, 1),
@@ -716,6 +718,9 @@ def main():
                     help="load the layers with MOE_LOAD_COPY_REPACK (context-owned, kernel-private weight layout)")
     ap.add_argument("--shared-expert", action="store_true",
                     help="one always-active shared expert per layer besides the top-8 routed ones")
+    ap.add_argument("--tc-down", choices=["auto", "mma", "cuda"], default="auto",
+                    help="tensor-core kernel's down projection: auto (the library's choice), mma (tcgen05), "
+                         "cuda (CUDA cores)")
     ap.add_argument("--splitk-down", action="store_true",
                     help="down projection split over K with CTA-local h (max 4 tokens)")
     ap.add_argument("--fp8-intermediate", action="store_true",

@@ -131,7 +131,7 @@ typedef enum {
                                        step; moe_query names the one a context
                                        runs. Setting both flags is
                                        MOE_ERR_INVALID_ARG */
-#define MOE_TC_MIN_TOKENS 2
+#define MOE_TC_MIN_TOKENS 4
 #define MOE_FLAG_TC_DOWN_MMA 0x40u   /* tensor-core kernel: run the down
                                        projection on tcgen05 MMAs as well
                                        (tiles of 128 output rows x up to 16
@@ -149,7 +149,7 @@ typedef enum {
                                        MOE_TC_DOWN_MMA_MIN_TOKENS tokens of
                                        max_tokens on. Both flags:
                                        MOE_ERR_INVALID_ARG */
-#define MOE_TC_DOWN_MMA_MIN_TOKENS 8
+#define MOE_TC_DOWN_MMA_MIN_TOKENS 2
 
 typedef struct {
   int32_t hidden;      /* H: multiple of 32, 32..8192                        */

@@ -214,9 +214,12 @@ bool make_tc_plan(const moe_config& c, int sm_count, size_t smem_limit, moe::TcP
   while (ns_d > 2 && room < ns_d * per_d + 2 * (size_t)pl->slot_gu) --ns_d;
   if (room < ns_d * per_d) return false;
   room -= ns_d * per_d;
-  size_t ns_gu = std::min<size_t>({(size_t)moe::kTcMaxSlots, nstage, room / pl->slot_gu});
-  if (ns_gu < 1) return false;
-  if (ns_gu < 2 && nstage >= 2) return false;
+  // the deepest gate/up ring whose exact layout fits (the estimate above
+  // is conservative)
+  const size_t ns_min = (nstage >= 2) ? 2 : 1;
+  if (room / pl->slot_gu < ns_min) return false;
+  for (size_t ns_gu = std::min<size_t>({(size_t)moe::kTcMaxSlots, nstage, room / pl->slot_gu + 2}); ns_gu >= ns_min;
+       --ns_gu) {
   pl->ns_gu = (int)ns_gu;
   pl->ns_d = (int)ns_d;
   // layout
@@ -263,7 +266,9 @@ bool make_tc_plan(const moe_config& c, int sm_count, size_t smem_limit, moe::TcP
   pl->o_poff = (int)take((UMAX + 1) * 4, 16);
   pl->o_dsm = (int)take(dsm_bytes, 16);
   pl->smem_bytes = (int)(off + 1024);
-  return (size_t)pl->smem_bytes <= smem_limit;
+  if ((size_t)pl->smem_bytes <= smem_limit) return true;
+  }
+  return false;
 }
 
 // cuTensorMapEncodeTiled from the driver, looked up once through the runtime

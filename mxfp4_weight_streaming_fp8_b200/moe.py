@@ -24,10 +24,10 @@ MOE_FLAG_SHARED_EXPERT = 0x4
 MOE_FLAG_FP8_INTERMEDIATE = 0x8
 MOE_FLAG_CUDA_CORES = 0x10
 MOE_FLAG_TENSOR_CORES = 0x20
-MOE_TC_MIN_TOKENS = 2
+MOE_TC_MIN_TOKENS = 4
 MOE_FLAG_TC_DOWN_MMA = 0x40
 MOE_FLAG_TC_DOWN_CUDA = 0x80
-MOE_TC_DOWN_MMA_MIN_TOKENS = 8
+MOE_TC_DOWN_MMA_MIN_TOKENS = 2
 MOE_FLAG_SPLITK_DOWN = 0x100
 MOE_LOAD_BORROW = 0x0
 MOE_LOAD_SKIP_VALIDATE = 0x1

@@ -228,12 +228,16 @@ def test_mma_down_ling(M, mode):
 
 
 def test_mma_down_is_default_from_min_tokens():
-    L = Layer(2560, 768, 256, 8, 2, seed=63, mode="gap")
-    ctx = L.make_ctx(0, max_tokens=moe.MOE_TC_DOWN_MMA_MIN_TOKENS)
+    L = Layer(2560, 768, 256, 8, 1, seed=63, mode="gap")
+    ctx = L.make_ctx(moe.MOE_FLAG_TENSOR_CORES, max_tokens=moe.MOE_TC_DOWN_MMA_MIN_TOKENS)
     assert ctx.query()["down"] == "tensor_cores"
     compare(L, L.run(ctx), L.oracle())
-    ctx = L.make_ctx(0, max_tokens=moe.MOE_TC_DOWN_MMA_MIN_TOKENS - 1)
+    ctx = L.make_ctx(moe.MOE_FLAG_TENSOR_CORES, max_tokens=moe.MOE_TC_DOWN_MMA_MIN_TOKENS - 1)
     assert ctx.query()["down"] == "cuda_cores"
+    # without a kernel flag the library picks the tensor-core kernel from
+    # MOE_TC_MIN_TOKENS tokens of max_tokens on
+    assert L.make_ctx(0, max_tokens=moe.MOE_TC_MIN_TOKENS).query()["variant"] == "tc"
+    assert L.make_ctx(0, max_tokens=moe.MOE_TC_MIN_TOKENS - 1).query()["variant"] == "fused"
 
 
 def test_mma_down_agrees_with_cuda_core_down():
