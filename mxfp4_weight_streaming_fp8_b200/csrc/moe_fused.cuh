@@ -534,12 +534,17 @@ __device__ __forceinline__ void stage_h(const Params& p, int pb, int pe, __half2
     const uint4* hp = reinterpret_cast<const uint4*>(p.ws.h + (size_t)pp * I);
     __half2* dst = hbuf + (size_t)j * (I / 2);
     if (I / 4 <= 32 * kQ) {
+      // lane's groups q = (lane + 32k + rot) mod I/4: the start rotates with
+      // the CTA, so the 148 CTAs that stage an expert's h together spread
+      // their first reads over its L2 lines instead of all asking for the
+      // same line at once
+      const int nq = I / 4, rot = (int)((blockIdx.x * 8u) % (unsigned)nq);
       uint4 v[kQ];
       float mx = 0.f;
 #pragma unroll
       for (int k = 0; k < kQ; ++k) {
-        const int q = lane + 32 * k;
-        v[k] = (q < I / 4) ? ld_cg_u4(hp + q) : make_uint4(0u, 0u, 0u, 0u);
+        const int q0 = lane + 32 * k, q = (q0 + rot >= nq) ? q0 + rot - nq : q0 + rot;
+        v[k] = (q0 < nq) ? ld_cg_u4(hp + q) : make_uint4(0u, 0u, 0u, 0u);
       }
 #pragma unroll
       for (int k = 0; k < kQ; ++k)
@@ -549,8 +554,8 @@ __device__ __forceinline__ void stage_h(const Params& p, int pb, int pe, __half2
         const float amax = warp_max(mx), inv = h_fp8_inv(amax);
 #pragma unroll
         for (int k = 0; k < kQ; ++k) {
-          const int q = lane + 32 * k;
-          if (q < I / 4) {
+          const int q0 = lane + 32 * k, q = (q0 + rot >= nq) ? q0 + rot - nq : q0 + rot;
+          if (q0 < nq) {
             uint32_t* d32 = reinterpret_cast<uint32_t*>(dst + 2 * q);
             d32[0] = h_fp8x2(__uint_as_float(v[k].x), __uint_as_float(v[k].y), inv);
             d32[1] = h_fp8x2(__uint_as_float(v[k].z), __uint_as_float(v[k].w), inv);
@@ -562,8 +567,8 @@ __device__ __forceinline__ void stage_h(const Params& p, int pb, int pe, __half2
         const float up = ldexpf(1.f, t);
 #pragma unroll
         for (int k = 0; k < kQ; ++k) {
-          const int q = lane + 32 * k;
-          if (q < I / 4) {
+          const int q0 = lane + 32 * k, q = (q0 + rot >= nq) ? q0 + rot - nq : q0 + rot;
+          if (q0 < nq) {
             dst[2 * q] = __floats2half2_rn(__uint_as_float(v[k].x) * up, __uint_as_float(v[k].y) * up);
             dst[2 * q + 1] = __floats2half2_rn(__uint_as_float(v[k].z) * up, __uint_as_float(v[k].w) * up);
           }
@@ -1015,13 +1020,18 @@ __device__ __forceinline__ bool poll_tagged_logits(const Params& p, const unsign
                                                    unsigned want, float* s_logit) {
   constexpr int kB = 8;
   const long long t0 = clock64();
+  // word order rotated by CTA, so the CTAs do not all ask for the same
+  // L2 line at once
+  const int rot = (int)((blockIdx.x * 16u) % (unsigned)n);
   bool ok = true;
   for (int i0 = threadIdx.x; i0 < n; i0 += kB * blockDim.x) {
     unsigned long long w[kB];
+    int idx[kB];
 #pragma unroll
     for (int j = 0; j < kB; ++j) {
       const int i = i0 + j * blockDim.x;
-      w[j] = (i < n) ? ld_relaxed_u64(words + i) : ((unsigned long long)want << 32);
+      idx[j] = (i + rot >= n) ? i + rot - n : i + rot;
+      w[j] = (i < n) ? ld_relaxed_u64(words + idx[j]) : ((unsigned long long)want << 32);
     }
 #pragma unroll
     for (int j = 0; j < kB; ++j) {
@@ -1032,9 +1042,9 @@ __device__ __forceinline__ bool poll_tagged_logits(const Params& p, const unsign
           atomicOr(p.ws.ctrl, kStatusTimeout);
           ok = false;
         }
-        w[j] = ld_relaxed_u64(words + i);
+        w[j] = ld_relaxed_u64(words + idx[j]);
       }
-      if (i < n) s_logit[i] = __uint_as_float((unsigned)w[j]);
+      if (i < n) s_logit[idx[j]] = __uint_as_float((unsigned)w[j]);
     }
   }
   return ok;
@@ -1363,7 +1373,10 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
     const uint4* x16 = reinterpret_cast<const uint4*>(p.x);
     int mcur = -1;
     float a = 0.f;
-    for (int i = tid; i < M * H / 8; i += kFusedThreads) {
+    // start rotated by CTA: the CTAs spread their first reads over x's lines
+    const int nx8 = M * H / 8, rot8 = (int)((b * 8u) % (unsigned)nx8);
+    for (int i0 = tid; i0 < nx8; i0 += kFusedThreads) {
+      const int i = (i0 + rot8 >= nx8) ? i0 + rot8 - nx8 : i0 + rot8;
       const int m = (i * 8) / H;
       if (m != mcur) {
         if (mcur >= 0) atomicMax(&s_amax_u[mcur], __float_as_uint(a));

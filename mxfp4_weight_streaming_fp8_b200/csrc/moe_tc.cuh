@@ -663,7 +663,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc(Params p, TcWs tw, TcPlan 
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   } else {
   // ---- A1 (first half): stage x (when it fits), per-token amax
-  for (int i = tid; i < M * H / 8; i += kTcThreads) {
+  const int nx8 = M * H / 8, rot8 = (int)((b * 8u) % (unsigned)nx8);  // CTA-rotated start
+  for (int i0 = tid; i0 < nx8; i0 += kTcThreads) {
+    const int i = (i0 + rot8 >= nx8) ? i0 + rot8 - nx8 : i0 + rot8;
     const int m = (i * 8) / H;
     const uint4 v = __ldcg(reinterpret_cast<const uint4*>(p.x) + i);
     if (pl.x_staged) x_s[i] = v;
