@@ -165,3 +165,67 @@ def test_lm_head_entry_points_reject_bad_arguments_without_a_gpu(L):
     buf = ctypes.create_string_buffer(64)
     assert L.moe_lm_query(None, buf, 64) == 1
     L.moe_lm_destroy(None)
+
+
+def _regions(t):
+    """(start, end, name) of the tensor-core kernel's shared-memory regions."""
+    NP, UMAX = t["max_pairs"], t["max_union"]
+    regs = {"ring_gu": (t["o_ring_gu"], max(t["ns_gu"] * t["slot_gu"], t["wr_bytes_max"])),
+            "bx": (t["o_bx"], t["bx_bytes"]), "sc": (t["o_sc"], 2 * t["sc_bytes"]),
+            "ring_d": (t["o_ring_d"], t["ns_d"] * t["slot_d"]),
+            "ids": (t["o_ids"], NP * 4), "w": (t["o_w"], NP * 4), "pm": (t["o_pm"], NP * 4),
+            "ppos": (t["o_ppos"], NP * 4), "union": (t["o_union"], UMAX * 4), "poff": (t["o_poff"], (UMAX + 1) * 4)}
+    if t["mma_down"]:
+        regs.update(bd=(t["o_bd"], 2 * t["bd_bytes"]), dsc=(t["o_dsc"], 4 * 16 * 4),
+                    dtoff=(t["o_dtoff"], (UMAX + 1) * 4))
+    else:
+        regs["dsm"] = (t["o_dsm"], NP * t["rpc_max"] * 4)
+    return sorted((o, o + s, n) for n, (o, s) in regs.items() if s > 0)
+
+
+@pytest.mark.parametrize("MM", [1, 2, 3, 4, 8, 16, 32])
+@pytest.mark.parametrize("extra", [0, moe.MOE_FLAG_SHARED_EXPERT])
+def test_tensor_core_plan_and_kernel_choice(L, MM, extra):
+    """The tensor-core kernel's plan at the Ling shape: chosen from
+    MOE_TC_MIN_TOKENS tokens on, its down projection on tensor cores from
+    MOE_TC_DOWN_MMA_MIN_TOKENS, non-overlapping shared-memory regions inside
+    the opt-in limit, a gate/up ring of at least two 16 KB slots when the
+    down projection shares it, and the B operand buffers large enough for
+    the routing scratch they hold until routing ends."""
+    st, pl = moe.plan_query(2560, 768, 256, 8, MM, flags=extra, sm_count=148, smem_limit=232448)
+    assert st == 0 and pl["ok"]
+    assert pl["variant"] == ("tc" if MM >= moe.MOE_TC_MIN_TOKENS else "fused")
+    t = pl["tc"]
+    assert t["ok"] and t["smem"] <= 232448
+    assert t["mma_down"] == int(MM >= moe.MOE_TC_DOWN_MMA_MIN_TOKENS)
+    if t["mma_down"]:
+        assert t["tu_max"] == 16 and t["ks"] == 1 and t["slot_gu"] == 16384 and t["ns_gu"] >= 2
+        assert t["ns_d"] == 0 and t["dkch"] == 768 // 128 and t["bd_bytes"] == 6 * 4096
+        assert t["o_bd"] % 1024 == 0
+        if t["o_lg"] == t["o_bd"]:
+            assert MM * 256 * 4 + 256 * 4 <= 2 * t["bd_bytes"]
+    regs = _regions(t)
+    for a, b in zip(regs, regs[1:]):
+        assert a[1] <= b[0], (a, b)
+    assert regs[-1][1] <= t["smem"] - 1024
+
+
+def test_tensor_core_down_flags_without_gpu(L):
+    out = ctypes.c_void_p()
+    both = moe.MOE_FLAG_TC_DOWN_MMA | moe.MOE_FLAG_TC_DOWN_CUDA
+    c = moe.moe_config(2560, 768, 256, 8, 4, both, 0)
+    assert L.moe_create(ctypes.byref(c), ctypes.byref(out)) == 1 and not out.value
+    c = moe.moe_config(2560, 768, 256, 8, 4, moe.MOE_FLAG_TENSOR_CORES | moe.MOE_FLAG_SPLITK_DOWN, 0)
+    assert L.moe_create(ctypes.byref(c), ctypes.byref(out)) == 1 and not out.value
+    # forced either way on the plan
+    st, pl = moe.plan_query(2560, 768, 256, 8, 1, flags=moe.MOE_FLAG_TC_DOWN_MMA)
+    assert st == 0 and pl["tc"]["mma_down"] == 1
+    st, pl = moe.plan_query(2560, 768, 256, 8, 32, flags=moe.MOE_FLAG_TC_DOWN_CUDA)
+    assert st == 0 and pl["tc"]["mma_down"] == 0 and pl["tc"]["ns_d"] >= 2
+    # I > H: a down tile's scale factors would not fit a gate/up tile's
+    # tensor-memory columns, so the default keeps the CUDA-core down and a
+    # forced tensor-core down has no plan
+    st, pl = moe.plan_query(512, 768, 64, 8, 8)
+    assert pl["tc"]["ok"] and pl["tc"]["mma_down"] == 0
+    st, pl = moe.plan_query(512, 768, 64, 8, 8, flags=moe.MOE_FLAG_TC_DOWN_MMA)
+    assert not pl["tc"]["ok"]
