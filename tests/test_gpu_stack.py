@@ -23,13 +23,17 @@ def _bf16_ulp_diff(a_bits, b_bits):
     return np.abs(sa - sb)
 
 
-@pytest.mark.parametrize("M", [1, 3])
-def test_three_layer_stack_teacher_forced(M):
+@pytest.mark.parametrize("M,kernel", [(1, 0), (3, 0), (1, moe.MOE_FLAG_TENSOR_CORES),
+                                      (5, moe.MOE_FLAG_TENSOR_CORES)])
+def test_three_layer_stack_teacher_forced(M, kernel):
+    """kernel 0: the library's choice (the CUDA-core kernel below 4 tokens);
+    MOE_FLAG_TENSOR_CORES: the tensor-core kernel (its one-token routing at
+    M=1, the per-warp token routing with the RMSNorm factor at M=5)."""
     H, I, E, K, seed = 2560, 768, 256, 8, 21
     dev = torch.device("cuda:0")
     x_in = synth.gen_x(seed, M, H)  # bf16, layer 0 input (not normalised)
     for l in range(3):
-        flags = moe.MOE_FLAG_PRE_RMSNORM if l > 0 else 0
+        flags = (moe.MOE_FLAG_PRE_RMSNORM if l > 0 else 0) | kernel
         xin_bits = bits(x_in)
         # the oracle's view of this layer's routing input
         xr_bits = oracle.rmsnorm(xin_bits, 1e-6) if l > 0 else xin_bits
@@ -37,6 +41,8 @@ def test_three_layer_stack_teacher_forced(M):
         wr = synth.force_router(xr, synth.gen_router(seed, l, E, H), K, "gap", seed=seed, layer=l)
         ex = synth.layer_experts_torch(seed, l, E, H, I, dev)
         ctx = moe.MoELayer(H, I, E, K, M, flags=flags)
+        if kernel:
+            assert ctx.query()["variant"] == "tc"
         ctx.load_experts(torch.from_numpy(wr).to(dev), *ex)
         out = ctx.decode(x_in.to(dev), routing=True)
         y, ids, w, xq, xs = out[:5]
