@@ -247,15 +247,18 @@ moe_status moe_plan_query(const moe_config* cfg, int32_t sm_count, size_t smem_l
  * reports MOE_ERR_TIMEOUT. Returns INVALID_ARG for a NULL ctx. */
 moe_status moe_debug_set_wait(moe_ctx* ctx, long long budget_cycles, int force_stall);
 
-/* Test hook for measurements of the tensor-core kernel: with a non-NULL
- * device pointer to grid x 16 uint64 words (8-byte aligned), every later
- * moe_decode of this context writes %globaltimer stamps of its phases per CTA
- * there (slot 0 kernel start, 1 after the programmatic-launch wait, 2 logits
- * published, 3 all logits gathered, 4 routing done, 5 first gate/up stage
- * landed, 6 last MMA issued, 7 gate/up epilogue done, 9 last entry's h
- * ready, 10/11 down work done, 12 kernel end); slots not reached keep their
- * value. NULL turns it off. Ignored by the other kernels. Returns
- * INVALID_ARG for a NULL ctx or a misaligned pointer. */
+/* Test hook for timeline measurements of the persistent kernels (k_fused and
+ * k_tc): with a non-NULL device pointer to grid x 64 uint64 words (8-byte
+ * aligned; grid = the "grid" moe_query reports), every later moe_decode of
+ * this context writes %globaltimer stamps of its phases, 64 slots per CTA
+ * (lane 0 of the warp that reaches a phase writes it; the last writer wins).
+ * Common slots: 0 kernel start, 1 after the programmatic-launch wait, 2 the
+ * E4M3 codes written, 3 logit words gathered, 4 routing done, 8 top-k done,
+ * 10/11 down work done and combine start, 12 kernel end; the other slots
+ * mark kernel-specific points (stages landed, MMAs issued, epilogue, down
+ * items or tiles). Slots not reached keep their value. NULL turns it off.
+ * Ignored by the three-kernel form. Returns INVALID_ARG for a NULL ctx or a
+ * misaligned pointer. */
 moe_status moe_debug_set_trace(moe_ctx* ctx, unsigned long long* trace);
 
 /* Size of the fixed device scratch array behind moe_decode_static. */

@@ -192,9 +192,15 @@ class MoELayer:
     def set_wait(self, budget_cycles: int, force_stall: bool = False) -> int:
         return lib().moe_debug_set_wait(self._ctx, int(budget_cycles), int(bool(force_stall)))
 
+    TRACE_SLOTS = 64  # timestamps per CTA the kernels may write
+
     def set_trace(self, trace) -> int:
-        """Per-CTA phase timestamps of the tensor-core kernel into a device
-        uint64 tensor of grid x 48 words (None turns it off)."""
+        """Per-CTA phase timestamps of the persistent kernels into a device
+        int64/uint64 tensor of at least grid x 64 words (None turns it off)."""
+        if trace is not None:
+            need = self.query()["grid"][0] * self.TRACE_SLOTS
+            if trace.numel() < need or trace.element_size() != 8:
+                raise ValueError(f"trace needs {need} 8-byte words")
         return lib().moe_debug_set_trace(self._ctx, _ptr(trace))
 
     def query(self) -> dict:
