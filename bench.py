@@ -373,6 +373,129 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+def run_split(args):
+    """--parts G: the intra-expert split of every pool layer (part g holds
+    gate/up rows [g*I/G, (g+1)*I/G) of each expert and the same down
+    columns). Under torchrun with N = G ranks, rank g holds part g and a
+    layer-step is moe_decode of the part (fp32 sums), one NCCL all-reduce of
+    the M x H sums and the bf16 round (moe.decode_split); the whole layer's
+    work is fixed, so scaling is strong and each token counts once. In one
+    process with G > 1 it times part 0 of G alone in one CUDA graph, as the
+    default bench times whole layers: the per-GPU kernel time of a G-way
+    split, without the exchange."""
+    import torch
+    ws, rank, local = dist_env()
+    G = args.parts
+    if ws > 1 and ws != G:
+        raise SystemExit("--parts must equal the number of ranks")
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    device = torch.device("cuda", local if ws > 1 else 0)
+    torch.cuda.set_device(device)
+    from mxfp4_weight_streaming_fp8_b200 import moe, synth
+    M, L, g = args.tokens, args.layers, (rank if ws > 1 else 0)
+    x = synth.gen_x(SEED, M, H)
+    ctxs = []
+    for l in range(L):
+        wr = synth.force_router(x, synth.gen_router(SEED, l, E, H), K, args.routing, seed=SEED, layer=l)
+        ex = synth.layer_experts_torch(SEED, l, E, H, I, device)
+        ctx = moe.MoELayer(H, I, E, K, M, device=device.index, shard=(g, G))
+        ctx.load_experts(torch.from_numpy(wr).to(device), *ex, validate=False)  # keeps a copy of part g
+        del ex
+        ctxs.append(ctx)
+    info = ctxs[0].query()
+    x_d = x.to(device)
+    y32 = [torch.empty((M, H), dtype=torch.float32, device=device) for _ in range(L)]
+    ys = [torch.empty_like(x_d) for _ in range(L)]
+    Us = []
+    for l in range(L):
+        out = ctxs[l].decode(x_d, y=y32[l], routing=True)
+        Us.append(len(set(out[1].cpu().numpy().ravel().tolist())))
+    torch.cuda.synchronize()
+    cur = torch.cuda.current_stream()
+    graph = None
+    if ws == 1:
+        stream = torch.cuda.Stream(device)
+        stream.wait_stream(cur)
+        with torch.cuda.stream(stream):
+            for l in range(L):
+                assert ctxs[l].decode_raw(x_d, M, y32[l], stream=stream) == moe.MOE_OK
+        cur.wait_stream(stream)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            for l in range(L):
+                assert ctxs[l].decode_raw(x_d, M, y32[l], stream=stream) == moe.MOE_OK
+
+    def step():
+        if graph is not None:
+            graph.replay()
+        else:
+            for l in range(L):
+                moe.decode_split(ctxs[l], x_d, y32=y32[l], y=ys[l])
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(device.index) as clk:
+        ev0.record(cur)
+        for _ in range(args.steps):
+            step()
+        ev1.record(cur)
+        ev1.synchronize()
+    torch.cuda.synchronize()
+    ms = max_over_ranks(ev0.elapsed_time(ev1), ws, device)
+    for c in ctxs:
+        st = c.sync_status()
+        if st != moe.MOE_OK:
+            raise RuntimeError(f"kernel status {moe.status_string(st)}")
+    us = ms * 1e3 / (args.steps * L)
+    U_mean = sum(Us) / len(Us)
+    # a part reads 1/G of each active expert, the whole router, x, and writes fp32 sums
+    alg = U_mean * expert_bytes(H, I // G) + E * H * 4 + M * H * 2 + M * H * 4
+    peak, peak_kind = load_peaks()
+    achieved = alg / (us * 1e-6) / 1e9
+    alone = ws == 1
+    line = {
+        "metric": METRIC, "value": round(M * args.steps * L / (ms / 1e3), 1), "unit": "tokens/s", "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 4),
+        "higher_is_better": True, "scaling": "weak" if alone else "strong", "vs_baseline": None,
+        "dtype": "fp8e4m3 x mxfp4 (f16/fp32 accumulate)",
+        "data": "synthetic (seeded SplitMix64; random MXFP4 weights, N(0,1) bf16 activations)",
+        "config": {"workload": f"ling_layer_M{M}_{args.routing}_split{G}" + ("_part0_alone" if alone else ""),
+                   "hidden": H, "inter": I, "inter_per_part": I // G, "num_experts": E, "top_k": K,
+                   "tokens": M, "routing": args.routing, "layers_in_pool": L,
+                   "l2": "inputs larger than L2: each layer-step reads a different layer of the pool",
+                   "step": (f"part 0 of {G} of {L} layers in one CUDA graph (no exchange)" if alone else
+                            f"{L} layers, each: part of rank g, NCCL all-reduce of fp32 sums, bf16 round"),
+                   "parallelism": f"intra-expert split x{G}", "variant": info["variant"]},
+        "us_per_layer_step": round(us, 3),
+        "union_experts": U_mean,
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "peak_kind": peak_kind, "traffic": None,
+                     "kernel": {"fused": "k_fused", "tc": "k_tc"}.get(info["variant"], "k_gateup+k_down"),
+                     "algorithmic_bytes_per_launch": alg},
+        "gpu_launches": args.steps * L * (1 if alone else 2),
+        "clocks": clk.summary(),
+        "e2e": None,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del graph
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def build_chain(device, ctxs, weights, x_d, M, flags, shared, repack=False):
     """Contexts over the pool's own weights chained as a stack (layers after
     the first normalise their input), captured in one CUDA graph."""
@@ -727,6 +850,9 @@ def main():
                     help="quantise the SwiGLU output to E4M3 per (token, expert) before the down projection")
     ap.add_argument("--stack", action="store_true",
                     help="chain the pool as a stack: layer l+1 takes RMSNorm(y_l)")
+    ap.add_argument("--parts", type=int, default=1,
+                    help="intra-expert split into this many parts: one per rank under torchrun; in one "
+                         "process, part 0 alone (its per-GPU kernel time)")
     ap.add_argument("--op", choices=["moe", "lm_head"], default="moe",
                     help="moe: the MoE layer step (default); lm_head: the FP8 LM head GEMV")
     args = ap.parse_args()
@@ -738,6 +864,8 @@ def main():
         run_reference(args)
     elif args.op == "lm_head":
         run_lm_head(args)
+    elif args.parts > 1:
+        run_split(args)
     else:
         run_ours(args)
 

@@ -159,7 +159,27 @@ typedef struct {
   int32_t max_tokens;  /* upper bound on M per call: 1..32                   */
   uint32_t flags;      /* MOE_FLAG_*                                         */
   int32_t device;      /* CUDA device ordinal the context lives on          */
+  int32_t shard_index; /* intra-expert split: this context's part g, 0..G-1  */
+  int32_t shard_count; /* G, the number of parts (0 or 1: the whole layer)   */
 } moe_config;
+
+/* Intra-expert split of one layer over G GPUs (shard_count = G > 1). Part g
+ * holds rows [g*I/G, (g+1)*I/G) of every expert's gate and of its up
+ * projection, and the same columns of its down projection: h_n depends on
+ * row n of gate and up only, and the down product is a sum over n, so
+ *   y[m][r] = bf16( sum over g of P_g[m][r] )
+ * where P_g is A8's slot-order sum taken over part g's columns alone. Every
+ * part reads 1/G of each active expert, so the parts stay balanced even for
+ * one token. Routing (A1-A4, and the RMSNorm of MOE_FLAG_PRE_RMSNORM) is not
+ * split: each part computes it from the same x and the whole router. Rules:
+ * I must be a multiple of 32*G (each part keeps whole E8M0 blocks of W2);
+ * G <= 128; 0 <= shard_index < G; MOE_FLAG_FP8_INTERMEDIATE is UNSUPPORTED
+ * (its per-token scale of h spans all I columns, which would need a second
+ * exchange). The context then plans its kernels for width I/G,
+ * moe_load_experts takes the whole layer's arrays and keeps a copy of the
+ * part (MOE_LOAD_COPY_REPACK is required), and moe_decode writes P_g as fp32
+ * [M][H]. The caller adds the parts (one all-reduce over the G GPUs) and
+ * rounds the sum with moe_round_bf16. */
 
 typedef struct moe_ctx moe_ctx; /* opaque */
 
@@ -177,7 +197,7 @@ moe_status moe_create(const moe_config* cfg, moe_ctx** out);
                                        caller may free its arrays after the call */
 
 /* Attach one layer's weights (device pointers, layouts above, each 16-byte
- * aligned).
+ * aligned; for a part of an intra-expert split, the whole layer's arrays).
  * Without MOE_LOAD_COPY_REPACK the context borrows them: nothing is copied,
  * and the caller keeps ownership; the arrays must outlive their use.
  * With MOE_LOAD_COPY_REPACK the context allocates one device buffer for a
@@ -192,7 +212,10 @@ moe_status moe_create(const moe_config* cfg, moe_ctx** out);
  * Unless MOE_LOAD_SKIP_VALIDATE is set, the scale bytes are scanned on the
  * device for the NaN encoding 0xFF, synchronously on the legacy default
  * stream; MOE_ERR_BAD_WEIGHTS if any is found. May be called again to point
- * the context at other weights. */
+ * the context at other weights. A part of an intra-expert split
+ * (shard_count > 1) copies its rows of W13 and its columns of W2 (and the
+ * whole router), so the call needs MOE_LOAD_COPY_REPACK (INVALID_ARG
+ * otherwise) and the copy is about 1/G of the layer. */
 moe_status moe_load_experts(moe_ctx* ctx, const float* router_w,
                             const uint8_t* w13_codes, const uint8_t* w13_scales,
                             const uint8_t* w2_codes, const uint8_t* w2_scales,
@@ -202,7 +225,9 @@ moe_status moe_load_experts(moe_ctx* ctx, const float* router_w,
  * default stream), asynchronous, allocation-free and capturable into a CUDA
  * graph.
  *   x_bf16  [M][H] bf16 device, read only
- *   y_bf16  [M][H] bf16 device, written (must not alias x)
+ *   y_bf16  [M][H] bf16 device, written (must not alias x); for a part of
+ *           an intra-expert split, [M][H] fp32: the part's P_g before the
+ *           bf16 round
  *   M       0..max_tokens; M == 0 returns MOE_OK and enqueues nothing
  * Optional device outputs (NULL to skip):
  *   topk_ids [M][top_k] int32, highest logit first
@@ -214,6 +239,15 @@ moe_status moe_load_experts(moe_ctx* ctx, const float* router_w,
 moe_status moe_decode(moe_ctx* ctx, const void* x_bf16, int32_t M, void* y_bf16,
                       void* stream, int32_t* topk_ids, float* topk_w, uint8_t* xq,
                       float* xscale, void* xnorm_bf16);
+
+/* y_bf16[i] = bf16(y_f32[i]), round to nearest even, for i < n: the last
+ * step of an intra-expert split, after the parts' fp32 sums have been added
+ * (an all-reduce, in place or not). Device pointers, y_f32 4-byte and y_bf16
+ * 2-byte aligned, not overlapping; asynchronous on `stream` (NULL: the
+ * legacy default stream) on the current device. n == 0 does nothing.
+ * INVALID_ARG on a NULL or misaligned pointer, a negative n or overlap; CUDA
+ * if the launch fails. */
+moe_status moe_round_bf16(const float* y_f32, void* y_bf16, int64_t n, void* stream);
 
 /* Synchronise `stream`, then read and clear the context's device status word.
  * Returns MOE_ERR_TIMEOUT if a device-side wait gave up since the last call,
@@ -273,7 +307,7 @@ moe_status moe_debug_set_trace(moe_ctx* ctx, unsigned long long* trace);
  * step (the MOE_FLAG_SPLIT_KERNELS path). There is no context. The layer's
  * shapes come from cfg (max_tokens and device are ignored; of the flags,
  * MOE_FLAG_SHARED_EXPERT, MOE_FLAG_PRE_RMSNORM and MOE_FLAG_FP8_INTERMEDIATE
- * return MOE_ERR_UNSUPPORTED
+ * return MOE_ERR_UNSUPPORTED, as does shard_count > 1
  * and MOE_FLAG_SPLIT_KERNELS is ignored), and the
  * weights, x and y are passed in directly with the layouts, alignment and
  * optional outputs of moe_load_experts and moe_decode. The scale bytes are not

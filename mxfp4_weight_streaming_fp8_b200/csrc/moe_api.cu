@@ -51,6 +51,22 @@ moe_status validate_config(const moe_config& c) {
   return MOE_OK;
 }
 
+// Intra-expert split (shard_count = G > 1): part g computes gate/up rows
+// [g*I/G, (g+1)*I/G) and the same columns of the down projection, i.e. the
+// step of a layer of width I/G whose A8 sum stays in fp32. Gives the part's
+// config (inter = I/G, shard_count normalised to >= 1) after checking the
+// split's own rules; the whole layer's config is checked by validate_config.
+moe_status shard_config(const moe_config& c, moe_config* part) {
+  const int G = c.shard_count == 0 ? 1 : c.shard_count;
+  if (G < 1 || G > 128 || c.shard_index < 0 || c.shard_index >= G) return MOE_ERR_INVALID_ARG;
+  if (c.inter % (32 * G)) return MOE_ERR_INVALID_ARG;  // whole E8M0 blocks of W2 per part
+  if (G > 1 && (c.flags & MOE_FLAG_FP8_INTERMEDIATE)) return MOE_ERR_UNSUPPORTED;
+  *part = c;
+  part->inter = c.inter / G;
+  part->shard_count = G;
+  return MOE_OK;
+}
+
 // Union entries and (token, slot) pairs a call can have; a shared expert adds
 // one entry holding one pair per token.
 void union_bounds(const moe_config& c, size_t* np, size_t* umax) {
@@ -372,6 +388,33 @@ __global__ void k_repack_w2(const uint8_t* w2c, const uint8_t* w2s, int E, int H
 
 }  // namespace
 
+namespace {
+
+// dst[r * dp + j] = src[r * sp + j] for j < width, r < rows (bytes).
+__global__ void k_copy_rows(const uint8_t* src, size_t sp, uint8_t* dst, size_t dp, size_t width, size_t rows) {
+  const size_t n = width * rows, stride = (size_t)gridDim.x * blockDim.x;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += stride) {
+    const size_t r = i / width, j = i - r * width;
+    dst[r * dp + j] = src[r * sp + j];
+  }
+}
+
+bool copy_rows(const uint8_t* src, size_t sp, uint8_t* dst, size_t dp, size_t width, size_t rows) {
+  if (width == 0 || rows == 0) return true;
+  const size_t blocks = (width * rows + 255) / 256;
+  k_copy_rows<<<(unsigned)(blocks < 8192 ? blocks : 8192), 256>>>(src, sp, dst, dp, width, rows);
+  return cudaGetLastError() == cudaSuccess;
+}
+
+// The one bf16 round of an intra-expert split, after the parts are added.
+__global__ void k_round_bf16(const float* y32, __nv_bfloat16* y, int64_t n) {
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += stride)
+    y[i] = __float2bfloat16_rn(y32[i]);
+}
+
+}  // namespace
+
 struct moe_ctx {
   moe_config cfg{};
   int dev = 0;
@@ -402,6 +445,7 @@ struct moe_ctx {
   moe::TcWs tws{};
   moe::TcMaps maps{};  // encoded at load, passed by value at every launch
   void* owned = nullptr;  // MOE_LOAD_COPY_REPACK: the context's copy of the weights
+  int inter_full = 0;     // I of the whole layer (cfg.inter is this part's I/G)
 };
 
 extern "C" {
@@ -422,9 +466,12 @@ const char* moe_status_string(moe_status s) {
 
 moe_status moe_create(const moe_config* cfg, moe_ctx** out) {
   if (!cfg || !out) return MOE_ERR_INVALID_ARG;
-  const moe_config c = *cfg;
-  const moe_status v = validate_config(c);
+  moe_status v = validate_config(*cfg);
   if (v != MOE_OK) return v;
+  moe_config part{};
+  v = shard_config(*cfg, &part);
+  if (v != MOE_OK) return v;
+  const moe_config c = part;  // from here on, the layer this context computes
   int ndev = 0;
   if (cudaGetDeviceCount(&ndev) != cudaSuccess) return MOE_ERR_CUDA;
   if (c.device < 0 || c.device >= ndev) return MOE_ERR_INVALID_ARG;
@@ -437,6 +484,7 @@ moe_status moe_create(const moe_config* cfg, moe_ctx** out) {
   moe_ctx* ctx = new (std::nothrow) moe_ctx();
   if (!ctx) return MOE_ERR_OOM;
   ctx->cfg = c;
+  ctx->inter_full = cfg->inter;
   ctx->dev = c.device;
   ctx->sm_count = prop.multiProcessorCount;
   ctx->variant = (c.flags & MOE_FLAG_SPLIT_KERNELS) ? kSplit : kFused;
@@ -594,11 +642,15 @@ moe_status moe_load_experts(moe_ctx* ctx, const float* router_w, const uint8_t* 
   if (!aligned16(router_w) || !aligned16(w13_codes) || !aligned16(w13_scales) || !aligned16(w2_codes) ||
       !aligned16(w2_scales))
     return MOE_ERR_INVALID_ARG;
+  const moe_config& c = ctx->cfg;
+  const bool part = c.shard_count > 1;
+  if (part && !(load_flags & MOE_LOAD_COPY_REPACK)) return MOE_ERR_INVALID_ARG;
   DeviceGuard guard(ctx->dev);
   if (!guard.ok) return MOE_ERR_CUDA;
-  const moe_config& c = ctx->cfg;
   if (!(load_flags & MOE_LOAD_SKIP_VALIDATE)) {
-    const size_t E = c.num_experts + ((c.flags & MOE_FLAG_SHARED_EXPERT) ? 1 : 0), H = c.hidden, I = c.inter;
+    // the caller's arrays: the whole layer's, also for a part of a split
+    const size_t E = c.num_experts + ((c.flags & MOE_FLAG_SHARED_EXPERT) ? 1 : 0), H = c.hidden,
+                 I = ctx->inter_full;
     unsigned* bad = ctx->ws.ctrl + 4;
     if (cudaMemset(bad, 0, sizeof(unsigned)) != cudaSuccess) return MOE_ERR_CUDA;
     moe::k_scan_scales<<<ctx->sm_count * 4, 256>>>(w13_scales, E * 2 * I * (H / 32), bad);
@@ -634,18 +686,41 @@ moe_status moe_load_experts(moe_ctx* ctx, const float* router_w, const uint8_t* 
     uint8_t* w13s = w13 + b_13;
     uint8_t* w2 = w13s + b_13s;
     uint8_t* w2s = w2 + b_2;
-    bool okc = cudaMemcpy(wr, router_w, (size_t)c.num_experts * H * 4, cudaMemcpyDeviceToDevice) == cudaSuccess &&
-               cudaMemcpy(w13s, w13_scales, Eall * 2 * I * (H / 32), cudaMemcpyDeviceToDevice) == cudaSuccess &&
-               cudaMemcpy(w2, w2_codes, Eall * H * (I / 2), cudaMemcpyDeviceToDevice) == cudaSuccess &&
-               cudaMemcpy(w2s, w2_scales, Eall * H * (I / 32), cudaMemcpyDeviceToDevice) == cudaSuccess;
+    bool okc = cudaMemcpy(wr, router_w, (size_t)c.num_experts * H * 4, cudaMemcpyDeviceToDevice) == cudaSuccess;
+    void* w13_part = nullptr;  // a part's gate/up codes before the tensor-core re-tiling
+    if (okc && part) {
+      // this part's rows of W13 (gate rows g*I.., up rows I_full + g*I..) and
+      // columns of W2, from the whole layer's arrays
+      const size_t IF = ctx->inter_full, g = c.shard_index;
+      uint8_t* d13 = w13;
+      if (ctx->variant == kTc) {
+        okc = cudaMalloc(&w13_part, b_13) == cudaSuccess;
+        d13 = static_cast<uint8_t*>(w13_part);
+      }
+      const size_t rc = H / 2, rs = H / 32;  // bytes per W13 row: codes, scales
+      for (int half = 0; half < 2 && okc; ++half) {
+        const size_t src_row = half * IF + g * I, dst_row = half * I;
+        okc = copy_rows(w13_codes + src_row * rc, 2 * IF * rc, d13 + dst_row * rc, 2 * I * rc, I * rc, Eall) &&
+              copy_rows(w13_scales + src_row * rs, 2 * IF * rs, w13s + dst_row * rs, 2 * I * rs, I * rs, Eall);
+      }
+      okc = okc && copy_rows(w2_codes + g * (I / 2), IF / 2, w2, I / 2, I / 2, Eall * H) &&
+            copy_rows(w2_scales + g * (I / 32), IF / 32, w2s, I / 32, I / 32, Eall * H) &&
+            cudaDeviceSynchronize() == cudaSuccess;
+      if (okc && ctx->variant == kTc) w13_codes = static_cast<const uint8_t*>(w13_part);
+    } else if (okc) {
+      okc = cudaMemcpy(w13s, w13_scales, Eall * 2 * I * (H / 32), cudaMemcpyDeviceToDevice) == cudaSuccess &&
+            cudaMemcpy(w2, w2_codes, Eall * H * (I / 2), cudaMemcpyDeviceToDevice) == cudaSuccess &&
+            cudaMemcpy(w2s, w2_scales, Eall * H * (I / 32), cudaMemcpyDeviceToDevice) == cudaSuccess;
+    }
     if (okc && ctx->variant == kTc) {
       moe::k_repack_w13<<<ctx->sm_count * 8, 256>>>(w13_codes, w13, (int)Eall, (int)H, (int)I);
       okc = cudaGetLastError() == cudaSuccess && cudaDeviceSynchronize() == cudaSuccess;
       ctx->tws.repacked = 1;
-    } else if (okc) {
+    } else if (okc && !part) {
       okc = cudaMemcpy(w13, w13_codes, Eall * 2 * I * (H / 2), cudaMemcpyDeviceToDevice) == cudaSuccess &&
             cudaDeviceSynchronize() == cudaSuccess;
     }
+    if (w13_part) cudaFree(w13_part);
     if (!okc) {
       cudaGetLastError();
       cudaFree(ctx->owned);
@@ -703,10 +778,11 @@ moe_status moe_decode(moe_ctx* ctx, const void* x_bf16, int32_t M, void* y_bf16,
   if (M < 0 || M > c.max_tokens) return MOE_ERR_INVALID_ARG;
   if (M == 0) return MOE_OK;
   if (!x_bf16 || !y_bf16 || !aligned16(x_bf16) || !aligned16(y_bf16)) return MOE_ERR_INVALID_ARG;
-  const size_t xbytes = (size_t)M * c.hidden * 2;
+  const bool part = c.shard_count > 1;  // y is the part's fp32 sum
+  const size_t xbytes = (size_t)M * c.hidden * 2, ybytes = xbytes * (part ? 2 : 1);
   const char* xb = static_cast<const char*>(x_bf16);
   const char* yb = static_cast<const char*>(y_bf16);
-  if (xb < yb + xbytes && yb < xb + xbytes) return MOE_ERR_INVALID_ARG;  // aliasing
+  if (xb < yb + ybytes && yb < xb + xbytes) return MOE_ERR_INVALID_ARG;  // aliasing
   if ((xq && !aligned16(xq)) || (topk_ids && (reinterpret_cast<uintptr_t>(topk_ids) & 3)) ||
       (topk_w && (reinterpret_cast<uintptr_t>(topk_w) & 3)) ||
       (xscale && (reinterpret_cast<uintptr_t>(xscale) & 3)) || (xnorm_bf16 && !aligned16(xnorm_bf16)))
@@ -722,7 +798,8 @@ moe_status moe_decode(moe_ctx* ctx, const void* x_bf16, int32_t M, void* y_bf16,
   p.K = c.top_k;
   p.M = M;
   p.x = static_cast<const __nv_bfloat16*>(x_bf16);
-  p.y = static_cast<__nv_bfloat16*>(y_bf16);
+  p.y = part ? nullptr : static_cast<__nv_bfloat16*>(y_bf16);
+  p.y32 = part ? static_cast<float*>(y_bf16) : nullptr;
   p.wr = ctx->wr;
   p.w13c = ctx->w13c;
   p.w13s = ctx->w13s;
@@ -787,13 +864,17 @@ moe_status moe_sync_status(moe_ctx* ctx, void* stream) {
 
 moe_status moe_plan_query(const moe_config* cfg, int32_t sm_count, size_t smem_limit, char* buf, size_t len) {
   if (!cfg || !buf || len == 0 || sm_count < 1) return MOE_ERR_INVALID_ARG;
-  const moe_status v = validate_config(*cfg);
+  moe_status v = validate_config(*cfg);
   if (v != MOE_OK) return v;
+  moe_config part{};
+  v = shard_config(*cfg, &part);
+  if (v != MOE_OK) return v;
+  cfg = &part;  // the plan of this part's layer (the whole layer when unsplit)
   moe::FusedPlan pl{};
   const bool ok = make_plan(*cfg, sm_count, smem_limit, &pl);
   moe::TcPlan tp{};
   const bool tok = make_tc_plan(*cfg, sm_count, smem_limit, &tp);
-  const bool tc = tok && !(cfg->flags & (MOE_FLAG_SPLIT_KERNELS | MOE_FLAG_CUDA_CORES)) &&
+  const bool tc = tok && !(cfg->flags & (MOE_FLAG_SPLIT_KERNELS | MOE_FLAG_CUDA_CORES | MOE_FLAG_SPLITK_DOWN)) &&
                   ((cfg->flags & MOE_FLAG_TENSOR_CORES) || cfg->max_tokens >= MOE_TC_MIN_TOKENS);
   const int n = snprintf(buf, len,
                          "{\"ok\": %s, \"variant\": \"%s\", \"grid\": %d, \"threads\": %d, \"smem\": %d, "
@@ -880,6 +961,25 @@ moe_status moe_query(const moe_ctx* ctx, char* buf, size_t len) {
                  c.top_k, c.max_tokens);
   }
   if (n < 0 || (size_t)n >= len) return MOE_ERR_INVALID_ARG;
+  // the split: "inter" above is this part's width
+  const int m = snprintf(buf + n - 1, len - (n - 1), ", \"shard\": [%d, %d], \"inter_full\": %d, \"y\": \"%s\"}",
+                         c.shard_index, c.shard_count, ctx->inter_full, c.shard_count > 1 ? "f32" : "bf16");
+  if (m < 0 || (size_t)m >= len - (n - 1)) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+moe_status moe_round_bf16(const float* y_f32, void* y_bf16, int64_t n, void* stream) {
+  if (n < 0 || !y_f32 || !y_bf16 || (reinterpret_cast<uintptr_t>(y_f32) & 3) ||
+      (reinterpret_cast<uintptr_t>(y_bf16) & 1))
+    return MOE_ERR_INVALID_ARG;
+  const char* a = reinterpret_cast<const char*>(y_f32);
+  const char* b = static_cast<const char*>(y_bf16);
+  if (a < b + 2 * n && b < a + 4 * n) return MOE_ERR_INVALID_ARG;
+  if (n == 0) return MOE_OK;
+  const int64_t blocks = (n + 255) / 256;
+  k_round_bf16<<<(unsigned)(blocks < 4096 ? blocks : 4096), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      y_f32, static_cast<__nv_bfloat16*>(y_bf16), n);
+  if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
   return MOE_OK;
 }
 

@@ -62,7 +62,18 @@ struct Params {
   int pre_rmsnorm;       // x <- bf16(x * rsqrt(mean(x^2) + eps)) before A1/A2
   unsigned long long* trace;  // test hook: per-CTA phase timestamps (globaltimer), or null
   __nv_bfloat16* out_xn; // optional [M][H] normalised input
+  float* y32;            // one part of an intra-expert split: fp32 [M][H] partial sums instead of y
 };
+
+// A8's store of output element i: bf16 y, or, for one part of an
+// intra-expert split, the fp32 slot-order sum itself (the parts' sums are
+// added before the one bf16 round).
+__device__ __forceinline__ void store_y(const Params& p, size_t i, float v) {
+  if (p.y32)
+    p.y32[i] = v;
+  else
+    p.y[i] = __float2bfloat16_rn(v);
+}
 
 // Test hook: lane 0 of the calling warp stores the global timer into stamp
 // `slot` of this CTA's row of the trace array (kTraceSlots stamps per CTA).

@@ -39,7 +39,8 @@
 //     drain an in-order queue of down items (A7). The first down item of u
 //     waits on the counter and stages h once into shared memory for the CTA;
 //     the other items of u wait for that.
-//  6. Each CTA combines its output rows in slot order (A8) and writes bf16 y.
+//  6. Each CTA combines its output rows in slot order (A8) and writes bf16 y
+//     (fp32 partial sums for one part of an intra-expert split).
 //
 // Every wait is bounded: on timeout the kernel sets the status word and goes
 // on (with garbage results) instead of hanging. moe_sync_status reports it.
@@ -1836,18 +1837,18 @@ __global__ void __launch_bounds__(kFusedThreads, 1) k_fused(Params p, FusedWs fw
       if (ct < nout) {
         float acc = 0.f;
         for (int j2 = 0; j2 < tpo; ++j2) acc += red[ct * tpo + j2];
-        p.y[(size_t)(ct / nrd) * H + r0 + ct % nrd] = __float2bfloat16_rn(acc);
+        store_y(p, (size_t)(ct / nrd) * H + r0 + ct % nrd, acc);
       }
     }
     if (b == 0 && ct == 0) st_relaxed_u32(fw.epoch, epoch);
   } else {
-  // ---- A8: combine in slot order, bf16 out
+  // ---- A8: combine in slot order, bf16 out (fp32 for one part of a split)
   for (int i = ct; i < M * nrd; i += kConsumers * 32) {
     const int m = i / nrd, rl = i % nrd;
     float acc = 0.f;
     for (int s = 0; s < K; ++s) acc = fmaf(s_w[m * K + s], dsm[(size_t)s_ppos[m * K + s] * pl.rpc_max + rl], acc);
     if constexpr (kShared) acc += dsm[(size_t)m * pl.rpc_max + rl];  // shared expert, weight 1
-    p.y[(size_t)m * H + r0 + rl] = __float2bfloat16_rn(acc);
+    store_y(p, (size_t)m * H + r0 + rl, acc);
   }
   if (b == 0 && ct == 0) {
     // keep every entry's counter at epoch * G for the next launch

@@ -129,7 +129,7 @@ static __global__ void __launch_bounds__(kThreads) k_down(Params p) {
     if (lane < p.M) {
       float y = 0.f;
       for (int s = 0; s < K; ++s) y = fmaf(__ldcg(p.ws.wts + lane * K + s), dslot[warp][lane * K + s], y);
-      p.y[(size_t)lane * H + r] = __float2bfloat16_rn(y);
+      store_y(p, (size_t)lane * H + r, y);
     }
     __syncwarp();
   }

@@ -111,6 +111,7 @@ moe_status moe_decode_static(const moe_config* cfg, const float* router_w, const
   if (M < 0 || M > moe::kMaxTokens) return MOE_ERR_INVALID_ARG;
   if (c.flags & (MOE_FLAG_SHARED_EXPERT | MOE_FLAG_PRE_RMSNORM | MOE_FLAG_FP8_INTERMEDIATE | MOE_FLAG_SPLITK_DOWN))
     return MOE_ERR_UNSUPPORTED;
+  if (c.shard_count > 1) return MOE_ERR_UNSUPPORTED;  // no context to hold a part's copy
   if (M == 0) return MOE_OK;
   if (!router_w || !w13_codes || !w13_scales || !w2_codes || !w2_scales || !x_bf16 || !y_bf16)
     return MOE_ERR_INVALID_ARG;

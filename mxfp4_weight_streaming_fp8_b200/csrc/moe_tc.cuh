@@ -45,7 +45,8 @@
 //     entry polls the entry's counter (acquire) until every tile covering it
 //     has arrived, then stages h once as f16 (rescaled by a power of two per
 //     pair).
-//  5. Each CTA combines its rows in slot order and writes bf16 y.
+//  5. Each CTA combines its rows in slot order and writes bf16 y (fp32
+//     partial sums for one part of an intra-expert split).
 // Every wait is bounded: a wait that runs out sets the status word and the
 // kernel finishes (with garbage output) instead of hanging.
 #pragma once
@@ -1434,14 +1435,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc(Params p, TcWs tw, TcPlan 
     }
     const bool all_ok = __syncthreads_and(ok ? 1 : 0) != 0;
     tc_trace(p, 11);
-    // ---- A8: combine in slot order, bf16 out
+    // ---- A8: combine in slot order, bf16 out (fp32 for one part of a split)
     for (int i = tid; i < M * nrd && all_ok; i += kTcThreads) {
       const int m = i / nrd, r = r0 + i % nrd;
       float acc = 0.f;
       for (int s = 0; s < K; ++s)
         acc = fmaf(s_w[m * K + s], __ldcg(tw.ypart + (size_t)s_ppos[m * K + s] * H + r), acc);
       if constexpr (kShared) acc += __ldcg(tw.ypart + (size_t)m * H + r);
-      p.y[(size_t)m * H + r] = __float2bfloat16_rn(acc);
+      store_y(p, (size_t)m * H + r, acc);
     }
   } else {
     // ---------------- down (CUDA cores): every warp once its role is done.
@@ -1489,13 +1490,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc(Params p, TcWs tw, TcPlan 
       tc_trace(p, 10);
       __syncthreads();
       tc_trace(p, 11);
-      // ---- A8: combine in slot order, bf16 out
+      // ---- A8: combine in slot order, bf16 out (fp32 for one part of a split)
       for (int i = tid; i < M * nrd; i += kTcThreads) {
         const int m = i / nrd, rl = i % nrd;
         float acc = 0.f;
         for (int s = 0; s < K; ++s) acc = fmaf(s_w[m * K + s], dsm[(size_t)s_ppos[m * K + s] * pl.rpc_max + rl], acc);
         if constexpr (kShared) acc += dsm[(size_t)m * pl.rpc_max + rl];
-        p.y[(size_t)m * H + r0 + rl] = __float2bfloat16_rn(acc);
+        store_y(p, (size_t)m * H + r0 + rl, acc);
       }
     }
   

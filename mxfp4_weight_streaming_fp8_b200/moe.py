@@ -43,7 +43,7 @@ class MoEError(RuntimeError):
 class moe_config(ctypes.Structure):
     _fields_ = [("hidden", ctypes.c_int32), ("inter", ctypes.c_int32), ("num_experts", ctypes.c_int32),
                 ("top_k", ctypes.c_int32), ("max_tokens", ctypes.c_int32), ("flags", ctypes.c_uint32),
-                ("device", ctypes.c_int32)]
+                ("device", ctypes.c_int32), ("shard_index", ctypes.c_int32), ("shard_count", ctypes.c_int32)]
 
 
 _lib = None
@@ -75,6 +75,8 @@ def lib() -> ctypes.CDLL:
         L.moe_plan_query.argtypes = [ctypes.POINTER(moe_config), ctypes.c_int32, ctypes.c_size_t,
                                      ctypes.c_char_p, ctypes.c_size_t]
         L.moe_plan_query.restype = ctypes.c_int
+        L.moe_round_bf16.argtypes = [_vp, _vp, ctypes.c_int64, _vp]
+        L.moe_round_bf16.restype = ctypes.c_int
         L.moe_decode_static.argtypes = [ctypes.POINTER(moe_config)] + [_vp] * 6 + [ctypes.c_int32] + [_vp] * 6
         L.moe_decode_static.restype = ctypes.c_int
         L.moe_debug_set_wait.argtypes = [_vp, ctypes.c_longlong, ctypes.c_int]
@@ -111,9 +113,11 @@ def _stream_handle(stream):
     return ctypes.c_void_p(stream.cuda_stream)
 
 
-def plan_query(hidden, inter, num_experts, top_k, max_tokens, flags=0, sm_count=148, smem_limit=232448):
-    """(status, plan dict) of the persistent kernel for a shape; host only."""
-    cfg = moe_config(hidden, inter, num_experts, top_k, max_tokens, flags, 0)
+def plan_query(hidden, inter, num_experts, top_k, max_tokens, flags=0, sm_count=148, smem_limit=232448,
+               shard=(0, 1)):
+    """(status, plan dict) of the persistent kernel for a shape (for part
+    shard[0] of an intra-expert split over shard[1] GPUs); host only."""
+    cfg = moe_config(hidden, inter, num_experts, top_k, max_tokens, flags, 0, shard[0], shard[1])
     buf = ctypes.create_string_buffer(4096)
     st = lib().moe_plan_query(ctypes.byref(cfg), sm_count, smem_limit, buf, len(buf))
     return st, (json.loads(buf.value.decode()) if buf.value else None)
@@ -129,6 +133,36 @@ def decode_static(hidden, inter, num_experts, top_k, router_w, w13_codes, w13_sc
                                    _stream_handle(stream), _ptr(topk_ids), _ptr(topk_w), _ptr(xq), _ptr(xscale))
 
 
+def round_bf16(y32, y=None, stream=None):
+    """moe_round_bf16: bf16 y (same shape) from the fp32 sum of an
+    intra-expert split's parts."""
+    import torch
+    if y is None:
+        y = torch.empty(y32.shape, dtype=torch.bfloat16, device=y32.device)
+    if y32.dtype != torch.float32 or y.dtype != torch.bfloat16 or y.numel() != y32.numel():
+        raise ValueError("round_bf16 takes fp32 in and bf16 out of the same size")
+    st = lib().moe_round_bf16(_ptr(y32), _ptr(y), y32.numel(), _stream_handle(stream))
+    if st != MOE_OK:
+        raise MoEError(st, "moe_round_bf16")
+    return y
+
+
+def decode_split(layer, x, group=None, y32=None, y=None, stream=None):
+    """One step of an intra-expert split, on this rank's part `layer` (a
+    MoELayer created with shard=(rank, world)): the part's fp32 sums
+    (moe_decode), their sum over the ranks of `group` (one all-reduce through
+    torch.distributed, NCCL on GPUs), and the bf16 round (moe_round_bf16).
+    Every rank of the group must call it with the same x."""
+    import torch
+    import torch.distributed as dist
+    if stream is not None:
+        with torch.cuda.stream(stream):
+            return decode_split(layer, x, group, y32, y)
+    y32 = layer.decode(x, y32)
+    dist.all_reduce(y32, op=dist.ReduceOp.SUM, group=group)
+    return round_bf16(y32, y)
+
+
 def status_string(s: int) -> str:
     return lib().moe_status_string(int(s)).decode()
 
@@ -137,8 +171,11 @@ class MoELayer:
     """One MoE layer's context: moe_create / moe_load_experts / moe_decode."""
 
     def __init__(self, hidden: int, inter: int, num_experts: int, top_k: int, max_tokens: int,
-                 flags: int = 0, device: int = 0):
-        self.cfg = moe_config(hidden, inter, num_experts, top_k, max_tokens, flags, device)
+                 flags: int = 0, device: int = 0, shard=(0, 1)):
+        """shard=(g, G): part g of an intra-expert split over G GPUs; decode
+        then returns the part's fp32 sums (see decode_split)."""
+        self.cfg = moe_config(hidden, inter, num_experts, top_k, max_tokens, flags, device, shard[0], shard[1])
+        self.shard = (int(shard[0]), max(1, int(shard[1])))
         self.hidden, self.inter, self.num_experts, self.top_k = hidden, inter, num_experts, top_k
         self.max_tokens = max_tokens
         self.device = device
@@ -151,7 +188,9 @@ class MoELayer:
     def load_experts(self, router_w, w13_codes, w13_scales, w2_codes, w2_scales, validate: bool = True,
                      repack: bool = False):
         """Borrow device tensors (kept referenced here so they outlive the
-        context), or with repack=True let the context copy (and re-tile) them."""
+        context), or with repack=True let the context copy (and re-tile) them.
+        A part of an intra-expert split always copies its slice."""
+        repack = repack or self.shard[1] > 1
         flags = (0 if validate else MOE_LOAD_SKIP_VALIDATE) | (MOE_LOAD_COPY_REPACK if repack else 0)
         st = lib().moe_load_experts(self._ctx, _ptr(router_w), _ptr(w13_codes), _ptr(w13_scales),
                                     _ptr(w2_codes), _ptr(w2_scales), flags)
@@ -167,11 +206,12 @@ class MoELayer:
 
     def decode(self, x, y=None, stream=None, routing: bool = False):
         """x: bf16 [M, H] on the device. Returns y, or with routing=True
-        (y, topk_ids, topk_w, xq, xscale[, xnorm when the context normalises])."""
+        (y, topk_ids, topk_w, xq, xscale[, xnorm when the context normalises]).
+        For a part of an intra-expert split y is fp32: the part's sums."""
         import torch
         M = x.shape[0]
         if y is None:
-            y = torch.empty_like(x)
+            y = torch.empty(x.shape, dtype=torch.float32 if self.shard[1] > 1 else x.dtype, device=x.device)
         extra = [None] * 4
         if routing:
             dev = x.device

@@ -67,6 +67,28 @@ class Layer:
             return oracle.moe_decode_shared(xb, self.wr, *per, sh, self.H, self.I, self.E, self.K)
         return oracle.moe_decode(xb, self.wr, *per, self.H, self.I, self.E, self.K)
 
+    def oracle_part(self, g, G, tokens=None):
+        """Oracle outputs of part g of an intra-expert split over G: the
+        layer of width I/G made of each expert's part (part_arrays); its y64
+        is the part's fp64 sum before any rounding."""
+        assert not self.a8
+        xb = bits(self.x)
+        if tokens is not None:
+            xb = xb[list(tokens)]
+        logits = oracle.router_logits(xb, self.wr)
+        ids, _ = oracle.topk(logits, self.K)
+        per = self.expert_slices(ids)
+        for e in range(self.E):
+            if per[0][e] is not None:
+                parts = part_arrays(*(per[t][e] for t in range(4)), self.I, g, G)
+                for t in range(4):
+                    per[t][e] = parts[t]
+        Ip = self.I // G
+        if self.shared:
+            sh = part_arrays(*synth.expert_np(self.seed, self.layer, self.E, self.H, self.I), self.I, g, G)
+            return oracle.moe_decode_shared(xb, self.wr, *per, sh, self.H, Ip, self.E, self.K)
+        return oracle.moe_decode(xb, self.wr, *per, self.H, Ip, self.E, self.K)
+
     def make_ctx(self, flags=0, max_tokens=None):
         if self.shared:
             flags |= moe.MOE_FLAG_SHARED_EXPERT
@@ -87,6 +109,17 @@ class Layer:
         if len(out) > 5:
             res["xn"] = out[5]
         return res
+
+
+def part_arrays(w13c, w13s, w2c, w2s, I, g, G):
+    """Part g of G of one expert's arrays (the layouts of synth.expert_np):
+    gate rows [g*I/G, (g+1)*I/G), the up rows I + the same, and the same
+    columns of the down projection (codes two per byte, scales one per 32)."""
+    Ip = I // G
+    rows = np.r_[g * Ip:(g + 1) * Ip, I + g * Ip:I + (g + 1) * Ip]
+    return (np.ascontiguousarray(w13c[rows]), np.ascontiguousarray(w13s[rows]),
+            np.ascontiguousarray(w2c[:, g * Ip // 2:(g + 1) * Ip // 2]),
+            np.ascontiguousarray(w2s[:, g * Ip // 32:(g + 1) * Ip // 32]))
 
 
 def min_gap(logits: np.ndarray, k: int) -> float:

@@ -1,5 +1,7 @@
-"""Host-side multi-process logic of bench.py (replica timing reduced as the
-max over ranks, throughput summed over ranks) on CPU with gloo, world size 2."""
+"""Host-side multi-process logic on CPU with gloo, world size 2: bench.py's
+replica timing (max over ranks, throughput summed over ranks), and the
+intra-expert split's exchange (each rank's part of the layer, one all-reduce
+of the partial sums, one bf16 round) against the whole layer's oracle."""
 import os
 import socket
 
@@ -52,3 +54,42 @@ def test_single_rank_is_identity():
     import bench
     assert bench.max_over_ranks(3.5, 1) == 3.5
     assert bench.sum_over_ranks(3.5, 1) == 3.5
+
+
+def _split_worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+    import sys
+    here = os.path.dirname(os.path.abspath(__file__))
+    sys.path[:0] = [here, os.path.dirname(here)]
+    import numpy as np
+    import oracle
+    from cases import Layer
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    L = Layer(256, 128, 16, 4, 3, seed=9, device="cpu", shared=True)
+    part = torch.from_numpy(L.oracle_part(rank, world)["y64"].copy())
+    dist.all_reduce(part, op=dist.ReduceOp.SUM)
+    y = np.array([[oracle.bf16_round(v) for v in row] for row in part.numpy()], dtype=np.uint16)
+    whole = L.oracle()["y64"]
+    ref = np.array([[oracle.bf16_round(v) for v in row] for row in whole], dtype=np.uint16)
+    out[rank] = (bool(np.array_equal(y, ref)), float(np.max(np.abs(part.numpy() - whole))),
+                 float(np.abs(whole).max()))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_split_parts_all_reduced_over_two_ranks_match_the_layer():
+    ctx = mp.get_context("spawn")
+    mgr = ctx.Manager()
+    out = mgr.dict()
+    port = _free_port()
+    procs = [ctx.Process(target=_split_worker, args=(r, 2, port, out)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(180)
+        assert p.exitcode == 0
+    for r in range(2):
+        same, err, scale = out[r]
+        assert same
+        assert err <= 1e-12 * scale
