@@ -1,7 +1,9 @@
 """Host-side multi-process logic on CPU with gloo, world size 2: bench.py's
 replica timing (max over ranks, throughput summed over ranks), and the
 intra-expert split's exchange (each rank's part of the layer, one all-reduce
-of the partial sums, one bf16 round) against the whole layer's oracle."""
+of the partial sums, one bf16 round; in fp64 from the oracle's parts, and
+through the binding's moe.decode_split with fp32 parts) against the whole
+layer's oracle."""
 import os
 import socket
 
@@ -72,8 +74,24 @@ def _split_worker(rank, world, port, out):
     y = np.array([[oracle.bf16_round(v) for v in row] for row in part.numpy()], dtype=np.uint16)
     whole = L.oracle()["y64"]
     ref = np.array([[oracle.bf16_round(v) for v in row] for row in whole], dtype=np.uint16)
+    # the binding's own exchange step (moe.decode_split) with the part's
+    # kernel replaced by its oracle and the bf16 round done by torch (the
+    # ranks here have no GPU)
+    from mxfp4_weight_streaming_fp8_b200 import moe
+
+    class OraclePart:
+        def decode(self, x, y=None):
+            y.copy_(torch.from_numpy(L.oracle_part(rank, world)["y64"]).float())
+            return y
+
+    def round_bf16(y32, y=None, stream=None):
+        return y.copy_(y32.to(torch.bfloat16))
+
+    moe.round_bf16 = round_bf16
+    yb = moe.decode_split(OraclePart(), L.x, y32=torch.empty(L.M, L.H), y=torch.empty(L.M, L.H, dtype=torch.bfloat16))
+    ulps = np.abs(yb.view(torch.int16).numpy().astype(np.int32) - ref.view(np.int16).astype(np.int32))
     out[rank] = (bool(np.array_equal(y, ref)), float(np.max(np.abs(part.numpy() - whole))),
-                 float(np.abs(whole).max()))
+                 float(np.abs(whole).max()), int(ulps.max()))
     dist.barrier()
     dist.destroy_process_group()
 
@@ -90,6 +108,7 @@ def test_split_parts_all_reduced_over_two_ranks_match_the_layer():
         p.join(180)
         assert p.exitcode == 0
     for r in range(2):
-        same, err, scale = out[r]
+        same, err, scale, ulps = out[r]
         assert same
         assert err <= 1e-12 * scale
+        assert ulps <= 1  # fp32 parts added in fp32, then rounded
