@@ -168,7 +168,7 @@ __device__ __forceinline__ bool mbar_wait_ok(uint64_t* bar, unsigned parity, con
   return true;
 }
 
-// Warp-uniform form: lane 0 waits, every lane gets its verdict (warps that
+// Warp-uniform form: lane 0 waits, every lane gets the outcome (warps that
 // run .sync.aligned instructions after the wait must not diverge on it).
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, unsigned parity, const Params& p) {
   bool r = true;
@@ -278,7 +278,7 @@ __device__ __forceinline__ uint32_t sw128_offset(int r, int k, int groups) {
 }
 
 // Wait (one lane, acquire at CTA scope) until a shared-memory flag is set;
-// the warp gets one verdict.
+// the warp gets one outcome.
 // Down item: rows [a, a+cnt) of one entry's chunk for each of its pairs. Lane
 // l takes 32-element block l of the pair's h, read once from L2 (I <= 1024:
 // one block per lane); the pair's power-of-two rescale (kFp8H: its E4M3
@@ -948,7 +948,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc(Params p, TcWs tw, TcPlan 
   // accesses to them were the router-row and staged-x reads before the
   // activation codes' fence)
   if (!pl.lg_own) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-  // one verdict for the CTA: after a routing wait ran out, no role starts
+  // one outcome for the CTA: after a routing wait ran out, no role starts
   ok = __syncthreads_and(ok ? 1 : 0) != 0;
   const int U = s_int[0];
   // tensor-core down tiles, entry-major: entry u has ceil(pairs / kTcDownPairs)
