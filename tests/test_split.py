@@ -113,3 +113,14 @@ def test_round_bf16_argument_checks_without_gpu():
     # overlap: 4 floats at a, 4 bf16 starting 8 bytes into them
     assert L.moe_round_bf16(a, ctypes.c_void_p((1 << 20) + 8), 4, None) == INVALID_ARG
     assert L.moe_round_bf16(a, b, 0, None) == moe.MOE_OK  # nothing to do, no launch
+
+
+@pytest.mark.parametrize("G,MM,flags", [(2, 1, 0), (2, 4, 0), (2, 32, 0), (3, 4, 0), (6, 32, 0), (4, 1, 0),
+                                        (2, 32, moe.MOE_FLAG_SHARED_EXPERT), (2, 4, moe.MOE_FLAG_SPLITK_DOWN)])
+def test_a_part_is_planned_as_the_narrow_layer(G, MM, flags):
+    """Every part of the Ling layer gets exactly the launch plan of the layer
+    of width I/G (the kernels see only the narrow layer)."""
+    for g in range(G):
+        st, part = moe.plan_query(2560, 768, 256, 8, MM, flags=flags, shard=(g, G))
+        st2, narrow = moe.plan_query(2560, 768 // G, 256, 8, MM, flags=flags)
+        assert st == st2 and part == narrow
