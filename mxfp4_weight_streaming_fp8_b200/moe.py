@@ -200,7 +200,8 @@ class MoELayer:
 
     def decode_raw(self, x, M: int, y, stream=None, topk_ids=None, topk_w=None, xq=None, xscale=None,
                    xnorm=None) -> int:
-        """moe_decode with explicit buffers; returns the status code."""
+        """moe_decode with explicit buffers (y: bf16 [M][H], fp32 for a part of a
+        split; sizes are the caller's to get right); returns the status code."""
         return lib().moe_decode(self._ctx, _ptr(x), int(M), _ptr(y), _stream_handle(stream), _ptr(topk_ids),
                                 _ptr(topk_w), _ptr(xq), _ptr(xscale), _ptr(xnorm))
 
@@ -210,8 +211,11 @@ class MoELayer:
         For a part of an intra-expert split y is fp32: the part's sums."""
         import torch
         M = x.shape[0]
+        ydt = torch.float32 if self.shard[1] > 1 else torch.bfloat16
         if y is None:
-            y = torch.empty(x.shape, dtype=torch.float32 if self.shard[1] > 1 else x.dtype, device=x.device)
+            y = torch.empty(x.shape, dtype=ydt, device=x.device)
+        elif y.dtype != ydt or y.numel() < M * self.hidden or not y.is_contiguous():
+            raise ValueError(f"y must be a contiguous {ydt} tensor of at least {M} x {self.hidden} elements")
         extra = [None] * 4
         if routing:
             dev = x.device
