@@ -17,7 +17,8 @@ G = 148
 UNITS_MAX, ACC_COLS, SF_COL, DOWN_PAIRS, DOWN_ROWS = 16, 32, 64, 16, 9
 
 SHAPES = [(2560, 768, 256, 8), (256, 128, 16, 2), (512, 256, 40, 6), (384, 128, 12, 4), (128, 128, 8, 8),
-          (1024, 512, 64, 8), (2560, 768, 257, 8), (640, 384, 300, 3)]
+          (1024, 512, 64, 8), (2560, 768, 257, 8), (640, 384, 300, 3),
+          (2560, 384, 256, 8), (2560, 384, 257, 8), (2560, 256, 256, 8)]  # the Ling layer's parts (I/2, I/3)
 
 
 def sw128(r, k, groups):
