@@ -386,10 +386,6 @@ __global__ void k_repack_w2(const uint8_t* w2c, const uint8_t* w2s, int E, int H
   }
 }
 
-}  // namespace
-
-namespace {
-
 // dst[r * dp + j] = src[r * sp + j] for j < width, r < rows (bytes).
 __global__ void k_copy_rows(const uint8_t* src, size_t sp, uint8_t* dst, size_t dp, size_t width, size_t rows) {
   const size_t n = width * rows, stride = (size_t)gridDim.x * blockDim.x;
