@@ -12,12 +12,11 @@
 //     starts a TMA bulk copy of its slice of the router weights into shared
 //     memory. Router weights never depend on the previous kernel.
 //  2. Each CTA quantises all M tokens to E4M3 into shared memory (A1) and
-//     computes the logits of its router rows (A2). A grid-wide arrival
-//     counter (+G per launch) tells when all logits are in L2. The CTA whose
-//     arrival completes the count writes the launch epoch to 8 flag copies on
-//     separate L2 lines, and each CTA polls one copy from a single thread,
-//     with back-off.
-//  3. Every CTA gathers all the logits and, redundantly, computes top-k,
+//     computes the logits of its router rows (A2). Each logit goes to L2 as
+//     one 64-bit word holding the launch epoch next to the fp32 value, so
+//     the data is its own flag: there is no arrival counter.
+//  3. Every CTA reads all M x E logit words until each carries this launch's
+//     epoch (bounded, CTA-rotated order), and, redundantly, computes top-k,
 //     softmax and the expert union (A3, A4) in shared memory.
 //  4. The CTA streams its share of every union expert into two
 //     shared-memory rings with TMA bulk copies:
