@@ -1,5 +1,6 @@
-// moe_tc.cuh -- the decode step as one persistent kernel whose gate/up
-// projection runs on the tensor cores (tcgen05 block-scaled MMA).
+// moe_tc.cuh -- the decode step as one persistent kernel whose gate/up and
+// (from MOE_TC_DOWN_MMA_MIN_TOKENS tokens) down projections run on the
+// tensor cores (tcgen05 block-scaled MMA).
 //
 // The step streams the active experts' MXFP4 weights from HBM once (MarkTechPost,
 // "NVIDIA Shows 3 Ways to Speed Up MoE Inference on DGX Spark", section "Why is
@@ -38,13 +39,25 @@
 //     (tcgen05.ld), apply the per-token scale and SwiGLU, and store h of each
 //     (token, slot) pair routed to the unit's expert to L2.
 //     After its stores each epilogue warp adds one (release, GPU scope) to a
-//     counter of every entry the tile touches.
-//  4. Down (CUDA cores): each CTA owns output rows [H*b/G, H*(b+1)/G) of every
-//     union expert, streamed by warp 2 into a ring of 1-D TMA copies. The
-//     consumer warps take down items in entry order; the first item of an
-//     entry polls the entry's counter (acquire) until every tile covering it
-//     has arrived, then stages h once as f16 (rescaled by a power of two per
-//     pair).
+//     counter of every entry the tile touches; one gatekeeper thread per CTA
+//     polls those counters in entry order and raises a shared-memory flag
+//     per entry once its h is complete on every CTA.
+//  4. Down on the tensor cores (the default from MOE_TC_DOWN_MMA_MIN_TOKENS
+//     tokens of max_tokens): down tiles (entry, group of up to 16 pairs, 128
+//     output rows) follow each CTA's gate/up tiles in the same pipeline. Warp
+//     0 loads the tile's W2 codes (a 2-D tensor map, 128 rows x 128-element
+//     K-chunks) and scales; warps 8..15 build the B operand once the entry's
+//     flag is up: per pair an fp32 scale and the E4M3 codes of h/scale and of
+//     16x its rounding residual, so the MMA sums hi + lo/16 (within 2^-8 of
+//     h). The epilogue applies the pair scales and writes each pair's 128
+//     outputs to L2; every CTA then arrives on a grid count (by launch
+//     parity), waits for all CTAs, and combines its rows from the per-pair
+//     outputs.
+//     Down on CUDA cores (below that, or forced): each CTA owns output rows
+//     [H*b/G, H*(b+1)/G) of every union expert, streamed by warp 2 into a
+//     ring of 1-D TMA copies; consumer warps take down items in entry order,
+//     each waiting for its entry's flag, and stage h once as f16 (rescaled by
+//     a power of two per pair).
 //  5. Each CTA combines its rows in slot order and writes bf16 y (fp32
 //     partial sums for one part of an intra-expert split).
 // Every wait is bounded: a wait that runs out sets the status word and the
