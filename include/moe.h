@@ -92,9 +92,11 @@ typedef enum {
                                        multiplies its own h slice by a K-major
                                        copy of W2 that moe_load_experts makes;
                                        partial outputs summed in a fixed
-                                       order). max_tokens <= 4; not with
-                                       MOE_FLAG_FP8_INTERMEDIATE or
-                                       MOE_FLAG_SPLIT_KERNELS */
+                                       order). A CUDA-core kernel option:
+                                       max_tokens <= 4; not with
+                                       MOE_FLAG_FP8_INTERMEDIATE,
+                                       MOE_FLAG_SPLIT_KERNELS or
+                                       MOE_FLAG_TENSOR_CORES */
 #define MOE_FLAG_FP8_INTERMEDIATE 0x8u /* FP8 input to the down projection too
                                        (W4A8 on the same page, section "Why
                                        is MoE decoding on DGX Spark
@@ -117,19 +119,25 @@ typedef enum {
                                        (E2M1 decoded in registers for both
                                        projections) */
 #define MOE_FLAG_TENSOR_CORES 0x20u  /* run the persistent tensor-core kernel
-                                       (gate/up on tcgen05 block-scaled MMAs,
-                                       down on CUDA cores); needs H and I to
+                                       (gate/up on tcgen05 block-scaled MMAs;
+                                       down on them too from
+                                       MOE_TC_DOWN_MMA_MIN_TOKENS tokens of
+                                       max_tokens, else on CUDA cores; see
+                                       MOE_FLAG_TC_DOWN_*); needs H and I to
                                        be multiples of 128 and its
                                        shared-memory plan to fit, else
                                        moe_create returns MOE_ERR_UNSUPPORTED.
                                        With neither flag (and without
-                                       MOE_FLAG_SPLIT_KERNELS) moe_create
+                                       MOE_FLAG_SPLIT_KERNELS or
+                                       MOE_FLAG_SPLITK_DOWN) moe_create
                                        picks the tensor-core kernel when the
                                        shape allows it and max_tokens is at
                                        least MOE_TC_MIN_TOKENS, else the
                                        CUDA-core kernel. Both compute the same
                                        step; moe_query names the one a context
-                                       runs. Setting both flags is
+                                       runs. Setting both flags, or this one
+                                       with MOE_FLAG_SPLIT_KERNELS or
+                                       MOE_FLAG_SPLITK_DOWN, is
                                        MOE_ERR_INVALID_ARG */
 #define MOE_TC_MIN_TOKENS 4
 #define MOE_FLAG_TC_DOWN_MMA 0x40u   /* tensor-core kernel: run the down
