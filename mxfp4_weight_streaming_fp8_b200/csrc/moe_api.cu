@@ -1,7 +1,9 @@
 // moe_api.cu -- the C ABI of libmoe (declared in include/moe.h): argument
 // validation, the per-context workspace, and kernel launches on the caller's
-// stream. No allocation happens after moe_create; nothing falls back to the
-// CPU.
+// stream. moe_decode allocates nothing; moe_load_experts allocates only the
+// context's own weight copies (MOE_LOAD_COPY_REPACK, a part of an
+// intra-expert split, the split-K down projection's K-major W2). Nothing
+// falls back to the CPU.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
