@@ -46,3 +46,12 @@ def test_reference_other_ranks_print_nothing():
                 {"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"}) == []
     assert _run(["--op", "lm_head", "--steps", "1", "--warmup", "1", "--ref-rows", "256"],
                 {"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"}) == []
+
+
+def test_split_needs_one_part_per_rank():
+    """--parts under a multi-rank launch must match the number of ranks (checked
+    before any device work)."""
+    env = dict(os.environ, RANK="0", WORLD_SIZE="2", LOCAL_RANK="0")
+    res = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--parts", "3"], capture_output=True,
+                         text=True, cwd=ROOT, env=env, timeout=600)
+    assert res.returncode != 0 and "--parts must equal the number of ranks" in res.stderr
